@@ -1,0 +1,19 @@
+"""fp64 CPU oracle of the frame-wise delta-rule memory (VDA).
+
+Test infrastructure only: imported by the tests, the smoke check and the
+benchmark's CPU-baseline leg, never by the product path.
+"""
+from .vda import (  # noqa: F401
+    chunk_maps,
+    chunk_readout,
+    frame_stats,
+    frame_update,
+    is_anchor,
+    num_chunks,
+    readout_state,
+    rel_frobenius,
+    scan_states,
+    text_state,
+    transition,
+    vda_head,
+)
