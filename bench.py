@@ -1,0 +1,397 @@
+#!/usr/bin/env python
+"""Throughput of the bidirectional frame-wise delta-rule memory (VDA) on B200.
+
+One step = the whole hot path over one H3-shaped synthetic batch (B=1,
+24 heads, 102 latent frames of 1008 tokens, d=128, 512 text tokens, bf16
+inputs, fp32 state): text state, frame Grams, per-frame factor, chunk
+composition, both scans and the chunk readout, each through its C-ABI entry
+point. Prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl vdn|reference]
+
+Multi-GPU (torchrun, one rank per GPU): heads are independent, so every rank
+runs its own full H3 problem with no collective on the data path (weak
+scaling); `value` is all ranks' frames / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "VDA scan+readout frames/s (tokens/s) at H3 shape on 1 B200; % of roofline"
+FALLBACK_HBM_GBS = 6650.0
+# FP32 FMA peak: 148 SMs x 128 lanes x 2 flop x 1.965 GHz (max SM clock).
+ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+# DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum)
+# for the kernel as it stands; None until a capture of the current kernel.
+NCU_TRAFFIC = {}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["vdn", "reference"], default="vdn")
+    ap.add_argument("--workload", default="h3")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d.get("bf16_tflops", 1590.0)), "measured"
+    return FALLBACK_HBM_GBS, 1590.0, "fallback"
+
+
+# --------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.3)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------- oracle arm
+def oracle_sample(w, full, seconds: float):
+    """Run the fp64 oracle head by head until `seconds` have passed."""
+    import oracle
+    import threadpoolctl
+
+    info = threadpoolctl.threadpool_info()
+    cores = max([i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"] or [1])
+    t0 = time.perf_counter()
+    heads = 0
+    for b in range(w.B):
+        for h in range(w.H):
+            oracle.vda_head({k: full[k][b, h] for k in full}, w.chunk, w.anchors)
+            heads += 1
+            if time.perf_counter() - t0 >= seconds:
+                break
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    frames = w.B * w.T * heads / (w.B * w.H)
+    return {"value": frames / dt, "unit": "frames/s", "cores": cores, "kind": "oracle",
+            "sample": f"{heads} of {w.B * w.H} (b,h) pairs of {w.name}, all {w.T} frames x {w.U} tokens each; "
+                      f"{dt:.1f} s fp64 numpy",
+            "tokens_per_s": frames * w.U / dt}
+
+
+def run_reference(args, w):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    from frame_wise_delta_b200 import synth
+
+    full = {}
+    # one head per step: a bounded sample of the same workload
+    pairs = [(b, h) for b in range(w.B) for h in range(w.H)]
+    import oracle
+
+    def step(i):
+        b, h = pairs[i % len(pairs)]
+        if (b, h) not in full:
+            full[(b, h)] = synth.generate_head(w, b, h)
+        oracle.vda_head(full[(b, h)], w.chunk, w.anchors)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    frames = w.T * args.steps / w.H  # each step: one of H heads of one batch item
+    import threadpoolctl
+
+    cores = max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()
+                 if i.get("user_api") == "blas"] or [1])
+    value = frames / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "frames/s", "cores": cores, "kind": "oracle",
+                         "sample": f"one (b,h) pair of {w.name} per step, all {w.T} frames"},
+        "e2e": {"value": value, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    return {"workload": f"{w.name}: B={w.B} H={w.H} T={w.T} U={w.U} d_k=d_v={w.d} n_text={w.n_text} "
+                        f"chunk={w.chunk} anchors={w.anchors} {w.dtype} inputs, fp32 state",
+            "global_batch": w.B, "frames": w.B * w.T, "tokens": w.B * w.T * w.U,
+            "l2": "inputs larger than L2 (Q+K+V bf16 = %.2f GB > 126 MB)" % (3 * w.B * w.H * w.T * w.U * w.d * 2 / 1e9),
+            "parallelism": "heads independent; one full problem per rank"}
+
+
+# ---------------------------------------------------------- the CUDA arm
+def main():
+    args = parse()
+    from frame_wise_delta_b200 import synth
+
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from frame_wise_delta_b200 import build, vdn
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=__import__("datetime").timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    full = synth.generate_all(w)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    host = {}
+    for k in ("Q", "K", "V", "Kx", "Vx"):
+        host[k] = torch.from_numpy(full[k]).to(dt).pin_memory()
+    for k in ("beta", "alpha", "beta_x"):
+        host[k] = torch.from_numpy(np.ascontiguousarray(full[k])).pin_memory()
+    d = {k: v.to(dev) for k, v in host.items()}
+    s = vdn.shape_for(w)
+    B, H, T, U, D, C = w.B, w.H, w.T, w.U, w.d, w.C
+    f32 = dict(dtype=torch.float32, device=dev)
+    A = torch.empty((B, H, T, D, D), **f32)
+    Bm = torch.empty_like(A)
+    M = torch.empty_like(A)
+    J = torch.empty_like(A)
+    maps = [torch.empty((B, H, C, D, D), **f32) for _ in range(4)]
+    F = torch.empty((B, H, C + 1, D, D), **f32)
+    G = torch.empty_like(F)
+    S_T = torch.empty((B, H, D, D), **f32)
+    tws = vdn.workspace(vdn.vdn_text_state_workspace_bytes(s), dev)
+    info = torch.zeros(1, dtype=torch.int32, device=dev)
+    O = torch.empty((B, H, T, U, D), dtype=dt, device=dev)
+    stream = torch.cuda.current_stream()
+
+    stages = ["text_state", "frame_grams", "frame_factor", "chunk_compose", "scan_bidir", "chunk_readout"]
+    launches_per_step = 7  # text gram + text factor + one kernel per other stage
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        vdn.vdn_text_state(s, d["Kx"], d["Vx"], d["beta_x"], S_T, tws, info)
+        mark(1)
+        vdn.vdn_frame_grams(s, d["K"], d["V"], d["beta"], A, Bm, info)
+        mark(2)
+        vdn.vdn_frame_factor(s, A, Bm, d["alpha"], M, J, info)
+        mark(3)
+        vdn.vdn_chunk_compose(s, M, J, *maps)
+        mark(4)
+        vdn.vdn_scan_bidir(s, maps[0], maps[1], maps[2], maps[3], S_T, F, G)
+        mark(5)
+        vdn.vdn_chunk_readout(s, d["Q"], F, G, O, info)
+        mark(6)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert int(info.item()) == 0, f"device status {int(info.item())}"
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                      else local) as clk:
+        for i in range(args.steps):
+            step(evs[i])
+        torch.cuda.synchronize()
+    barrier()
+    step_ms = [e[0].elapsed_time(e[6]) for e in evs]
+    stage_ms = {name: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j, name in enumerate(stages)}
+    total_ms = evs[0][0].elapsed_time(evs[-1][6])
+    t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    frames_all = world * B * T
+    value = frames_all / (ms_per_step / 1e3)
+
+    # ---- end to end: pinned host inputs -> device -> vdn_forward -> O to host
+    fwd = vdn.Forward(s, device=dev, keep_states=False)
+    O_host = torch.empty(O.shape, dtype=dt).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = O_host.numel() * O_host.element_size()
+
+    def e2e_step():
+        for k in host:
+            d[k].copy_(host[k], non_blocking=True)
+        fwd(d["Q"], d["K"], d["V"], d["beta"], d["alpha"], d["Kx"], d["Vx"], d["beta_x"])
+        O_host.copy_(fwd.O, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(3, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    te = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = frames_all / (float(te.item()) / e2e_steps / 1e3)
+    assert int(fwd.info.item()) == 0
+
+    if rank == 0:
+        hbm_gbs, bf16_tflops, peak_src = load_peaks()
+        roof = roofline(w, stage_ms, hbm_gbs, peak_src)
+        line = {
+            "metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "state_dtype": "f32",
+            "data": "synthetic", "config": workload_config(w),
+            "tokens_per_s": value * U,
+            "hbm_frac_whole_pass": alg_bytes(w) * world / (ms_per_step / 1e3) / (hbm_gbs * 1e9),
+            "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+            "step_ms_min_max": [min(step_ms), max(step_ms)],
+            "roofline": roof,
+            "e2e": {"value": e2e_value, "unit": "frames/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = oracle_sample(w, full, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def alg_bytes(w):
+    """Algorithmic HBM bytes of the whole pass: Q, K, V read, O written (bf16),
+    text keys/values read, gates read."""
+    e = 2 if w.dtype == "bf16" else 4
+    qkvo = 4 * w.B * w.H * w.T * w.U * w.d * e
+    text = 2 * w.B * w.H * w.n_text * w.d * e
+    gates = w.B * w.H * w.T * (w.d + 1) * 4
+    return qkvo + text + gates
+
+
+def roofline(w, stage_ms, hbm_gbs, peak_src):
+    """Roofline of the dominant stage. Per-unit algorithmic figures:
+    frame_grams: per frame reads K, V (2 U d bf16) and writes A, B (2 d^2 fp32);
+    chunk_readout: per frame reads Q, writes O (2 U d bf16) plus two states per chunk;
+    frame_factor: 4 d^3 flop per non-anchor frame (Gauss-Jordan on [I+A; B]);
+    chunk_compose: 4 d^3 flop per frame after the first of each chunk and direction;
+    scan_bidir: 2 directions x C x 2 d^3 flop."""
+    B, H, T, U, d, C = w.B, w.H, w.T, w.U, w.d, w.C
+    BH = B * H
+    e = 2 if w.dtype == "bf16" else 4
+    frames = BH * T
+    live = BH * (T - (2 if w.anchors and T > 1 else (1 if w.anchors else 0)))
+    steps = sum(max(0, min(5 * c + 5, T) - 5 * c - 1) for c in range(C))
+    units = {
+        "frame_grams": ("hbm", frames * (2 * U * d * e + 2 * d * d * 4)),
+        "chunk_readout": ("hbm", frames * 2 * U * d * e + BH * C * 2 * d * d * 4),
+        "frame_factor": ("alu", live * 4 * d ** 3),
+        "chunk_compose": ("alu", BH * 2 * steps * 4 * d ** 3),
+        "scan_bidir": ("alu", BH * 2 * C * 2 * d ** 3),
+    }
+    name = max((k for k in units), key=lambda k: stage_ms.get(k, 0.0))
+    bound, amount = units[name]
+    sec = stage_ms[name] / 1e3
+    if bound == "hbm":
+        achieved = amount / sec / 1e9
+        peak, unit = hbm_gbs, "GB/s"
+        src = f"{peak_src} HBM copy bandwidth"
+    else:
+        achieved = amount / sec / 1e12
+        peak, unit = ALU_F32_TFLOPS, "TFLOP/s"
+        src = "FP32 FMA: 148 SMs x 128 lanes x 2 flop x 1.965 GHz"
+    tr = NCU_TRAFFIC.get(name)
+    return {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "traffic": tr, "peak_source": src,
+            "per_stage_ms": {k: round(v, 4) for k, v in stage_ms.items()}}
+
+
+if __name__ == "__main__":
+    main()

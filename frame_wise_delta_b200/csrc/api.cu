@@ -1,0 +1,399 @@
+// C ABI of libvdn: host-side validation and dispatch of the VDA kernels.
+// Every entry point checks its arguments before enqueuing anything, never
+// allocates, and never synchronises. See include/vdn.h for the contract.
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace vdn {
+
+void *tensor_map_encoder() {
+  static std::once_flag once;
+  static void *fn = nullptr;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = p;
+  });
+  return fn;
+}
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+    return 1;
+  return n;
+}
+
+}  // namespace vdn
+
+using namespace vdn;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+vdn_status fail(vdn_status st, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+vdn_status cuda_fail(cudaError_t e, const char *where) {
+  return fail(VDN_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+struct Geo {
+  long long BH;
+  int T, U, D, C, chunk, anchors, n_text, in_dtype, out_dtype;
+  size_t in_elem, out_elem;
+};
+
+vdn_status check_shape(const vdn_shape *s, Geo *g) {
+  if (!s) return fail(VDN_ERR_INVALID, "shape is NULL");
+  if (s->B < 0 || s->H < 0 || s->T < 0 || s->U < 0 || s->n_text < 0)
+    return fail(VDN_ERR_INVALID, "negative size (B=%d H=%d T=%d U=%d n_text=%d)", s->B, s->H, s->T,
+                s->U, s->n_text);
+  if (s->dk != s->dv) return fail(VDN_ERR_UNSUPPORTED, "dk (%d) != dv (%d)", s->dk, s->dv);
+  if (s->dk != 16 && s->dk != 32 && s->dk != 64 && s->dk != 128)
+    return fail(VDN_ERR_UNSUPPORTED, "d = %d not in {16, 32, 64, 128}", s->dk);
+  if (s->chunk < 1 || s->chunk > 16) return fail(VDN_ERR_INVALID, "chunk = %d not in [1, 16]", s->chunk);
+  if (s->anchors != 0 && s->anchors != 1) return fail(VDN_ERR_INVALID, "anchors must be 0 or 1");
+  if ((s->in_dtype != VDN_F32 && s->in_dtype != VDN_BF16) ||
+      (s->out_dtype != VDN_F32 && s->out_dtype != VDN_BF16))
+    return fail(VDN_ERR_INVALID, "dtype must be VDN_F32 or VDN_BF16");
+  g->BH = (long long)s->B * s->H;
+  g->T = s->T;
+  g->U = s->U;
+  g->D = s->dk;
+  g->chunk = s->chunk;
+  g->C = (s->T + s->chunk - 1) / s->chunk;
+  g->anchors = s->anchors;
+  g->n_text = s->n_text;
+  g->in_dtype = s->in_dtype;
+  g->out_dtype = s->out_dtype;
+  g->in_elem = s->in_dtype == VDN_BF16 ? 2 : 4;
+  g->out_elem = s->out_dtype == VDN_BF16 ? 2 : 4;
+  if (g->BH * (long long)(g->T > 0 ? g->T : 1) > 0x7fffffffLL)
+    return fail(VDN_ERR_UNSUPPORTED, "B*H*T = %lld exceeds 2^31-1", g->BH * g->T);
+  if (g->C > 65535) return fail(VDN_ERR_UNSUPPORTED, "more than 65535 chunks");
+  if ((double)g->BH * g->T * g->U * g->D > 4.0e18)
+    return fail(VDN_ERR_UNSUPPORTED, "tensor too large");
+  return VDN_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+vdn_status need(const void *p, const char *name, bool required) {
+  if (!required) return VDN_OK;
+  if (!p) return fail(VDN_ERR_INVALID, "%s is NULL", name);
+  if (!aligned16(p)) return fail(VDN_ERR_INVALID, "%s is not 16-byte aligned", name);
+  return VDN_OK;
+}
+
+#define VDN_TRY(x)                    \
+  do {                                \
+    vdn_status st_ = (x);             \
+    if (st_ != VDN_OK) return st_;    \
+  } while (0)
+
+#define VDN_CUDA(x, where)                        \
+  do {                                            \
+    cudaError_t e_ = (x);                         \
+    if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+  } while (0)
+
+size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+// ----------------------------------------------------------- stage calls
+vdn_status run_grams(const Geo &g, const void *K, const void *V, const float *beta, float *A,
+                     float *Bm, long long nframes, int U, int32_t *info, cudaStream_t st) {
+  if (nframes <= 0) return VDN_OK;
+  const size_t bytes = (size_t)nframes * g.D * g.D * sizeof(float);
+  if (U == 0) {
+    VDN_CUDA(cudaMemsetAsync(A, 0, bytes, st), "memset A");
+    VDN_CUDA(cudaMemsetAsync(Bm, 0, bytes, st), "memset Bm");
+    return VDN_OK;
+  }
+  if (gram_tc_supported(g.in_dtype, g.D, U)) {
+    VDN_CUDA(launch_gram_tc(K, V, beta, A, Bm, nframes, U, info, st), "gram_tc");
+  } else {
+    VDN_CUDA(launch_gram_simt(K, V, g.in_dtype, beta, A, Bm, nframes, U, g.D, st), "gram_simt");
+  }
+  return VDN_OK;
+}
+
+vdn_status run_readout(const Geo &g, const void *Q, const float *F, const float *G, void *O,
+                       int32_t *info, cudaStream_t st) {
+  if (g.BH * g.T * g.U == 0) return VDN_OK;
+  if (readout_tc_supported(g.in_dtype, g.out_dtype, g.D, g.U)) {
+    VDN_CUDA(launch_readout_tc(Q, F, G, O, g.BH, g.T, g.U, g.chunk, g.anchors, info, st),
+             "readout_tc");
+  } else {
+    VDN_CUDA(launch_readout_simt(Q, g.in_dtype, F, G, O, g.out_dtype, g.BH, g.T, g.U, g.chunk,
+                                 g.anchors, g.D, st),
+             "readout_simt");
+  }
+  return VDN_OK;
+}
+
+vdn_status run_text_state(const Geo &g, const void *Kx, const void *Vx, const float *beta_x,
+                          float *S_T, float *Ax, float *Bx, int32_t *info, cudaStream_t st) {
+  if (g.BH == 0) return VDN_OK;
+  if (g.n_text == 0) {
+    VDN_CUDA(cudaMemsetAsync(S_T, 0, (size_t)g.BH * g.D * g.D * sizeof(float), st), "memset S_T");
+    return VDN_OK;
+  }
+  VDN_TRY(run_grams(g, Kx, Vx, beta_x, Ax, Bx, g.BH, g.n_text, info, st));
+  VDN_CUDA(launch_factor_simt(Ax, Bx, nullptr, nullptr, S_T, info, g.BH, 1, 0, g.D, st),
+           "text factor");
+  return VDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *vdn_status_string(vdn_status st) {
+  switch (st) {
+    case VDN_OK: return "VDN_OK";
+    case VDN_ERR_INVALID: return "VDN_ERR_INVALID";
+    case VDN_ERR_UNSUPPORTED: return "VDN_ERR_UNSUPPORTED";
+    case VDN_ERR_CUDA: return "VDN_ERR_CUDA";
+    case VDN_ERR_NUMERIC: return "VDN_ERR_NUMERIC";
+  }
+  return "VDN_ERR_UNKNOWN";
+}
+
+const char *vdn_last_error(void) { return g_err; }
+
+int32_t vdn_version(void) { return 100; }
+
+vdn_status vdn_frame_grams(const vdn_shape *s, const void *K, const void *V, const float *beta,
+                           float *A, float *Bm, int32_t *info, vdn_stream_t stream) {
+  g_err[0] = 0;
+  Geo g;
+  VDN_TRY(check_shape(s, &g));
+  const bool any = g.BH * g.T > 0;
+  VDN_TRY(need(K, "K", any && g.U > 0));
+  VDN_TRY(need(V, "V", any && g.U > 0));
+  VDN_TRY(need(beta, "beta", any && g.U > 0));
+  VDN_TRY(need(A, "A", any));
+  VDN_TRY(need(Bm, "Bm", any));
+  return run_grams(g, K, V, beta, A, Bm, g.BH * g.T, g.U, info, (cudaStream_t)stream);
+}
+
+vdn_status vdn_frame_factor(const vdn_shape *s, const float *A, const float *Bm, const float *alpha,
+                            float *M, float *J, int32_t *info, vdn_stream_t stream) {
+  g_err[0] = 0;
+  Geo g;
+  VDN_TRY(check_shape(s, &g));
+  const bool any = g.BH * g.T > 0;
+  VDN_TRY(need(A, "A", any));
+  VDN_TRY(need(Bm, "Bm", any));
+  VDN_TRY(need(alpha, "alpha", any));
+  VDN_TRY(need(M, "M", any));
+  VDN_TRY(need(J, "J", any));
+  VDN_TRY(need(info, "info", true));
+  cudaStream_t st = (cudaStream_t)stream;
+  VDN_CUDA(cudaMemsetAsync(info, 0, sizeof(int32_t), st), "memset info");
+  VDN_CUDA(launch_factor_simt(A, Bm, alpha, M, J, info, g.BH * g.T, g.T, g.anchors, g.D, st),
+           "factor");
+  return VDN_OK;
+}
+
+vdn_status vdn_chunk_compose(const vdn_shape *s, const float *M, const float *J, float *Mf,
+                             float *Jf, float *Mb, float *Jb, vdn_stream_t stream) {
+  g_err[0] = 0;
+  Geo g;
+  VDN_TRY(check_shape(s, &g));
+  const bool any = g.BH * g.T > 0;
+  VDN_TRY(need(M, "M", any));
+  VDN_TRY(need(J, "J", any));
+  VDN_TRY(need(Mf, "Mf", any));
+  VDN_TRY(need(Jf, "Jf", any));
+  VDN_TRY(need(Mb, "Mb", any));
+  VDN_TRY(need(Jb, "Jb", any));
+  VDN_CUDA(launch_compose_simt(M, J, Mf, Jf, Mb, Jb, g.BH, g.T, g.chunk, g.D, (cudaStream_t)stream),
+           "compose");
+  return VDN_OK;
+}
+
+static vdn_status scan_common(const vdn_shape *s, const float *Mf, const float *Jf, const float *Mb,
+                              const float *Jb, const float *S_T, float *F, float *G, int mask,
+                              vdn_stream_t stream) {
+  g_err[0] = 0;
+  Geo g;
+  VDN_TRY(check_shape(s, &g));
+  const bool any = g.BH > 0;
+  const bool fw = mask & 1, bw = mask & 2;
+  VDN_TRY(need(S_T, "S_T", any));
+  VDN_TRY(need(Mf, "Mf", any && fw && g.C > 0));
+  VDN_TRY(need(Jf, "Jf", any && fw && g.C > 0));
+  VDN_TRY(need(F, "F", any && fw));
+  VDN_TRY(need(Mb, "Mb", any && bw && g.C > 0));
+  VDN_TRY(need(Jb, "Jb", any && bw && g.C > 0));
+  VDN_TRY(need(G, "G", any && bw));
+  VDN_CUDA(launch_scan_simt(Mf, Jf, Mb, Jb, S_T, F, G, g.BH, g.C, g.D, mask, (cudaStream_t)stream),
+           "scan");
+  return VDN_OK;
+}
+
+vdn_status vdn_scan_fwd(const vdn_shape *s, const float *Mf, const float *Jf, const float *S_T,
+                        float *F, vdn_stream_t stream) {
+  return scan_common(s, Mf, Jf, nullptr, nullptr, S_T, F, nullptr, 1, stream);
+}
+
+vdn_status vdn_scan_bwd(const vdn_shape *s, const float *Mb, const float *Jb, const float *S_T,
+                        float *G, vdn_stream_t stream) {
+  return scan_common(s, nullptr, nullptr, Mb, Jb, S_T, nullptr, G, 2, stream);
+}
+
+vdn_status vdn_scan_bidir(const vdn_shape *s, const float *Mf, const float *Jf, const float *Mb,
+                          const float *Jb, const float *S_T, float *F, float *G,
+                          vdn_stream_t stream) {
+  return scan_common(s, Mf, Jf, Mb, Jb, S_T, F, G, 3, stream);
+}
+
+vdn_status vdn_chunk_readout(const vdn_shape *s, const void *Q, const float *F, const float *G,
+                             void *O, int32_t *info, vdn_stream_t stream) {
+  g_err[0] = 0;
+  Geo g;
+  VDN_TRY(check_shape(s, &g));
+  const bool any = g.BH * g.T * g.U > 0;
+  VDN_TRY(need(Q, "Q", any));
+  VDN_TRY(need(F, "F", any));
+  VDN_TRY(need(G, "G", any));
+  VDN_TRY(need(O, "O", any));
+  return run_readout(g, Q, F, G, O, info, (cudaStream_t)stream);
+}
+
+size_t vdn_text_state_workspace_bytes(const vdn_shape *s) {
+  Geo g;
+  if (check_shape(s, &g) != VDN_OK) return 0;
+  return 2 * align256((size_t)g.BH * g.D * g.D * sizeof(float));
+}
+
+vdn_status vdn_text_state(const vdn_shape *s, const void *Kx, const void *Vx, const float *beta_x,
+                          float *S_T, void *workspace, size_t workspace_bytes, int32_t *info,
+                          vdn_stream_t stream) {
+  g_err[0] = 0;
+  Geo g;
+  VDN_TRY(check_shape(s, &g));
+  const bool any = g.BH > 0;
+  VDN_TRY(need(Kx, "Kx", any && g.n_text > 0));
+  VDN_TRY(need(Vx, "Vx", any && g.n_text > 0));
+  VDN_TRY(need(beta_x, "beta_x", any && g.n_text > 0));
+  VDN_TRY(need(S_T, "S_T", any));
+  VDN_TRY(need(info, "info", true));
+  const size_t ws = vdn_text_state_workspace_bytes(s);
+  VDN_TRY(need(workspace, "workspace", any && ws > 0));
+  if (workspace_bytes < ws)
+    return fail(VDN_ERR_INVALID, "workspace of %zu bytes < %zu required", workspace_bytes, ws);
+  cudaStream_t st = (cudaStream_t)stream;
+  VDN_CUDA(cudaMemsetAsync(info, 0, sizeof(int32_t), st), "memset info");
+  float *Ax = (float *)workspace;
+  float *Bx = (float *)((char *)workspace + align256((size_t)g.BH * g.D * g.D * sizeof(float)));
+  return run_text_state(g, Kx, Vx, beta_x, S_T, Ax, Bx, info, st);
+}
+
+namespace {
+struct FwdLayout {
+  size_t ax, bx, st, a, b, mf, jf, mb, jb, f, g, total;
+};
+FwdLayout fwd_layout(const Geo &g) {
+  FwdLayout L{};
+  const size_t dd = (size_t)g.D * g.D * sizeof(float);
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    size_t o = off;
+    off += align256(n);
+    return o;
+  };
+  L.ax = take(g.BH * dd);
+  L.bx = take(g.BH * dd);
+  L.st = take(g.BH * dd);
+  L.a = take(g.BH * g.T * dd);
+  L.b = take(g.BH * g.T * dd);
+  L.mf = take(g.BH * g.C * dd);
+  L.jf = take(g.BH * g.C * dd);
+  L.mb = take(g.BH * g.C * dd);
+  L.jb = take(g.BH * g.C * dd);
+  L.f = take(g.BH * (g.C + 1) * dd);
+  L.g = take(g.BH * (g.C + 1) * dd);
+  L.total = off;
+  return L;
+}
+}  // namespace
+
+size_t vdn_forward_workspace_bytes(const vdn_shape *s) {
+  Geo g;
+  if (check_shape(s, &g) != VDN_OK) return 0;
+  return fwd_layout(g).total;
+}
+
+vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K, const void *V,
+                       const float *beta, const float *alpha, const void *Kx, const void *Vx,
+                       const float *beta_x, void *O, float *F, float *G, void *workspace,
+                       size_t workspace_bytes, int32_t *info, vdn_stream_t stream) {
+  g_err[0] = 0;
+  Geo g;
+  VDN_TRY(check_shape(s, &g));
+  const bool frames = g.BH * g.T > 0;
+  VDN_TRY(need(Q, "Q", frames && g.U > 0));
+  VDN_TRY(need(K, "K", frames && g.U > 0));
+  VDN_TRY(need(V, "V", frames && g.U > 0));
+  VDN_TRY(need(beta, "beta", frames && g.U > 0));
+  VDN_TRY(need(alpha, "alpha", frames));
+  VDN_TRY(need(Kx, "Kx", g.BH > 0 && g.n_text > 0));
+  VDN_TRY(need(Vx, "Vx", g.BH > 0 && g.n_text > 0));
+  VDN_TRY(need(beta_x, "beta_x", g.BH > 0 && g.n_text > 0));
+  VDN_TRY(need(O, "O", frames && g.U > 0));
+  VDN_TRY(need(F, "F", false));
+  VDN_TRY(need(G, "G", false));
+  if ((F && !aligned16(F)) || (G && !aligned16(G)))
+    return fail(VDN_ERR_INVALID, "F/G not 16-byte aligned");
+  VDN_TRY(need(info, "info", true));
+  const FwdLayout L = fwd_layout(g);
+  VDN_TRY(need(workspace, "workspace", g.BH > 0));
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(VDN_ERR_INVALID, "workspace is not 256-byte aligned");
+  if (workspace_bytes < L.total)
+    return fail(VDN_ERR_INVALID, "workspace of %zu bytes < %zu required", workspace_bytes, L.total);
+  if (g.BH == 0) return VDN_OK;
+
+  cudaStream_t st = (cudaStream_t)stream;
+  char *w = (char *)workspace;
+  float *Ax = (float *)(w + L.ax), *Bx = (float *)(w + L.bx), *S_T = (float *)(w + L.st);
+  float *A = (float *)(w + L.a), *Bm = (float *)(w + L.b);
+  float *Mf = (float *)(w + L.mf), *Jf = (float *)(w + L.jf);
+  float *Mb = (float *)(w + L.mb), *Jb = (float *)(w + L.jb);
+  float *Fo = F ? F : (float *)(w + L.f);
+  float *Go = G ? G : (float *)(w + L.g);
+
+  VDN_CUDA(cudaMemsetAsync(info, 0, sizeof(int32_t), st), "memset info");
+  VDN_TRY(run_text_state(g, Kx, Vx, beta_x, S_T, Ax, Bx, info, st));
+  if (frames) {
+    VDN_TRY(run_grams(g, K, V, beta, A, Bm, g.BH * g.T, g.U, info, st));
+    // M and J overwrite A and Bm in place (each element is read and written
+    // by the same thread).
+    VDN_CUDA(launch_factor_simt(A, Bm, alpha, A, Bm, info, g.BH * g.T, g.T, g.anchors, g.D, st),
+             "factor");
+    VDN_CUDA(launch_compose_simt(A, Bm, Mf, Jf, Mb, Jb, g.BH, g.T, g.chunk, g.D, st), "compose");
+  }
+  VDN_CUDA(launch_scan_simt(Mf, Jf, Mb, Jb, S_T, Fo, Go, g.BH, g.C, g.D, 3, st), "scan");
+  if (frames) VDN_TRY(run_readout(g, Q, Fo, Go, O, info, st));
+  return VDN_OK;
+}
+
+}  // extern "C"

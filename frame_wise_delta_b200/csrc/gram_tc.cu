@@ -1,0 +1,246 @@
+// Frame statistics on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+// Paper: "Video DeltaNet: A Video-Native Hybrid Attention for Livestream
+// Video Generation" (summary page), "Method steps" step (3):
+//   A_t = beta_t K_t^T K_t,   B_t = beta_t V_t^T K_t   (bf16 in, fp32 out, d = 128).
+//
+// One MMA stream per frame computes D = K^T [K | V] (M = 128, N = 256,
+// contraction over the frame's U tokens): columns 0..127 of D are A_t and
+// columns 128..255 are B_t^T. Both operands come straight from the TMA
+// tiles: a tile of 64 tokens x 128 channels is stored as 64-channel blocks,
+// 128-byte swizzled, which is the MN-major canonical layout (token = K
+// index, channel = M/N index). K-block stride 1024 B per 8 tokens, M/N-block
+// stride 8 KB.
+//
+// Persistent kernel, one CTA per SM, 6 warps:
+//   warp 0     : TMA producer (4 loads of 8 KB per 64-token stage)
+//   warp 1     : TMEM allocator and single-thread MMA issuer
+//   warps 2..5 : epilogue: TMEM -> registers -> scaled fp32 stores
+// TMEM holds two 256-column accumulators so a frame's epilogue overlaps the
+// next frame's MMAs. Every wait is bounded (see common.cuh).
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace vdn {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kUT = 64;                          // tokens per pipeline stage
+constexpr int kStages = 4;
+constexpr int kStageBytes = 4 * kUT * 128;       // K lo, K hi, V lo, V hi blocks
+constexpr int kBlockBytes = kUT * 128;           // one 64-channel block
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kBarBytes = 8 * (2 * kStages + 2 + 2 + 1);
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + kBarBytes + 16;
+
+struct GramArgs {
+  float *A;
+  float *Bm;
+  const float *beta;
+  int32_t *info;
+  long long nframes;
+  int ntiles;
+};
+
+__device__ __forceinline__ void fail(volatile int *abort, int32_t *info) {
+  *abort = 1;
+  if (info) atomicExch(info, VDN_INFO_TIMEOUT);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gram_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                   GramArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  uint8_t *stages = smem;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kStages * kStageBytes + kBarBytes);
+  volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = full0 + 8 * kStages;
+  const uint32_t tfull0 = empty0 + 8 * kStages;
+  const uint32_t tempty0 = tfull0 + 16;
+  const uint32_t drain = tempty0 + 16;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, 128);
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      int stage = 0;
+      uint32_t phase = 0;
+      int armed_parity[kStages];
+      for (int s = 0; s < kStages; ++s) armed_parity[s] = -1;
+      bool ok = true;
+      for (long long f = blockIdx.x; ok && f < p.nframes; f += gridDim.x) {
+        for (int j = 0; j < p.ntiles; ++j) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, abort)) {
+            fail(abort, p.info);
+            ok = false;
+            break;
+          }
+          const uint32_t dst = smem_u32(stages + stage * kStageBytes);
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_arrive_expect_tx(fb, kStageBytes);
+          armed_parity[stage] = (int)phase;
+          const int y = j * kUT, z = (int)f;
+          tma_load_3d(dst + 0 * kBlockBytes, &tmK, fb, 0, y, z);
+          tma_load_3d(dst + 1 * kBlockBytes, &tmK, fb, 64, y, z);
+          tma_load_3d(dst + 2 * kBlockBytes, &tmV, fb, 0, y, z);
+          tma_load_3d(dst + 3 * kBlockBytes, &tmV, fb, 64, y, z);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // Never leave with copies in flight: wait (bounded) for the last
+      // arming of every stage to land.
+      volatile int never = 0;
+      for (int s = 0; s < kStages; ++s)
+        if (armed_parity[s] >= 0) mbar_wait(full0 + 8 * s, (uint32_t)armed_parity[s], &never);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 256, true, true);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (long long f = blockIdx.x; ok && f < p.nframes; f += gridDim.x, ++it) {
+        const int buf = it & 1;
+        const uint32_t use = (uint32_t)(it >> 1);
+        if (!mbar_wait(tempty0 + 8 * buf, (use & 1) ^ 1, abort)) {
+          fail(abort, p.info);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dcol = tmem_base + (uint32_t)(buf * 256);
+        for (int j = 0; j < p.ntiles; ++j) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort)) {
+            fail(abort, p.info);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t base = smem_u32(stages + stage * kStageBytes);
+#pragma unroll
+          for (int ks = 0; ks < kUT / 16; ++ks) {
+            const uint64_t desc = smem_desc_sw128(base + ks * 2048, kBlockBytes, 1024);
+            tc_mma_bf16(dcol, desc, desc, idesc, (j > 0 || ks > 0) ? 1u : 0u);
+          }
+          tc_commit(empty0 + 8 * stage);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) tc_commit(tfull0 + 8 * buf);
+      }
+      // Let every issued MMA finish before TMEM is released.
+      tc_commit(drain);
+      volatile int never = 0;
+      mbar_wait(drain, 0, &never);
+    }
+  } else {
+    // epilogue warps 2..5 -> TMEM sub-partitions 2, 3, 0, 1
+    const int sub = warp & 3;
+    const int row = sub * 32 + lane;
+    int it = 0;
+    for (long long f = blockIdx.x; f < p.nframes; f += gridDim.x, ++it) {
+      const int buf = it & 1;
+      const uint32_t use = (uint32_t)(it >> 1);
+      // every lane waits (acquire); the warp then agrees on the outcome so
+      // that it enters the aligned TMEM loads together or not at all
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * buf, use & 1, abort));
+      if (!ok) {
+        fail(abort, p.info);
+        break;
+      }
+      tc_fence_after();
+      const float bt = p.beta[f];
+      float *Af = p.A + f * (long long)(kD * kD);
+      float *Bf = p.Bm + f * (long long)(kD * kD);
+#pragma unroll 1
+      for (int cc = 0; cc < 8; ++cc) {
+        float v[32];
+        tmem_ld32(tmem_base + (uint32_t)(buf * 256 + cc * 32) + ((uint32_t)(sub * 32) << 16), v);
+        // D[row][n]: n < 128 -> A[row][n] = A[n][row] (symmetric; written by
+        // column so that a warp stores 32 consecutive floats); n >= 128 ->
+        // B[n-128][row].
+        float *dst = (cc < 4 ? Af + (cc * 32) * kD : Bf + ((cc - 4) * 32) * kD) + row;
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) dst[jj * kD] = bt * v[jj];
+      }
+      tc_fence_before();
+      mbar_arrive(tempty0 + 8 * buf);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace
+
+bool gram_tc_supported(int in_dtype, int D, int U) { return in_dtype == VDN_BF16 && D == 128 && U > 0; }
+
+// 3-D tensor map over [frames][rows][128] bf16 with a (64 ch x box_rows x 1) box.
+bool make_rows_map(CUtensorMap *m, const void *base, long long frames, int rows, int box_rows) {
+  auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
+  if (!enc) return false;
+  cuuint64_t dims[3] = {128, (cuuint64_t)rows, (cuuint64_t)frames};
+  cuuint64_t strides[2] = {128 * 2, (cuuint64_t)rows * 128 * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+cudaError_t launch_gram_tc(const void *K, const void *V, const float *beta, float *A, float *Bm,
+                           long long nframes, int U, int32_t *info, cudaStream_t st) {
+  if (nframes <= 0) return cudaSuccess;
+  CUtensorMap tmK, tmV;
+  if (!make_rows_map(&tmK, K, nframes, U, kUT) || !make_rows_map(&tmV, V, nframes, U, kUT))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int sms = device_sm_count();
+  const long long grid = nframes < sms ? nframes : sms;
+  GramArgs a{A, Bm, beta, info, nframes, (U + kUT - 1) / kUT};
+  gram_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(tmK, tmV, a);
+  return cudaGetLastError();
+}
+
+}  // namespace vdn

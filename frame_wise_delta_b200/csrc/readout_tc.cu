@@ -1,0 +1,320 @@
+// Chunk readout on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+// Paper: "Video DeltaNet: A Video-Native Hybrid Attention for Livestream
+// Video Generation" (summary page), "Core method" (each query chunk reads the
+// forward state before its 15-frame window plus the backward state after it)
+// and "Method steps" step (5):
+//   R_c = F[max(c-1,0)] + G[min(c+2,C)],   o_{t,u} = R_c q_{t,u}.
+//
+// D = R Q_tile^T with M = 128 (value channel i), N = 128 tokens, K = 128 key
+// channels. The fp32 state R is split into bf16 hi + lo parts (R = hi + lo to
+// ~2^-17 relative) and both products accumulate into one fp32 TMEM tile, so
+// the readout keeps fp32-state accuracy while Q is read once, as bf16.
+// Operands are K-major and 128-byte swizzled: Q tiles come from TMA, R is
+// written by the CTA into the same layout.
+//
+// Persistent kernel, one CTA per SM, 6 warps; each CTA walks a contiguous
+// range of frames so consecutive frames usually share a chunk and R is
+// rebuilt only when the chunk changes.
+//   warp 0     : TMA producer (two 16 KB loads per 128-token stage)
+//   warp 1     : TMEM allocator and single-thread MMA issuer
+//   warps 2..5 : R builder and epilogue (TMEM -> bf16 stores; anchor frames
+//                are written as zeros without touching the tensor cores)
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace vdn {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kNT = 128;                      // tokens per tile (MMA N)
+constexpr int kStages = 4;
+constexpr int kStageBytes = kNT * 128 * 2;    // two 64-channel regions
+constexpr int kRegionQ = kNT * 128;           // 16 KB
+constexpr int kRBytes = kD * 128 * 2;         // one bf16 R operand, 2 regions
+constexpr int kRegionR = kD * 128;
+constexpr int kAcc = 4;                       // TMEM accumulators (128 columns each)
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kBarBytes = 8 * (2 * kStages + 2 * kAcc + 2);
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 2 * kRBytes + kBarBytes + 16;
+
+struct ReadoutArgs {
+  const float *F;
+  const float *G;
+  __nv_bfloat16 *O;
+  int32_t *info;
+  long long nframes;
+  int T, U, chunk, anchors, C, ntiles;
+};
+
+__device__ __forceinline__ void fail(volatile int *abort, int32_t *info) {
+  *abort = 1;
+  if (info) atomicExch(info, VDN_INFO_TIMEOUT);
+}
+
+__device__ __forceinline__ bool is_anchor(const ReadoutArgs &p, long long f) {
+  const int t = (int)(f % p.T);
+  return p.anchors && (t == 0 || t == p.T - 1);
+}
+
+__device__ __forceinline__ long long chunk_key(const ReadoutArgs &p, long long f) {
+  return (f / p.T) * p.C + (f % p.T) / p.chunk;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(a));
+  const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(b));
+  return lo | (hi << 16);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    readout_tc_kernel(const __grid_constant__ CUtensorMap tmQ, ReadoutArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  uint8_t *stages = smem;
+  uint8_t *Rhi = smem + kStages * kStageBytes;
+  uint8_t *Rlo = Rhi + kRBytes;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(Rlo + kRBytes);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(bars) + kBarBytes);
+  volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = full0 + 8 * kStages;
+  const uint32_t tfull0 = empty0 + 8 * kStages;
+  const uint32_t tempty0 = tfull0 + 8 * kAcc;
+  const uint32_t rfull = tempty0 + 8 * kAcc;
+  const uint32_t drain = rfull + 8;
+
+  // contiguous, balanced frame range of this CTA
+  const long long f_begin = p.nframes * blockIdx.x / gridDim.x;
+  const long long f_end = p.nframes * (blockIdx.x + 1) / gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < kAcc; ++b) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, 128);
+    }
+    mbar_init(rfull, 1);
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      int stage = 0;
+      uint32_t phase = 0;
+      int armed_parity[kStages];
+      for (int s = 0; s < kStages; ++s) armed_parity[s] = -1;
+      bool ok = true;
+      for (long long f = f_begin; ok && f < f_end; ++f) {
+        if (is_anchor(p, f)) continue;
+        for (int j = 0; j < p.ntiles; ++j) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, abort)) {
+            fail(abort, p.info);
+            ok = false;
+            break;
+          }
+          const uint32_t dst = smem_u32(stages + stage * kStageBytes);
+          const uint32_t fb = full0 + 8 * stage;
+          mbar_arrive_expect_tx(fb, kStageBytes);
+          armed_parity[stage] = (int)phase;
+          tma_load_3d(dst, &tmQ, fb, 0, j * kNT, (int)f);
+          tma_load_3d(dst + kRegionQ, &tmQ, fb, 64, j * kNT, (int)f);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      volatile int never = 0;
+      for (int s = 0; s < kStages; ++s)
+        if (armed_parity[s] >= 0) mbar_wait(full0 + 8 * s, (uint32_t)armed_parity[s], &never);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, kNT, false, false);
+      const uint32_t rhi = smem_u32(Rhi), rlo = smem_u32(Rlo);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t tile = 0;
+      uint32_t rbuilds = 0;
+      long long cur = -1;
+      bool ok = true;
+      for (long long f = f_begin; ok && f < f_end; ++f) {
+        if (is_anchor(p, f)) continue;
+        const long long key = chunk_key(p, f);
+        if (key != cur) {
+          if (!mbar_wait(rfull, rbuilds & 1, abort)) {
+            fail(abort, p.info);
+            break;
+          }
+          ++rbuilds;
+          cur = key;
+          tc_fence_after();
+        }
+        for (int j = 0; j < p.ntiles; ++j, ++tile) {
+          const int buf = (int)(tile % kAcc);
+          const uint32_t use = tile / kAcc;
+          if (!mbar_wait(tempty0 + 8 * buf, (use & 1) ^ 1, abort) ||
+              !mbar_wait(full0 + 8 * stage, phase, abort)) {
+            fail(abort, p.info);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t q = smem_u32(stages + stage * kStageBytes);
+          const uint32_t dcol = tmem_base + (uint32_t)(buf * kNT);
+#pragma unroll
+          for (int part = 0; part < 2; ++part) {
+            const uint32_t r = part == 0 ? rhi : rlo;
+#pragma unroll
+            for (int ks = 0; ks < kD / 16; ++ks) {
+              const uint32_t koff = (uint32_t)(ks & 3) * 32;  // 16 bf16 = 32 B inside the swizzle atom
+              const uint64_t adesc = smem_desc_sw128(r + (ks >> 2) * kRegionR + koff, 16, 1024);
+              const uint64_t bdesc = smem_desc_sw128(q + (ks >> 2) * kRegionQ + koff, 16, 1024);
+              tc_mma_bf16(dcol, adesc, bdesc, idesc, (part > 0 || ks > 0) ? 1u : 0u);
+            }
+          }
+          tc_commit(empty0 + 8 * stage);
+          tc_commit(tfull0 + 8 * buf);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      tc_commit(drain);
+      volatile int never = 0;
+      mbar_wait(drain, 0, &never);
+    }
+  } else {
+    const int et = threadIdx.x - 64;  // 0..127
+    const int sub = warp & 3;
+    const int row = sub * 32 + lane;  // value channel i held by this thread
+    uint32_t tile = 0;
+    long long cur = -1;
+    for (long long f = f_begin; f < f_end; ++f) {
+      __nv_bfloat16 *Of = p.O + f * (long long)p.U * kD;
+      if (is_anchor(p, f)) {
+        uint4 z = make_uint4(0, 0, 0, 0);
+        uint4 *o4 = reinterpret_cast<uint4 *>(Of);
+        const long long n16 = (long long)p.U * kD / 8;
+        for (long long e = et; e < n16; e += 128) o4[e] = z;
+        continue;
+      }
+      const long long key = chunk_key(p, f);
+      if (key != cur) {
+        // All MMAs that read the previous R have completed: every one of
+        // their tiles was drained below before we got here.
+        cur = key;
+        const long long bh = f / p.T;
+        const int c = (int)((f % p.T) / p.chunk);
+        const float *Fs = p.F + (bh * (p.C + 1) + max(c - 1, 0)) * (long long)(kD * kD);
+        const float *Gs = p.G + (bh * (p.C + 1) + min(c + 2, p.C)) * (long long)(kD * kD);
+        for (int e8 = et; e8 < kD * kD / 8; e8 += 128) {
+          const int i = e8 >> 4, k0 = (e8 & 15) * 8;
+          const float4 *f4 = reinterpret_cast<const float4 *>(Fs + i * kD + k0);
+          const float4 *g4 = reinterpret_cast<const float4 *>(Gs + i * kD + k0);
+          const float4 a0 = f4[0], a1 = f4[1], b0 = g4[0], b1 = g4[1];
+          const float r[8] = {a0.x + b0.x, a0.y + b0.y, a0.z + b0.z, a0.w + b0.w,
+                              a1.x + b1.x, a1.y + b1.y, a1.z + b1.z, a1.w + b1.w};
+          float h[8], l[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            h[q] = __bfloat162float(__float2bfloat16_rn(r[q]));
+            l[q] = r[q] - h[q];
+          }
+          const uint32_t off = kmajor_sw128_offset(i, k0, kD);
+          *reinterpret_cast<uint4 *>(Rhi + off) =
+              make_uint4(pack_bf16(h[0], h[1]), pack_bf16(h[2], h[3]), pack_bf16(h[4], h[5]),
+                         pack_bf16(h[6], h[7]));
+          *reinterpret_cast<uint4 *>(Rlo + off) =
+              make_uint4(pack_bf16(l[0], l[1]), pack_bf16(l[2], l[3]), pack_bf16(l[4], l[5]),
+                         pack_bf16(l[6], l[7]));
+        }
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (et == 0) mbar_arrive(rfull);
+      }
+      bool ok = true;
+      for (int j = 0; j < p.ntiles; ++j, ++tile) {
+        const int buf = (int)(tile % kAcc);
+        const uint32_t use = tile / kAcc;
+        if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * buf, use & 1, abort))) {
+          fail(abort, p.info);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int cc = 0; cc < kNT / 32; ++cc) {
+          float v[32];
+          tmem_ld32(tmem_base + (uint32_t)(buf * kNT + cc * 32) + ((uint32_t)(sub * 32) << 16), v);
+          const int u0 = j * kNT + cc * 32;
+          __nv_bfloat16 *dst = Of + (long long)u0 * kD + row;
+          if (u0 + 32 <= p.U) {
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) dst[jj * kD] = __float2bfloat16_rn(v[jj]);
+          } else {
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj)
+              if (u0 + jj < p.U) dst[jj * kD] = __float2bfloat16_rn(v[jj]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(tempty0 + 8 * buf);
+      }
+      if (!ok) break;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace
+
+bool make_rows_map(CUtensorMap *m, const void *base, long long frames, int rows, int box_rows);
+
+bool readout_tc_supported(int in_dtype, int out_dtype, int D, int U) {
+  return in_dtype == VDN_BF16 && out_dtype == VDN_BF16 && D == 128 && U > 0;
+}
+
+cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, void *O, long long BH,
+                              int T, int U, int chunk, int anchors, int32_t *info, cudaStream_t st) {
+  const long long nframes = BH * T;
+  if (nframes <= 0) return cudaSuccess;
+  CUtensorMap tmQ;
+  if (!make_rows_map(&tmQ, Q, nframes, U, kNT)) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(readout_tc_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int sms = device_sm_count();
+  const long long grid = nframes < sms ? nframes : sms;
+  ReadoutArgs a{F, G, (__nv_bfloat16 *)O, info, nframes, T, U, chunk, anchors,
+                (T + chunk - 1) / chunk, (U + kNT - 1) / kNT};
+  readout_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(tmQ, a);
+  return cudaGetLastError();
+}
+
+}  // namespace vdn

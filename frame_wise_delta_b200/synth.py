@@ -133,24 +133,30 @@ def _keys(w: Workload, b: int, h: int, rows: tuple) -> np.ndarray:
     return _unit_rows(base + sigma * g)
 
 
-def generate_head(w: Workload, b: int, h: int) -> dict:
-    """All inputs of one (b, h) pair as float32 numpy arrays.
+ALL_PARTS = ("Q", "K", "V", "Kx", "Vx", "beta", "alpha", "beta_x")
+
+
+def generate_head(w: Workload, b: int, h: int, parts=ALL_PARTS) -> dict:
+    """Inputs of one (b, h) pair as float32 numpy arrays.
 
     Q, K, V: [T, U, d]; Kx, Vx: [n_text, d]; beta: [T]; alpha: [T, d];
     beta_x: float. For bf16 workloads Q/K/V/Kx/Vx hold bf16-representable
-    values (rounded to nearest even), which both sides read.
+    values (rounded to nearest even), which both sides read. `parts` selects
+    a subset; every tensor has its own stream, so a subset is drawn exactly as
+    it is in the full set.
     """
     T, U, d = w.T, w.U, w.d
-    out = {}
-    out["Q"] = _store(w, _rng(w, b, h, "Q").standard_normal((T, U, d), dtype=np.float32))
-    out["K"] = _store(w, _keys(w, b, h, (T, U)))
-    out["V"] = _store(w, _rng(w, b, h, "V").standard_normal((T, U, d), dtype=np.float32))
-    out["Kx"] = _store(w, _unit_rows(_rng(w, b, h, "Kx").standard_normal((w.n_text, d), dtype=np.float32)))
-    out["Vx"] = _store(w, _rng(w, b, h, "Vx").standard_normal((w.n_text, d), dtype=np.float32))
-    out["beta"] = _rng(w, b, h, "beta").uniform(w.beta_lo, 1.0, size=T).astype(np.float32)
-    out["alpha"] = _rng(w, b, h, "alpha").uniform(w.alpha_lo, 1.0, size=(T, d)).astype(np.float32)
-    out["beta_x"] = np.float32(1.0)
-    return out
+    make = {
+        "Q": lambda: _store(w, _rng(w, b, h, "Q").standard_normal((T, U, d), dtype=np.float32)),
+        "K": lambda: _store(w, _keys(w, b, h, (T, U))),
+        "V": lambda: _store(w, _rng(w, b, h, "V").standard_normal((T, U, d), dtype=np.float32)),
+        "Kx": lambda: _store(w, _unit_rows(_rng(w, b, h, "Kx").standard_normal((w.n_text, d), dtype=np.float32))),
+        "Vx": lambda: _store(w, _rng(w, b, h, "Vx").standard_normal((w.n_text, d), dtype=np.float32)),
+        "beta": lambda: _rng(w, b, h, "beta").uniform(w.beta_lo, 1.0, size=T).astype(np.float32),
+        "alpha": lambda: _rng(w, b, h, "alpha").uniform(w.alpha_lo, 1.0, size=(T, d)).astype(np.float32),
+        "beta_x": lambda: np.float32(1.0),
+    }
+    return {k: make[k]() for k in parts}
 
 
 def generate_all(w: Workload, threads: int = 8) -> dict:

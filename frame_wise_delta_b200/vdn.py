@@ -1,0 +1,229 @@
+"""Python binding of libvdn (ctypes; argument marshalling only).
+
+Every function has the name of its C entry point in include/vdn.h, takes
+torch CUDA tensors (or None where the C call accepts NULL), passes their
+device pointers and the current torch stream, and raises VdnError on any
+status other than VDN_OK. All arithmetic happens in the library's kernels;
+there is no fallback: if libvdn.so is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libvdn.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "vdn.h")
+
+VDN_OK, VDN_ERR_INVALID, VDN_ERR_UNSUPPORTED, VDN_ERR_CUDA, VDN_ERR_NUMERIC = range(5)
+VDN_F32, VDN_BF16 = 0, 1
+VDN_INFO_TIMEOUT = -1
+_DTYPES = {"f32": VDN_F32, "bf16": VDN_BF16, VDN_F32: VDN_F32, VDN_BF16: VDN_BF16}
+TORCH_DTYPE = {VDN_F32: torch.float32, VDN_BF16: torch.bfloat16}
+
+
+class VdnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+class vdn_shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("B", "H", "T", "U", "dk", "dv", "n_text", "chunk", "anchors", "in_dtype", "out_dtype")]
+
+    @property
+    def C(self) -> int:
+        return -(-self.T // self.chunk) if self.T > 0 else 0
+
+
+def make_shape(B, H, T, U, d, n_text, chunk=5, anchors=0, in_dtype="bf16", out_dtype=None) -> vdn_shape:
+    in_dt = _DTYPES[in_dtype]
+    out_dt = in_dt if out_dtype is None else _DTYPES[out_dtype]
+    return vdn_shape(B, H, T, U, d, d, n_text, chunk, anchors, in_dt, out_dt)
+
+
+def shape_for(w, B=None, H=None) -> vdn_shape:
+    """Shape of a synth.Workload (optionally with other batch/head counts)."""
+    return make_shape(w.B if B is None else B, w.H if H is None else H, w.T, w.U, w.d, w.n_text,
+                      w.chunk, w.anchors, w.dtype)
+
+
+_lib = None
+
+_P = ctypes.c_void_p
+_SIGS = {
+    "vdn_frame_grams": [_P, _P, _P, _P, _P, _P, _P, _P],
+    "vdn_frame_factor": [_P, _P, _P, _P, _P, _P, _P, _P],
+    "vdn_chunk_compose": [_P, _P, _P, _P, _P, _P, _P, _P],
+    "vdn_scan_fwd": [_P, _P, _P, _P, _P, _P],
+    "vdn_scan_bwd": [_P, _P, _P, _P, _P, _P],
+    "vdn_scan_bidir": [_P, _P, _P, _P, _P, _P, _P, _P, _P],
+    "vdn_chunk_readout": [_P, _P, _P, _P, _P, _P, _P],
+    "vdn_text_state": [_P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P],
+    "vdn_forward": [_P] * 13 + [ctypes.c_size_t, _P, _P],
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libvdn.so (built in-tree by frame_wise_delta_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise VdnError(VDN_ERR_CUDA, f"{LIB_PATH} is missing; build it with "
+                                         "`python -m frame_wise_delta_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, args in _SIGS.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        for name in ("vdn_text_state_workspace_bytes", "vdn_forward_workspace_bytes"):
+            fn = getattr(L, name)
+            fn.argtypes = [_P]
+            fn.restype = ctypes.c_size_t
+        L.vdn_status_string.argtypes = [ctypes.c_int]
+        L.vdn_status_string.restype = ctypes.c_char_p
+        L.vdn_last_error.argtypes = []
+        L.vdn_last_error.restype = ctypes.c_char_p
+        L.vdn_version.argtypes = []
+        L.vdn_version.restype = ctypes.c_int32
+        _lib = L
+    return _lib
+
+
+def declared_symbols() -> list[str]:
+    """Every function name that include/vdn.h declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vdn_\w+)\s*\(", text)))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise VdnError(VDN_ERR_INVALID, "tensor is not on a CUDA device")
+    if not t.is_contiguous():
+        raise VdnError(VDN_ERR_INVALID, "tensor is not contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int):
+    if status != VDN_OK:
+        L = lib()
+        name = L.vdn_status_string(status).decode()
+        msg = L.vdn_last_error().decode()
+        raise VdnError(status, f"{name}: {msg}")
+
+
+def _shp(s: vdn_shape):
+    return ctypes.cast(ctypes.pointer(s), _P)
+
+
+def vdn_frame_grams(s, K, V, beta, A, Bm, info=None, stream=None):
+    _check(lib().vdn_frame_grams(_shp(s), _ptr(K), _ptr(V), _ptr(beta), _ptr(A), _ptr(Bm), _ptr(info),
+                                 _stream(stream)))
+
+
+def vdn_frame_factor(s, A, Bm, alpha, M, J, info, stream=None):
+    _check(lib().vdn_frame_factor(_shp(s), _ptr(A), _ptr(Bm), _ptr(alpha), _ptr(M), _ptr(J), _ptr(info),
+                                  _stream(stream)))
+
+
+def vdn_chunk_compose(s, M, J, Mf, Jf, Mb, Jb, stream=None):
+    _check(lib().vdn_chunk_compose(_shp(s), _ptr(M), _ptr(J), _ptr(Mf), _ptr(Jf), _ptr(Mb), _ptr(Jb),
+                                   _stream(stream)))
+
+
+def vdn_scan_fwd(s, Mf, Jf, S_T, F, stream=None):
+    _check(lib().vdn_scan_fwd(_shp(s), _ptr(Mf), _ptr(Jf), _ptr(S_T), _ptr(F), _stream(stream)))
+
+
+def vdn_scan_bwd(s, Mb, Jb, S_T, G, stream=None):
+    _check(lib().vdn_scan_bwd(_shp(s), _ptr(Mb), _ptr(Jb), _ptr(S_T), _ptr(G), _stream(stream)))
+
+
+def vdn_scan_bidir(s, Mf, Jf, Mb, Jb, S_T, F, G, stream=None):
+    _check(lib().vdn_scan_bidir(_shp(s), _ptr(Mf), _ptr(Jf), _ptr(Mb), _ptr(Jb), _ptr(S_T), _ptr(F),
+                                _ptr(G), _stream(stream)))
+
+
+def vdn_chunk_readout(s, Q, F, G, O, info=None, stream=None):
+    _check(lib().vdn_chunk_readout(_shp(s), _ptr(Q), _ptr(F), _ptr(G), _ptr(O), _ptr(info),
+                                   _stream(stream)))
+
+
+def vdn_text_state_workspace_bytes(s) -> int:
+    return int(lib().vdn_text_state_workspace_bytes(_shp(s)))
+
+
+def vdn_text_state(s, Kx, Vx, beta_x, S_T, workspace, info, stream=None):
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().vdn_text_state(_shp(s), _ptr(Kx), _ptr(Vx), _ptr(beta_x), _ptr(S_T), _ptr(workspace),
+                                nbytes, _ptr(info), _stream(stream)))
+
+
+def vdn_forward_workspace_bytes(s) -> int:
+    return int(lib().vdn_forward_workspace_bytes(_shp(s)))
+
+
+def vdn_forward(s, Q, K, V, beta, alpha, Kx, Vx, beta_x, O, F, G, workspace, info, stream=None):
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().vdn_forward(_shp(s), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(alpha), _ptr(Kx),
+                             _ptr(Vx), _ptr(beta_x), _ptr(O), _ptr(F), _ptr(G), _ptr(workspace), nbytes,
+                             _ptr(info), _stream(stream)))
+
+
+def vdn_status_string(status: int) -> str:
+    return lib().vdn_status_string(status).decode()
+
+
+def vdn_last_error() -> str:
+    return lib().vdn_last_error().decode()
+
+
+def vdn_version() -> int:
+    return int(lib().vdn_version())
+
+
+# ------------------------------------------------------------------ helpers
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A 256-byte-aligned uint8 device buffer of at least nbytes bytes."""
+    return torch.empty(max(1, nbytes), dtype=torch.uint8, device=device)
+
+
+class Forward:
+    """Preallocated buffers for repeated vdn_forward calls on one shape."""
+
+    def __init__(self, s: vdn_shape, device="cuda", keep_states=True):
+        self.s = s
+        BH = s.B * s.H
+        C = s.C
+        self.ws = workspace(vdn_forward_workspace_bytes(s), device)
+        self.info = torch.zeros(1, dtype=torch.int32, device=device)
+        out_dt = TORCH_DTYPE[s.out_dtype]
+        self.O = torch.empty((s.B, s.H, s.T, s.U, s.dv), dtype=out_dt, device=device)
+        self.F = self.G = None
+        if keep_states:
+            self.F = torch.empty((s.B, s.H, C + 1, s.dv, s.dk), dtype=torch.float32, device=device)
+            self.G = torch.empty_like(self.F)
+        del BH
+
+    def __call__(self, Q, K, V, beta, alpha, Kx, Vx, beta_x, stream=None):
+        vdn_forward(self.s, Q, K, V, beta, alpha, Kx, Vx, beta_x, self.O, self.F, self.G, self.ws,
+                    self.info, stream)
+        return self.O

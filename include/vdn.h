@@ -1,0 +1,206 @@
+/*
+ * vdn.h - C ABI of the B200 (sm_100a) frame-wise delta-rule memory (VDA).
+ *
+ * The operations follow the paper "Video DeltaNet: A Video-Native Hybrid
+ * Attention for Livestream Video Generation" (summary page). Notation, per
+ * (batch b, head h): frames t = 0..T-1, tokens u = 0..U-1, keys/queries of
+ * width d_k, values of width d_v, state S of shape [d_v, d_k] (S maps a key to
+ * a value; a query reads S q). Chunks hold `chunk` (= 5) consecutive frames,
+ * C = ceil(T / chunk), the last one possibly partial.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Layout     : dense row-major, innermost index fastest. Q, K, V are
+ *              [B, H, T, U, d]; text keys/values are [B, H, n_text, d];
+ *              per-frame matrices are [B, H, T, d, d]; chunk maps are
+ *              [B, H, C, d, d]; boundary states are [B, H, C+1, d_v, d_k].
+ * Types      : Q/K/V/Kx/Vx are float32 or bfloat16 (shape.in_dtype); O is
+ *              float32 or bfloat16 (shape.out_dtype); beta, alpha, every
+ *              matrix and every state are float32.
+ * Memory     : every pointer is a DEVICE pointer, 16-byte aligned, owned by
+ *              the caller. The library never allocates, frees or keeps a
+ *              pointer after the call; the fused call takes a caller
+ *              workspace.
+ * Streams    : each call validates its arguments on the host, enqueues its
+ *              kernels on `stream` (NULL = the legacy default stream) and
+ *              returns without synchronising. There is no global mutable
+ *              state; calls on different streams may run concurrently if
+ *              their outputs do not overlap.
+ * Errors     : argument problems are reported synchronously (VDN_ERR_INVALID
+ *              or VDN_ERR_UNSUPPORTED) before anything is enqueued; a launch
+ *              failure returns VDN_ERR_CUDA. vdn_last_error() gives a one-line
+ *              message for the calling thread. A numeric failure on the device
+ *              (a non-positive or non-finite pivot when factoring I + A_t) is
+ *              written to the device word *info: 0 = success, otherwise
+ *              1 + the smallest failing linear frame index (b*H + h)*T + t.
+ *              No kernel traps, asserts or waits without a time limit; a
+ *              pipeline wait that exceeds its limit sets *info to
+ *              VDN_INFO_TIMEOUT instead.
+ * Sizes      : B, H, T, U, n_text >= 0 (zero sizes are valid and do no work);
+ *              d_k == d_v in {16, 32, 64, 128}; 1 <= chunk <= 16.
+ */
+#ifndef VDN_H
+#define VDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; NULL selects the legacy default stream. */
+typedef struct CUstream_st *vdn_stream_t;
+
+typedef enum {
+  VDN_OK = 0,
+  VDN_ERR_INVALID = 1,     /* null/misaligned pointer, bad size or enum */
+  VDN_ERR_UNSUPPORTED = 2, /* valid request this build has no kernel for */
+  VDN_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  VDN_ERR_NUMERIC = 4      /* reserved for host-side numeric checks */
+} vdn_status;
+
+typedef enum { VDN_F32 = 0, VDN_BF16 = 1 } vdn_dtype;
+
+/* *info value written when a device-side wait ran out of time. */
+#define VDN_INFO_TIMEOUT (-1)
+
+typedef struct {
+  int32_t B, H, T, U; /* batch, heads, latent frames, tokens per frame */
+  int32_t dk, dv;     /* key and value width (equal in this build) */
+  int32_t n_text;     /* text tokens per (b, h) */
+  int32_t chunk;      /* frames per chunk (5 in the paper) */
+  int32_t anchors;    /* 1: frames 0 and T-1 are anchors (no write, no read) */
+  int32_t in_dtype;   /* vdn_dtype of Q, K, V, Kx, Vx */
+  int32_t out_dtype;  /* vdn_dtype of O */
+} vdn_shape;
+
+/*
+ * Frame statistics. Paper: "Method steps", step (3):
+ *   A_t = K_t^T Diag(beta_t) K_t   [d_k, d_k]   (symmetric)
+ *   B_t = V_t^T Diag(beta_t) K_t   [d_v, d_k]
+ * with one scalar write gate beta_t per (b, h, t).
+ * In : K [B,H,T,U,dk], V [B,H,T,U,dv] (in_dtype); beta [B,H,T] float32.
+ * Out: A [B,H,T,dk,dk], Bm [B,H,T,dv,dk] float32 (fully overwritten).
+ * Every frame, anchors included, is computed (the factor step skips anchors).
+ * info: optional device int32 (may be NULL) that receives VDN_INFO_TIMEOUT if
+ *       a pipeline wait runs out of time; it is not reset by this call.
+ */
+vdn_status vdn_frame_grams(const vdn_shape *s, const void *K, const void *V,
+                           const float *beta, float *A, float *Bm,
+                           int32_t *info, vdn_stream_t stream);
+
+/*
+ * Per-frame factor/solve. Paper: "Core method" (closed form
+ * S_t = (S_{t-1} Diag(alpha_t) + B_t)(I + A_t)^{-1}) and "Method steps",
+ * step (3) ("factor I + A_t in batch to get the transition M_t and the
+ * injection J_t"):
+ *   M_t = Diag(alpha_t) (I + A_t)^{-1},   J_t = B_t (I + A_t)^{-1},
+ * so that S_t = S_{t-1} M_t + J_t. Anchor frames (shape.anchors) get M = I,
+ * J = 0. The frames do not depend on the state and are factored in parallel.
+ * In : A [B,H,T,dk,dk], Bm [B,H,T,dv,dk], alpha [B,H,T,dk] float32.
+ * Out: M [B,H,T,dk,dk], J [B,H,T,dv,dk] float32; *info (device int32) is
+ *      reset to 0 and then set as described in the file header.
+ */
+vdn_status vdn_frame_factor(const vdn_shape *s, const float *A, const float *Bm,
+                            const float *alpha, float *M, float *J,
+                            int32_t *info, vdn_stream_t stream);
+
+/*
+ * Chunk-level composition. Paper: "Technical novelty" (frame-level affine
+ * transitions are composed into chunk-level transitions before the scan,
+ * cutting the scan depth to about 1/5) and "Method steps", step (4)
+ * (S_out = S_in M_chunk + J_chunk). For chunk c with frames f0 < ... < fn:
+ *   forward : S -> S Mf_c + Jf_c applies frames f0, f1, ..., fn in order;
+ *   backward: S -> S Mb_c + Jb_c applies frames fn, ..., f1, f0.
+ * In : M [B,H,T,dk,dk], J [B,H,T,dv,dk] (from vdn_frame_factor).
+ * Out: Mf, Mb [B,H,C,dk,dk]; Jf, Jb [B,H,C,dv,dk] float32.
+ */
+vdn_status vdn_chunk_compose(const vdn_shape *s, const float *M, const float *J,
+                             float *Mf, float *Jf, float *Mb, float *Jb,
+                             vdn_stream_t stream);
+
+/*
+ * Forward scan over chunk boundaries. Paper: "Core method" (the forward scan
+ * summarises the context before the window; the text state initialises both
+ * scans) and step (4) (half-and-half initialisation):
+ *   F_0 = S_T / 2,   F_{c+1} = F_c Mf_c + Jf_c,   c = 0..C-1.
+ * In : Mf [B,H,C,dk,dk], Jf [B,H,C,dv,dk], S_T [B,H,dv,dk].
+ * Out: F [B,H,C+1,dv,dk] float32.
+ */
+vdn_status vdn_scan_fwd(const vdn_shape *s, const float *Mf, const float *Jf,
+                        const float *S_T, float *F, vdn_stream_t stream);
+
+/*
+ * Backward scan, the mirror of vdn_scan_fwd:
+ *   G_C = S_T / 2,   G_c = G_{c+1} Mb_c + Jb_c,   c = C-1..0.
+ * Out: G [B,H,C+1,dv,dk] float32.
+ */
+vdn_status vdn_scan_bwd(const vdn_shape *s, const float *Mb, const float *Jb,
+                        const float *S_T, float *G, vdn_stream_t stream);
+
+/* Both scans in one launch, on separate thread blocks. */
+vdn_status vdn_scan_bidir(const vdn_shape *s, const float *Mf, const float *Jf,
+                          const float *Mb, const float *Jb, const float *S_T,
+                          float *F, float *G, vdn_stream_t stream);
+
+/*
+ * Chunk readout. Paper: "Core method" (each query chunk keeps exact softmax
+ * attention inside a chunk-aligned bidirectional 15-frame window; the linear
+ * memory carries everything outside it; the forward and backward readouts are
+ * summed, so nothing is counted twice) and step (2) (the linear branch drops
+ * the anchor rows). For frame t of chunk c = t / chunk:
+ *   R_c = F_{max(c-1,0)} + G_{min(c+2,C)},   o_{t,u} = R_c q_{t,u},
+ * and o = 0 on anchor frames.
+ * In : Q [B,H,T,U,dk] (in_dtype); F, G [B,H,C+1,dv,dk] float32.
+ * Out: O [B,H,T,U,dv] (out_dtype, rounded to nearest even), fully written.
+ * info: optional, as for vdn_frame_grams.
+ */
+vdn_status vdn_chunk_readout(const vdn_shape *s, const void *Q, const float *F,
+                             const float *G, void *O, int32_t *info,
+                             vdn_stream_t stream);
+
+/*
+ * Text state. Paper: "Core method" (the text prompt is summarised into a text
+ * state S^T that initialises both scans). Reading: one VDA update from the
+ * zero state over the n_text text tokens, with gate beta_x and no decay:
+ *   S_T = beta_x V_x^T K_x (I + beta_x K_x^T K_x)^{-1}.
+ * In : Kx [B,H,n_text,dk], Vx [B,H,n_text,dv] (in_dtype); beta_x [B,H] float32.
+ * Out: S_T [B,H,dv,dk] float32; *info as for vdn_frame_factor.
+ * workspace: device scratch of at least vdn_text_state_workspace_bytes(s)
+ * bytes, 256-byte aligned, not read before it is written.
+ */
+size_t vdn_text_state_workspace_bytes(const vdn_shape *s);
+vdn_status vdn_text_state(const vdn_shape *s, const void *Kx, const void *Vx,
+                          const float *beta_x, float *S_T, void *workspace,
+                          size_t workspace_bytes, int32_t *info,
+                          vdn_stream_t stream);
+
+/*
+ * The whole linear branch in one call: text state, frame statistics,
+ * factor, chunk composition, both scans and the chunk readout.
+ * In : Q, K, V [B,H,T,U,d] and Kx, Vx [B,H,n_text,d] (in_dtype);
+ *      beta [B,H,T], alpha [B,H,T,dk], beta_x [B,H] float32.
+ * Out: O [B,H,T,U,dv] (out_dtype). If F and G are not NULL they receive the
+ *      boundary states [B,H,C+1,dv,dk]; *info as for vdn_frame_factor.
+ * workspace: at least vdn_forward_workspace_bytes(s) bytes, 256-byte aligned.
+ */
+size_t vdn_forward_workspace_bytes(const vdn_shape *s);
+vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K,
+                       const void *V, const float *beta, const float *alpha,
+                       const void *Kx, const void *Vx, const float *beta_x,
+                       void *O, float *F, float *G, void *workspace,
+                       size_t workspace_bytes, int32_t *info,
+                       vdn_stream_t stream);
+
+/* Name of a status code (static string). */
+const char *vdn_status_string(vdn_status st);
+/* Message of the last failing call on this thread ("" if none). */
+const char *vdn_last_error(void);
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t vdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VDN_H */

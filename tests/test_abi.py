@@ -1,0 +1,115 @@
+"""The C ABI without a GPU: the library loads, exports every symbol that
+include/vdn.h declares, and rejects bad arguments on the host before it
+touches the device."""
+import ctypes
+
+import pytest
+
+from frame_wise_delta_b200 import build, vdn
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return vdn.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = vdn.declared_symbols()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_version_and_status_strings(L):
+    assert vdn.vdn_version() >= 100
+    assert vdn.vdn_status_string(vdn.VDN_OK) == "VDN_OK"
+    assert vdn.vdn_status_string(vdn.VDN_ERR_INVALID) == "VDN_ERR_INVALID"
+    assert vdn.vdn_status_string(99) == "VDN_ERR_UNKNOWN"
+
+
+def _call(L, name, *args):
+    fn = getattr(L, name)
+    return fn(*args)
+
+
+def _shape(**kw):
+    base = dict(B=1, H=2, T=10, U=16, d=16, n_text=8, chunk=5, anchors=0, in_dtype="f32")
+    base.update(kw)
+    return vdn.make_shape(**base)
+
+
+def _p(s):
+    return ctypes.cast(ctypes.pointer(s), ctypes.c_void_p)
+
+
+def test_null_shape_is_invalid(L):
+    st = L.vdn_frame_grams(None, None, None, None, None, None, None, None)
+    assert st == vdn.VDN_ERR_INVALID
+    assert "shape" in vdn.vdn_last_error()
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=48), vdn.VDN_ERR_UNSUPPORTED),
+    (dict(chunk=0), vdn.VDN_ERR_INVALID),
+    (dict(chunk=17), vdn.VDN_ERR_INVALID),
+    (dict(anchors=2), vdn.VDN_ERR_INVALID),
+    (dict(T=-1), vdn.VDN_ERR_INVALID),
+    (dict(U=-3), vdn.VDN_ERR_INVALID),
+])
+def test_bad_shapes(L, kw, status):
+    s = _shape(**kw)
+    assert L.vdn_frame_grams(_p(s), 16, 16, 16, 16, 16, None, None) == status
+
+
+def test_bad_dtype(L):
+    s = _shape()
+    s.in_dtype = 7
+    assert L.vdn_chunk_readout(_p(s), 16, 16, 16, 16, None, None) == vdn.VDN_ERR_INVALID
+
+
+def test_dk_dv_mismatch(L):
+    s = _shape()
+    s.dv = 32
+    assert L.vdn_frame_grams(_p(s), 16, 16, 16, 16, 16, None, None) == vdn.VDN_ERR_UNSUPPORTED
+
+
+def test_null_and_misaligned_pointers(L):
+    s = _shape()
+    assert L.vdn_frame_grams(_p(s), None, 16, 16, 16, 16, None, None) == vdn.VDN_ERR_INVALID
+    assert "K is NULL" in vdn.vdn_last_error()
+    assert L.vdn_frame_grams(_p(s), 16, 16, 16, 16, 0x1008, None, None) == vdn.VDN_ERR_INVALID
+    assert "Bm is not 16-byte aligned" in vdn.vdn_last_error()
+    assert L.vdn_chunk_compose(_p(s), 16, 16, 16, None, 16, 16, None) == vdn.VDN_ERR_INVALID
+    assert L.vdn_scan_bidir(_p(s), 16, 16, 16, 16, None, 16, 16, None) == vdn.VDN_ERR_INVALID
+    assert "S_T" in vdn.vdn_last_error()
+
+
+def test_workspace_checks(L):
+    s = _shape()
+    need = vdn.vdn_forward_workspace_bytes(s)
+    assert need > 0 and need % 256 == 0
+    args = [_p(s)] + [16] * 9 + [16, 16, 16]  # Q..O, F, G, workspace
+    st = L.vdn_forward(*args[:13], need - 1, 16, None)
+    assert st == vdn.VDN_ERR_INVALID and "workspace" in vdn.vdn_last_error()
+    st = L.vdn_forward(*args[:12], 0x1010, need, 16, None)
+    assert st == vdn.VDN_ERR_INVALID and "256-byte" in vdn.vdn_last_error()
+    assert vdn.vdn_text_state_workspace_bytes(s) == 2 * 2 * 16 * 16 * 4
+
+
+def test_forward_workspace_grows_with_frames(L):
+    a = vdn.vdn_forward_workspace_bytes(_shape(T=10))
+    b = vdn.vdn_forward_workspace_bytes(_shape(T=20))
+    assert b > a
+    # zero-size problems are valid and need no device work
+    s = _shape(B=0)
+    assert L.vdn_frame_grams(_p(s), None, None, None, None, None, None, None) == vdn.VDN_OK
+    assert L.vdn_chunk_readout(_p(s), None, None, None, None, None, None) == vdn.VDN_OK
+
+
+def test_binding_refuses_host_tensors(L):
+    import torch
+    s = _shape()
+    x = torch.zeros(4)
+    with pytest.raises(vdn.VdnError):
+        vdn.vdn_frame_grams(s, x, x, x, x, x)
