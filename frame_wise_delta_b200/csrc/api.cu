@@ -162,6 +162,8 @@ vdn_status run_text_state(const Geo &g, const void *Kx, const void *Vx, const fl
 
 }  // namespace
 
+void vdn::set_last_error(const char *msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+
 extern "C" {
 
 const char *vdn_status_string(vdn_status st) {

@@ -32,6 +32,9 @@ bool readout_tc_supported(int in_dtype, int out_dtype, int D, int U);
 cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, void *O, long long BH,
                               int T, int U, int chunk, int anchors, int32_t *info, cudaStream_t st);
 
+// Message returned by vdn_last_error() on this thread.
+void set_last_error(const char *msg);
+
 // Driver entry point for tensor-map encoding (resolved once, thread-safe).
 void *tensor_map_encoder();
 int device_sm_count();

@@ -65,6 +65,7 @@ _SIGS = {
     "vdn_chunk_readout": [_P, _P, _P, _P, _P, _P, _P],
     "vdn_text_state": [_P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P],
     "vdn_forward": [_P] * 13 + [ctypes.c_size_t, _P, _P],
+    "vdn_text_state_noalloc": [_P, _P, _P, _P, _P, _P, _P],
 }
 
 
@@ -175,6 +176,12 @@ def vdn_text_state(s, Kx, Vx, beta_x, S_T, workspace, info, stream=None):
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().vdn_text_state(_shp(s), _ptr(Kx), _ptr(Vx), _ptr(beta_x), _ptr(S_T), _ptr(workspace),
                                 nbytes, _ptr(info), _stream(stream)))
+
+
+def vdn_text_state_noalloc(s, Kx, Vx, beta_x, S_T, info, stream=None):
+    """vdn_text_state with the library's fixed device scratch instead of a workspace."""
+    _check(lib().vdn_text_state_noalloc(_shp(s), _ptr(Kx), _ptr(Vx), _ptr(beta_x), _ptr(S_T), _ptr(info),
+                                        _stream(stream)))
 
 
 def vdn_forward_workspace_bytes(s) -> int:

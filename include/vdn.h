@@ -177,6 +177,26 @@ vdn_status vdn_text_state(const vdn_shape *s, const void *Kx, const void *Vx,
                           vdn_stream_t stream);
 
 /*
+ * Text state without a caller workspace (the paper has no counterpart: this
+ * is a deployment addition). Same result as vdn_text_state, for callers that
+ * cannot allocate device memory, such as a serving engine that reserves all
+ * of its memory at start-up or a real-time loop that must not call cudaMalloc.
+ * The two Gram matrices per (b, h) go to a fixed 4 MiB scratch array that the
+ * library keeps in device memory on every GPU that loads it, until exit; so
+ * 2 * B * H * dk * dk * 4 bytes must not exceed 4 MiB (B*H <= 32 at d = 128),
+ * else VDN_ERR_UNSUPPORTED is returned before anything is enqueued.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make it before any stream capture.
+ * Every call shares the array and it keeps the last call's contents (nothing
+ * in it needs to start at zero); calls that overlap on the GPU race on it.
+ * In/Out/info as for vdn_text_state. Allocates nothing.
+ */
+vdn_status vdn_text_state_noalloc(const vdn_shape *s, const void *Kx,
+                                  const void *Vx, const float *beta_x,
+                                  float *S_T, int32_t *info,
+                                  vdn_stream_t stream);
+
+/*
  * The whole linear branch in one call: text state, frame statistics,
  * factor, chunk composition, both scans and the chunk readout.
  * In : Q, K, V [B,H,T,U,d] and Kx, Vx [B,H,n_text,d] (in_dtype);
