@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["vdn", "reference"], default="vdn")
     ap.add_argument("--workload", default="h3")
+    ap.add_argument("--heads", type=int, default=0, help="override the head count (small profiling cases)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     return ap.parse_args()
@@ -194,6 +196,9 @@ def main():
     from frame_wise_delta_b200 import synth
 
     w = synth.WORKLOADS[args.workload]
+    if args.heads:
+        import dataclasses
+        w = dataclasses.replace(w, H=args.heads, name=f"{w.name}_h{args.heads}")
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -291,8 +296,43 @@ def main():
     value = frames_all / (ms_per_step / 1e3)
 
     # ---- end to end: pinned host inputs -> device -> vdn_forward -> O to host
+    e2e = e2e_measure(args, host, d, s, dev, stream, barrier, world, frames_all, dt) if not args.no_e2e else None
+
+    if rank == 0:
+        hbm_gbs, bf16_tflops, peak_src = load_peaks()
+        roof = roofline(w, stage_ms, hbm_gbs, peak_src)
+        line = {
+            "metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "state_dtype": "f32",
+            "data": "synthetic", "config": workload_config(w),
+            "tokens_per_s": value * U,
+            "hbm_frac_whole_pass": alg_bytes(w) * world / (ms_per_step / 1e3) / (hbm_gbs * 1e9),
+            "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+            "step_ms_min_max": [min(step_ms), max(step_ms)],
+            "roofline": roof,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = oracle_sample(w, full, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def e2e_measure(args, host, d, s, dev, stream, barrier, world, frames_all, dt):
+    """Same metric through vdn_forward with the step's inputs copied from pinned
+    host memory and O copied back, inside the timed region."""
+    import torch
+    import torch.distributed as dist
+
+    from frame_wise_delta_b200 import vdn
+
     fwd = vdn.Forward(s, device=dev, keep_states=False)
-    O_host = torch.empty(O.shape, dtype=dt).pin_memory()
+    O_host = torch.empty(fwd.O.shape, dtype=dt).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = O_host.numel() * O_host.element_size()
 
@@ -318,32 +358,9 @@ def main():
     te = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
     if world > 1:
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = frames_all / (float(te.item()) / e2e_steps / 1e3)
     assert int(fwd.info.item()) == 0
-
-    if rank == 0:
-        hbm_gbs, bf16_tflops, peak_src = load_peaks()
-        roof = roofline(w, stage_ms, hbm_gbs, peak_src)
-        line = {
-            "metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": world, "steps": args.steps,
-            "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "state_dtype": "f32",
-            "data": "synthetic", "config": workload_config(w),
-            "tokens_per_s": value * U,
-            "hbm_frac_whole_pass": alg_bytes(w) * world / (ms_per_step / 1e3) / (hbm_gbs * 1e9),
-            "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
-            "step_ms_min_max": [min(step_ms), max(step_ms)],
-            "roofline": roof,
-            "e2e": {"value": e2e_value, "unit": "frames/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clk.summary(),
-        }
-        if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = oracle_sample(w, full, args.cpu_seconds)
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    return {"value": frames_all / (float(te.item()) / e2e_steps / 1e3), "unit": "frames/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
 
 def alg_bytes(w):
