@@ -49,6 +49,22 @@ def parse():
     return ap.parse_args()
 
 
+def event_ms(a, b) -> float:
+    """Elapsed ms between two recorded CUDA events (recorded by the library on
+    the launching stream), read through the driver API."""
+    import ctypes
+
+    global _CU
+    if "_CU" not in globals():
+        _CU = ctypes.CDLL("libcuda.so.1")
+        _CU.cuEventElapsedTime.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_void_p, ctypes.c_void_p]
+    out = ctypes.c_float()
+    r = _CU.cuEventElapsedTime(ctypes.byref(out), ctypes.c_void_p(a.cuda_event), ctypes.c_void_p(b.cuda_event))
+    if r != 0:
+        raise RuntimeError(f"cuEventElapsedTime failed ({r})")
+    return float(out.value)
+
+
 def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
 
@@ -236,39 +252,18 @@ def main():
     s = vdn.shape_for(w)
     B, H, T, U, D, C = w.B, w.H, w.T, w.U, w.d, w.C
     f32 = dict(dtype=torch.float32, device=dev)
-    A = torch.empty((B, H, T, D, D), **f32)
-    Bm = torch.empty_like(A)
-    M = torch.empty_like(A)
-    J = torch.empty_like(A)
-    maps = [torch.empty((B, H, C, D, D), **f32) for _ in range(4)]
-    F = torch.empty((B, H, C + 1, D, D), **f32)
-    G = torch.empty_like(F)
-    S_T = torch.empty((B, H, D, D), **f32)
-    tws = vdn.workspace(vdn.vdn_text_state_workspace_bytes(s), dev)
-    info = torch.zeros(1, dtype=torch.int32, device=dev)
-    O = torch.empty((B, H, T, U, D), dtype=dt, device=dev)
+    fwd_dev = vdn.Forward(s, device=dev)
     stream = torch.cuda.current_stream()
 
     stages = ["text_state", "frame_grams", "frame_factor", "chunk_compose", "scan_bidir", "chunk_readout"]
-    launches_per_step = 7  # text gram + text factor + one kernel per other stage
+    tensor_path = w.dtype == "bf16" and D == 128
+    # our kernels per step: text (gram, invert, injection chain) + gram +
+    # invert + compose (M and J chains) + scan + readout
+    launches_per_step = 9 if tensor_path else 7
 
     def step(ev=None):
-        def mark(i):
-            if ev is not None:
-                ev[i].record(stream)
-        mark(0)
-        vdn.vdn_text_state(s, d["Kx"], d["Vx"], d["beta_x"], S_T, tws, info)
-        mark(1)
-        vdn.vdn_frame_grams(s, d["K"], d["V"], d["beta"], A, Bm, info)
-        mark(2)
-        vdn.vdn_frame_factor(s, A, Bm, d["alpha"], M, J, info)
-        mark(3)
-        vdn.vdn_chunk_compose(s, M, J, *maps)
-        mark(4)
-        vdn.vdn_scan_bidir(s, maps[0], maps[1], maps[2], maps[3], S_T, F, G)
-        mark(5)
-        vdn.vdn_chunk_readout(s, d["Q"], F, G, O, info)
-        mark(6)
+        fwd_dev(d["Q"], d["K"], d["V"], d["beta"], d["alpha"], d["Kx"], d["Vx"], d["beta_x"], events=ev)
+    info = fwd_dev.info
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -284,9 +279,9 @@ def main():
             step(evs[i])
         torch.cuda.synchronize()
     barrier()
-    step_ms = [e[0].elapsed_time(e[6]) for e in evs]
-    stage_ms = {name: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j, name in enumerate(stages)}
-    total_ms = evs[0][0].elapsed_time(evs[-1][6])
+    step_ms = [event_ms(e[0], e[6]) for e in evs]
+    stage_ms = {name: statistics.mean(event_ms(e[j], e[j + 1]) for e in evs) for j, name in enumerate(stages)}
+    total_ms = event_ms(evs[0][0], evs[-1][6])
     t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -300,7 +295,7 @@ def main():
 
     if rank == 0:
         hbm_gbs, bf16_tflops, peak_src = load_peaks()
-        roof = roofline(w, stage_ms, hbm_gbs, peak_src)
+        roof = roofline(w, stage_ms, hbm_gbs, peak_src, bf16_tflops)
         line = {
             "metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -373,25 +368,30 @@ def alg_bytes(w):
     return qkvo + text + gates
 
 
-def roofline(w, stage_ms, hbm_gbs, peak_src):
+def roofline(w, stage_ms, hbm_gbs, peak_src, bf16_tflops=1607.7):
     """Roofline of the dominant stage. Per-unit algorithmic figures:
     frame_grams: per frame reads K, V (2 U d bf16) and writes A, B (2 d^2 fp32);
     chunk_readout: per frame reads Q, writes O (2 U d bf16) plus two states per chunk;
-    frame_factor: 4 d^3 flop per non-anchor frame (Gauss-Jordan on [I+A; B]);
-    chunk_compose: 4 d^3 flop per frame after the first of each chunk and direction;
-    scan_bidir: 2 directions x C x 2 d^3 flop."""
+    frame_factor: d^3 flop per non-anchor frame on the tensor path (symmetric
+      sweep), 4 d^3 on the CUDA-core path (Gauss-Jordan on [I+A; B]);
+    chunk_compose: 4 d^3 flop per frame step (M and J chains), per direction;
+    scan_bidir: 2 d^3 flop per chunk and direction."""
     B, H, T, U, d, C = w.B, w.H, w.T, w.U, w.d, w.C
     BH = B * H
     e = 2 if w.dtype == "bf16" else 4
+    tensor_path = w.dtype == "bf16" and d == 128
     frames = BH * T
     live = BH * (T - (2 if w.anchors and T > 1 else (1 if w.anchors else 0)))
-    steps = sum(max(0, min(5 * c + 5, T) - 5 * c - 1) for c in range(C))
+    steps = 0
+    for c in range(C):
+        fr = [t for t in range(5 * c, min(5 * c + 5, T)) if not (w.anchors and t in (0, T - 1))]
+        steps += len(fr) if tensor_path else max(0, len(range(5 * c, min(5 * c + 5, T))) - 1)
     units = {
         "frame_grams": ("hbm", frames * (2 * U * d * e + 2 * d * d * 4)),
         "chunk_readout": ("hbm", frames * 2 * U * d * e + BH * C * 2 * d * d * 4),
-        "frame_factor": ("alu", live * 4 * d ** 3),
-        "chunk_compose": ("alu", BH * 2 * steps * 4 * d ** 3),
-        "scan_bidir": ("alu", BH * 2 * C * 2 * d ** 3),
+        "frame_factor": ("alu", live * (d ** 3 if tensor_path else 4 * d ** 3)),
+        "chunk_compose": ("tensor" if tensor_path else "alu", BH * 2 * steps * 4 * d ** 3),
+        "scan_bidir": ("tensor" if tensor_path else "alu", BH * 2 * C * 2 * d ** 3),
     }
     name = max((k for k in units), key=lambda k: stage_ms.get(k, 0.0))
     bound, amount = units[name]
@@ -400,6 +400,10 @@ def roofline(w, stage_ms, hbm_gbs, peak_src):
         achieved = amount / sec / 1e9
         peak, unit = hbm_gbs, "GB/s"
         src = f"{peak_src} HBM copy bandwidth"
+    elif bound == "tensor":
+        achieved = amount / sec / 1e12
+        peak, unit = bf16_tflops, "TFLOP/s"
+        src = f"{peak_src} dense bf16 (burst); fp32 products issued as 3 bf16 MMAs"
     else:
         achieved = amount / sec / 1e12
         peak, unit = ALU_F32_TFLOPS, "TFLOP/s"

@@ -115,6 +115,7 @@ vdn_status need(const void *p, const char *name, bool required) {
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
+
 // ----------------------------------------------------------- stage calls
 vdn_status run_grams(const Geo &g, const void *K, const void *V, const float *beta, float *A,
                      float *Bm, long long nframes, int U, int32_t *info, cudaStream_t st) {
@@ -147,16 +148,46 @@ vdn_status run_readout(const Geo &g, const void *Q, const float *F, const float 
   return VDN_OK;
 }
 
+bool tensor_path(const Geo &g) { return g.in_dtype == VDN_BF16 && g.out_dtype == VDN_BF16 && g.D == 128; }
+
+size_t align256(size_t n);
+
+// Scratch of the text state: Ax, Bx (fp32) and, on the tensor path, the W images.
+struct TextLayout {
+  size_t ax, bx, wimg, total;
+};
+TextLayout text_layout(const Geo &g) {
+  TextLayout L{};
+  const size_t dd = (size_t)g.D * g.D * sizeof(float);
+  L.ax = 0;
+  L.bx = align256(g.BH * dd);
+  L.wimg = L.bx + align256(g.BH * dd);
+  L.total = L.wimg + (tensor_path(g) ? align256((size_t)g.BH * kImgBytes) : 0);
+  return L;
+}
+
 vdn_status run_text_state(const Geo &g, const void *Kx, const void *Vx, const float *beta_x,
-                          float *S_T, float *Ax, float *Bx, int32_t *info, cudaStream_t st) {
+                          float *S_T, char *ws, int32_t *info, cudaStream_t st) {
   if (g.BH == 0) return VDN_OK;
   if (g.n_text == 0) {
     VDN_CUDA(cudaMemsetAsync(S_T, 0, (size_t)g.BH * g.D * g.D * sizeof(float), st), "memset S_T");
     return VDN_OK;
   }
+  const TextLayout L = text_layout(g);
+  float *Ax = (float *)(ws + L.ax), *Bx = (float *)(ws + L.bx);
   VDN_TRY(run_grams(g, Kx, Vx, beta_x, Ax, Bx, g.BH, g.n_text, info, st));
-  VDN_CUDA(launch_factor_simt(Ax, Bx, nullptr, nullptr, S_T, info, g.BH, 1, 0, g.D, st),
-           "text factor");
+  if (tensor_path(g)) {
+    // S_T is the injection of one "frame" made of the text tokens: invert,
+    // then one J-chain step (B_x W_x) on the tensor cores.
+    uint8_t *Wimg = (uint8_t *)(ws + L.wimg);
+    VDN_CUDA(launch_invert_simt(Ax, nullptr, Wimg, info, g.BH, g.D, st), "text invert");
+    VDN_CUDA(launch_compose_tc(Wimg, Bx, Ax, nullptr, S_T, nullptr, nullptr, nullptr, g.BH, 1, 1, 0,
+                               /*parts=*/2, /*ndirs=*/1, info, st),
+             "text injection");
+  } else {
+    VDN_CUDA(launch_factor_simt(Ax, Bx, nullptr, nullptr, S_T, info, g.BH, 1, 0, g.D, st),
+             "text factor");
+  }
   return VDN_OK;
 }
 
@@ -283,7 +314,7 @@ vdn_status vdn_chunk_readout(const vdn_shape *s, const void *Q, const float *F, 
 size_t vdn_text_state_workspace_bytes(const vdn_shape *s) {
   Geo g;
   if (check_shape(s, &g) != VDN_OK) return 0;
-  return 2 * align256((size_t)g.BH * g.D * g.D * sizeof(float));
+  return text_layout(g).total;
 }
 
 vdn_status vdn_text_state(const vdn_shape *s, const void *Kx, const void *Vx, const float *beta_x,
@@ -300,37 +331,54 @@ vdn_status vdn_text_state(const vdn_shape *s, const void *Kx, const void *Vx, co
   VDN_TRY(need(info, "info", true));
   const size_t ws = vdn_text_state_workspace_bytes(s);
   VDN_TRY(need(workspace, "workspace", any && ws > 0));
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(VDN_ERR_INVALID, "workspace is not 256-byte aligned");
   if (workspace_bytes < ws)
     return fail(VDN_ERR_INVALID, "workspace of %zu bytes < %zu required", workspace_bytes, ws);
   cudaStream_t st = (cudaStream_t)stream;
   VDN_CUDA(cudaMemsetAsync(info, 0, sizeof(int32_t), st), "memset info");
-  float *Ax = (float *)workspace;
-  float *Bx = (float *)((char *)workspace + align256((size_t)g.BH * g.D * g.D * sizeof(float)));
-  return run_text_state(g, Kx, Vx, beta_x, S_T, Ax, Bx, info, st);
+  return run_text_state(g, Kx, Vx, beta_x, S_T, (char *)workspace, info, st);
+}
+
+vdn_status vdn_frame_invert(const vdn_shape *s, const float *A, float *W, int32_t *info,
+                            vdn_stream_t stream) {
+  g_err[0] = 0;
+  Geo g;
+  VDN_TRY(check_shape(s, &g));
+  const bool any = g.BH * g.T > 0;
+  VDN_TRY(need(A, "A", any));
+  VDN_TRY(need(W, "W", any));
+  VDN_TRY(need(info, "info", true));
+  cudaStream_t st = (cudaStream_t)stream;
+  VDN_CUDA(cudaMemsetAsync(info, 0, sizeof(int32_t), st), "memset info");
+  VDN_CUDA(launch_invert_simt(A, W, nullptr, info, g.BH * g.T, g.D, st), "invert");
+  return VDN_OK;
 }
 
 namespace {
 struct FwdLayout {
-  size_t ax, bx, st, a, b, mf, jf, mb, jb, f, g, total;
+  size_t text, st, a, b, wimg, mf, jf, mb, jb, mimg, f, g, total;
 };
 FwdLayout fwd_layout(const Geo &g) {
   FwdLayout L{};
   const size_t dd = (size_t)g.D * g.D * sizeof(float);
+  const bool tc = tensor_path(g);
   size_t off = 0;
   auto take = [&](size_t n) {
     size_t o = off;
     off += align256(n);
     return o;
   };
-  L.ax = take(g.BH * dd);
-  L.bx = take(g.BH * dd);
+  L.text = take(text_layout(g).total);
   L.st = take(g.BH * dd);
   L.a = take(g.BH * g.T * dd);
   L.b = take(g.BH * g.T * dd);
+  L.wimg = take(tc ? (size_t)g.BH * g.T * kImgBytes : 0);
   L.mf = take(g.BH * g.C * dd);
   L.jf = take(g.BH * g.C * dd);
   L.mb = take(g.BH * g.C * dd);
   L.jb = take(g.BH * g.C * dd);
+  L.mimg = take(tc ? (size_t)g.BH * 2 * g.C * kImgBytes : 0);
   L.f = take(g.BH * (g.C + 1) * dd);
   L.g = take(g.BH * (g.C + 1) * dd);
   L.total = off;
@@ -347,7 +395,8 @@ size_t vdn_forward_workspace_bytes(const vdn_shape *s) {
 vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K, const void *V,
                        const float *beta, const float *alpha, const void *Kx, const void *Vx,
                        const float *beta_x, void *O, float *F, float *G, void *workspace,
-                       size_t workspace_bytes, int32_t *info, vdn_stream_t stream) {
+                       size_t workspace_bytes, int32_t *info, const void *const *stage_events,
+                       vdn_stream_t stream) {
   g_err[0] = 0;
   Geo g;
   VDN_TRY(check_shape(s, &g));
@@ -361,40 +410,72 @@ vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K, const v
   VDN_TRY(need(Vx, "Vx", g.BH > 0 && g.n_text > 0));
   VDN_TRY(need(beta_x, "beta_x", g.BH > 0 && g.n_text > 0));
   VDN_TRY(need(O, "O", frames && g.U > 0));
-  VDN_TRY(need(F, "F", false));
-  VDN_TRY(need(G, "G", false));
   if ((F && !aligned16(F)) || (G && !aligned16(G)))
     return fail(VDN_ERR_INVALID, "F/G not 16-byte aligned");
   VDN_TRY(need(info, "info", true));
   const FwdLayout L = fwd_layout(g);
   VDN_TRY(need(workspace, "workspace", g.BH > 0));
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(VDN_ERR_INVALID, "workspace is not 256-byte aligned");
   if (workspace_bytes < L.total)
     return fail(VDN_ERR_INVALID, "workspace of %zu bytes < %zu required", workspace_bytes, L.total);
-  if (g.BH == 0) return VDN_OK;
 
   cudaStream_t st = (cudaStream_t)stream;
+  auto mark = [&](int i) -> vdn_status {
+    if (stage_events && stage_events[i]) {
+      VDN_CUDA(cudaEventRecord((cudaEvent_t)stage_events[i], st), "event record");
+    }
+    return VDN_OK;
+  };
+  VDN_TRY(mark(0));
+  if (g.BH == 0) {
+    for (int i = 1; i < 7; ++i) VDN_TRY(mark(i));
+    return VDN_OK;
+  }
   char *w = (char *)workspace;
-  float *Ax = (float *)(w + L.ax), *Bx = (float *)(w + L.bx), *S_T = (float *)(w + L.st);
+  float *S_T = (float *)(w + L.st);
   float *A = (float *)(w + L.a), *Bm = (float *)(w + L.b);
+  uint8_t *Wimg = (uint8_t *)(w + L.wimg), *Mimg = (uint8_t *)(w + L.mimg);
   float *Mf = (float *)(w + L.mf), *Jf = (float *)(w + L.jf);
   float *Mb = (float *)(w + L.mb), *Jb = (float *)(w + L.jb);
   float *Fo = F ? F : (float *)(w + L.f);
   float *Go = G ? G : (float *)(w + L.g);
+  const bool tc = tensor_path(g);
 
   VDN_CUDA(cudaMemsetAsync(info, 0, sizeof(int32_t), st), "memset info");
-  VDN_TRY(run_text_state(g, Kx, Vx, beta_x, S_T, Ax, Bx, info, st));
+  VDN_TRY(run_text_state(g, Kx, Vx, beta_x, S_T, w + L.text, info, st));
+  VDN_TRY(mark(1));
+  if (frames) VDN_TRY(run_grams(g, K, V, beta, A, Bm, g.BH * g.T, g.U, info, st));
+  VDN_TRY(mark(2));
   if (frames) {
-    VDN_TRY(run_grams(g, K, V, beta, A, Bm, g.BH * g.T, g.U, info, st));
-    // M and J overwrite A and Bm in place (each element is read and written
-    // by the same thread).
-    VDN_CUDA(launch_factor_simt(A, Bm, alpha, A, Bm, info, g.BH * g.T, g.T, g.anchors, g.D, st),
-             "factor");
-    VDN_CUDA(launch_compose_simt(A, Bm, Mf, Jf, Mb, Jb, g.BH, g.T, g.chunk, g.D, st), "compose");
+    if (tc) {
+      VDN_CUDA(launch_invert_simt(A, nullptr, Wimg, info, g.BH * g.T, g.D, st), "invert");
+    } else {
+      // M and J overwrite A and Bm in place (each element is read and
+      // written by the same thread).
+      VDN_CUDA(launch_factor_simt(A, Bm, alpha, A, Bm, info, g.BH * g.T, g.T, g.anchors, g.D, st),
+               "factor");
+    }
   }
-  VDN_CUDA(launch_scan_simt(Mf, Jf, Mb, Jb, S_T, Fo, Go, g.BH, g.C, g.D, 3, st), "scan");
+  VDN_TRY(mark(3));
+  if (frames) {
+    if (tc) {
+      VDN_CUDA(launch_compose_tc(Wimg, Bm, alpha, Mf, Jf, Mb, Jb, Mimg, g.BH, g.T, g.chunk, g.anchors,
+                                 3, 2, info, st),
+               "compose");
+    } else {
+      VDN_CUDA(launch_compose_simt(A, Bm, Mf, Jf, Mb, Jb, g.BH, g.T, g.chunk, g.D, st), "compose");
+    }
+  }
+  VDN_TRY(mark(4));
+  if (tc && frames) {
+    VDN_CUDA(launch_scan_tc(Mimg, Jf, Jb, S_T, Fo, Go, g.BH, g.C, 3, info, st), "scan");
+  } else {
+    VDN_CUDA(launch_scan_simt(Mf, Jf, Mb, Jb, S_T, Fo, Go, g.BH, g.C, g.D, 3, st), "scan");
+  }
+  VDN_TRY(mark(5));
   if (frames) VDN_TRY(run_readout(g, Q, Fo, Go, O, info, st));
+  VDN_TRY(mark(6));
   return VDN_OK;
 }
 

@@ -104,6 +104,48 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *desc, uint
       : "memory");
 }
 
+// Untiled bulk copy global -> shared (16-byte aligned, size multiple of 16),
+// completion counted on `bar` (bytes).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// ---------------------------------------------------------- bf16 images
+// A 128 x 128 bf16 operand image in the MN-major, 128-byte-swizzled layout
+// the tensor cores read: rows r (the K index) of 128 bytes, two 64-column
+// regions of 16 KB, 16-byte chunks permuted by (chunk ^ (r & 7)). An "image"
+// of an fp32 matrix is its bf16 hi part followed by its bf16 lo part
+// (x ~ hi + lo to ~2^-17 relative), 64 KB in all.
+constexpr int kImgHalf = 128 * 128 * 2;   // one bf16 image
+constexpr int kImgBytes = 2 * kImgHalf;   // hi + lo
+constexpr int kImgRegion = 128 * 128;     // 64-column region
+
+__device__ __forceinline__ uint32_t mn_off(int r, int x) {
+  return (uint32_t)(x >> 6) * kImgRegion + (uint32_t)r * 128u +
+         ((((uint32_t)(x & 63) >> 3) ^ (uint32_t)(r & 7)) << 4) + (uint32_t)(x & 7) * 2u;
+}
+
+__device__ __forceinline__ void split_bf16(float v, __nv_bfloat16 &h, __nv_bfloat16 &l) {
+  h = __float2bfloat16_rn(v);
+  l = __float2bfloat16_rn(v - __bfloat162float(h));
+}
+
+__device__ __forceinline__ uint32_t pack2(__nv_bfloat16 a, __nv_bfloat16 b) {
+  return (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
+}
+
+// Store one element (row r, column x) of a hi/lo image in global memory.
+__device__ __forceinline__ void img_store(uint8_t *img, int r, int x, float v) {
+  __nv_bfloat16 h, l;
+  split_bf16(v, h, l);
+  const uint32_t off = mn_off(r, x);
+  *reinterpret_cast<__nv_bfloat16 *>(img + off) = h;
+  *reinterpret_cast<__nv_bfloat16 *>(img + kImgHalf + off) = l;
+}
+
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),

@@ -64,7 +64,8 @@ _SIGS = {
     "vdn_scan_bidir": [_P, _P, _P, _P, _P, _P, _P, _P, _P],
     "vdn_chunk_readout": [_P, _P, _P, _P, _P, _P, _P],
     "vdn_text_state": [_P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P],
-    "vdn_forward": [_P] * 13 + [ctypes.c_size_t, _P, _P],
+    "vdn_forward": [_P] * 13 + [ctypes.c_size_t, _P, _P, _P],
+    "vdn_frame_invert": [_P, _P, _P, _P, _P],
     "vdn_text_state_noalloc": [_P, _P, _P, _P, _P, _P, _P],
 }
 
@@ -145,6 +146,10 @@ def vdn_frame_factor(s, A, Bm, alpha, M, J, info, stream=None):
                                   _stream(stream)))
 
 
+def vdn_frame_invert(s, A, W, info, stream=None):
+    _check(lib().vdn_frame_invert(_shp(s), _ptr(A), _ptr(W), _ptr(info), _stream(stream)))
+
+
 def vdn_chunk_compose(s, M, J, Mf, Jf, Mb, Jb, stream=None):
     _check(lib().vdn_chunk_compose(_shp(s), _ptr(M), _ptr(J), _ptr(Mf), _ptr(Jf), _ptr(Mb), _ptr(Jb),
                                    _stream(stream)))
@@ -188,11 +193,17 @@ def vdn_forward_workspace_bytes(s) -> int:
     return int(lib().vdn_forward_workspace_bytes(_shp(s)))
 
 
-def vdn_forward(s, Q, K, V, beta, alpha, Kx, Vx, beta_x, O, F, G, workspace, info, stream=None):
+def vdn_forward(s, Q, K, V, beta, alpha, Kx, Vx, beta_x, O, F, G, workspace, info, events=None,
+                stream=None):
+    """events: None or 7 torch.cuda.Event (enable_timing) recorded between the stages."""
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    ev = None
+    if events is not None:
+        arr = (ctypes.c_void_p * 7)(*[e.cuda_event if e is not None else None for e in events])
+        ev = ctypes.cast(arr, ctypes.c_void_p)
     _check(lib().vdn_forward(_shp(s), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(alpha), _ptr(Kx),
                              _ptr(Vx), _ptr(beta_x), _ptr(O), _ptr(F), _ptr(G), _ptr(workspace), nbytes,
-                             _ptr(info), _stream(stream)))
+                             _ptr(info), ev, _stream(stream)))
 
 
 def vdn_status_string(status: int) -> str:
@@ -230,7 +241,7 @@ class Forward:
             self.G = torch.empty_like(self.F)
         del BH
 
-    def __call__(self, Q, K, V, beta, alpha, Kx, Vx, beta_x, stream=None):
+    def __call__(self, Q, K, V, beta, alpha, Kx, Vx, beta_x, events=None, stream=None):
         vdn_forward(self.s, Q, K, V, beta, alpha, Kx, Vx, beta_x, self.O, self.F, self.G, self.ws,
-                    self.info, stream)
+                    self.info, events, stream)
         return self.O

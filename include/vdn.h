@@ -107,6 +107,18 @@ vdn_status vdn_frame_factor(const vdn_shape *s, const float *A, const float *Bm,
                             int32_t *info, vdn_stream_t stream);
 
 /*
+ * Per-frame inverse, the factor step as the fused path runs it:
+ *   W_t = (I + A_t)^{-1}      (symmetric; anchors are not special-cased here)
+ * so that M_t = Diag(alpha_t) W_t and J_t = B_t W_t. Paper: "Core method"
+ * (closed form) and "Method steps" step (3); "Technical novelty" (the inverse
+ * is produced directly, without a separate solve pipeline).
+ * In : A [B,H,T,dk,dk] float32.  Out: W [B,H,T,dk,dk] float32.
+ * *info is reset to 0 and then set as for vdn_frame_factor.
+ */
+vdn_status vdn_frame_invert(const vdn_shape *s, const float *A, float *W,
+                            int32_t *info, vdn_stream_t stream);
+
+/*
  * Chunk-level composition. Paper: "Technical novelty" (frame-level affine
  * transitions are composed into chunk-level transitions before the scan,
  * cutting the scan depth to about 1/5) and "Method steps", step (4)
@@ -204,6 +216,13 @@ vdn_status vdn_text_state_noalloc(const vdn_shape *s, const void *Kx,
  * Out: O [B,H,T,U,dv] (out_dtype). If F and G are not NULL they receive the
  *      boundary states [B,H,C+1,dv,dk]; *info as for vdn_frame_factor.
  * workspace: at least vdn_forward_workspace_bytes(s) bytes, 256-byte aligned.
+ * stage_events: NULL, or 7 cudaEvent_t (entries may be NULL) recorded on
+ *      `stream` before the text state and after the text state, the frame
+ *      statistics, the factor, the composition, the scans and the readout.
+ * With bf16 inputs and output and d = 128 the factor, composition and scans
+ * run on the tensor-core path (per-frame inverses W_t, then
+ * X <- (X Diag(alpha_t) + B_t) W_t chains, which equal X M_t + J_t); other
+ * shapes use the CUDA-core kernels of the stage calls above.
  */
 size_t vdn_forward_workspace_bytes(const vdn_shape *s);
 vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K,
@@ -211,7 +230,7 @@ vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K,
                        const void *Kx, const void *Vx, const float *beta_x,
                        void *O, float *F, float *G, void *workspace,
                        size_t workspace_bytes, int32_t *info,
-                       vdn_stream_t stream);
+                       const void *const *stage_events, vdn_stream_t stream);
 
 /* Name of a status code (static string). */
 const char *vdn_status_string(vdn_status st);

@@ -89,12 +89,15 @@ def test_workspace_checks(L):
     s = _shape()
     need = vdn.vdn_forward_workspace_bytes(s)
     assert need > 0 and need % 256 == 0
-    args = [_p(s)] + [16] * 9 + [16, 16, 16]  # Q..O, F, G, workspace
-    st = L.vdn_forward(*args[:13], need - 1, 16, None)
+    args = [_p(s)] + [16] * 9 + [16, 16, 256]  # Q..O, F, G, workspace
+    st = L.vdn_forward(*args[:13], need - 1, 16, None, None)
     assert st == vdn.VDN_ERR_INVALID and "workspace" in vdn.vdn_last_error()
-    st = L.vdn_forward(*args[:12], 0x1010, need, 16, None)
+    st = L.vdn_forward(*args[:12], 0x1010, need, 16, None, None)
     assert st == vdn.VDN_ERR_INVALID and "256-byte" in vdn.vdn_last_error()
     assert vdn.vdn_text_state_workspace_bytes(s) == 2 * 2 * 16 * 16 * 4
+    # bf16, d = 128: the tensor path also keeps one 64 KB inverse image per (b, h)
+    s2 = _shape(d=128, in_dtype="bf16")
+    assert vdn.vdn_text_state_workspace_bytes(s2) == 2 * 2 * 128 * 128 * 4 + 2 * 65536
 
 
 def test_forward_workspace_grows_with_frames(L):

@@ -114,6 +114,22 @@ def test_frame_factor(w):
     assert rel(M, Mr) <= 1e-5 and rel(J, Jr) <= 1e-5, (rel(M, Mr), rel(J, Jr))
 
 
+@pytest.mark.parametrize("w", SMALL_CASES, ids=lambda w: w.name)
+def test_frame_invert(w):
+    full = _full(w)
+    Ar, _ = _stats_ref(w, full)
+    s = vdn.shape_for(w)
+    W = torch.empty((w.B, w.H, w.T, w.d, w.d), device="cuda")
+    info = torch.ones(1, dtype=torch.int32, device="cuda")
+    vdn.vdn_frame_invert(s, to_dev(Ar), W, info)
+    torch.cuda.synchronize()
+    assert int(info.item()) == 0
+    ref = np.linalg.inv(np.eye(w.d) + Ar)
+    assert rel(W, ref) <= 1e-5, rel(W, ref)
+    Wc = W.double().cpu().numpy()
+    assert np.allclose(Wc, np.swapaxes(Wc, -1, -2), rtol=0, atol=1e-6)
+
+
 def _maps_ref(w, full):
     C = w.C
     out = [np.zeros((w.B, w.H, C, w.d, w.d)) for _ in range(4)]
@@ -242,6 +258,21 @@ def test_no_frame_outside_window_reads_text_state():
         ST = oracle.text_state(full["Kx"][0, h], full["Vx"][0, h], 1.0)
         ref = np.einsum("tuk,vk->tuv", full["Q"][0, h].astype(np.float64), ST)
         assert rel(fw.O[0, h], ref) <= 3e-3
+
+
+@pytest.mark.parametrize("d", [16, 128])
+def test_nonpositive_pivot_is_reported_by_invert(d):
+    w = custom("poison_inv", index=47, dtype="f32", d=d, T=9, anchors=0)
+    full = _full(w)
+    Ar, _ = _stats_ref(w, full)
+    Ar[0, 1, 4, 2, 2] = -7.0      # (b=0, h=1, t=4): linear index 13
+    Ar[0, 1, 7, 5, 5] = np.inf    # (0, 1, 7): 16
+    s = vdn.shape_for(w)
+    W = torch.empty((w.B, w.H, w.T, w.d, w.d), device="cuda")
+    info = torch.zeros(1, dtype=torch.int32, device="cuda")
+    vdn.vdn_frame_invert(s, to_dev(Ar), W, info)
+    torch.cuda.synchronize()
+    assert int(info.item()) == 1 + 13
 
 
 def test_nonpositive_pivot_is_reported():
