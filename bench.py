@@ -271,6 +271,10 @@ def main():
     assert int(info.item()) == 0, f"device status {int(info.item())}"
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    for e in evs:  # torch creates the CUDA event on its first record
+        for x in e:
+            x.record(stream)
+    torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ

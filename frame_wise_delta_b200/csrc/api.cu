@@ -182,7 +182,7 @@ vdn_status run_text_state(const Geo &g, const void *Kx, const void *Vx, const fl
     uint8_t *Wimg = (uint8_t *)(ws + L.wimg);
     VDN_CUDA(launch_invert_simt(Ax, nullptr, Wimg, info, g.BH, g.D, st), "text invert");
     VDN_CUDA(launch_compose_tc(Wimg, Bx, Ax, nullptr, S_T, nullptr, nullptr, nullptr, g.BH, 1, 1, 0,
-                               /*parts=*/2, /*ndirs=*/1, info, st),
+                               /*ndirs=*/1, info, st),
              "text injection");
   } else {
     VDN_CUDA(launch_factor_simt(Ax, Bx, nullptr, nullptr, S_T, info, g.BH, 1, 0, g.D, st),
@@ -460,8 +460,9 @@ vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K, const v
   VDN_TRY(mark(3));
   if (frames) {
     if (tc) {
-      VDN_CUDA(launch_compose_tc(Wimg, Bm, alpha, Mf, Jf, Mb, Jb, Mimg, g.BH, g.T, g.chunk, g.anchors,
-                                 3, 2, info, st),
+      // the fp32 Mc are not needed here: the scan reads their images
+      VDN_CUDA(launch_compose_tc(Wimg, Bm, alpha, nullptr, Jf, nullptr, Jb, Mimg, g.BH, g.T, g.chunk,
+                                 g.anchors, 2, info, st),
                "compose");
     } else {
       VDN_CUDA(launch_compose_simt(A, Bm, Mf, Jf, Mb, Jb, g.BH, g.T, g.chunk, g.D, st), "compose");
@@ -469,7 +470,7 @@ vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K, const v
   }
   VDN_TRY(mark(4));
   if (tc && frames) {
-    VDN_CUDA(launch_scan_tc(Mimg, Jf, Jb, S_T, Fo, Go, g.BH, g.C, 3, info, st), "scan");
+    VDN_CUDA(launch_scan_tc(Mimg, Jf, Jb, S_T, Fo, Go, g.BH, g.C, info, st), "scan");
   } else {
     VDN_CUDA(launch_scan_simt(Mf, Jf, Mb, Jb, S_T, Fo, Go, g.BH, g.C, g.D, 3, st), "scan");
   }

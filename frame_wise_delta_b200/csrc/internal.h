@@ -36,17 +36,16 @@ cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, voi
 // images of kImgBytes per frame, d = 128 only), each optional.
 cudaError_t launch_invert_simt(const float *A, float *W, uint8_t *Wimg, int32_t *info,
                                long long nframes, int D, cudaStream_t st);
-// Chunk maps from W images (tensor cores, d = 128). parts: bit 0 the M-chain
-// (writes Mf/Mb and, if Mimg, their images), bit 1 the J-chain (Jf/Jb);
-// ndirs = 1 runs the forward direction only.
+// Chunk maps from W images (tensor cores, d = 128): per (direction, b*h,
+// chunk) the M-chain (Mf/Mb, and their images if Mimg) and the J-chain
+// (Jf/Jb); any output pointer may be NULL. ndirs = 1 runs the forward
+// direction only.
 cudaError_t launch_compose_tc(const uint8_t *Wimg, const float *Bm, const float *alpha, float *Mf,
                               float *Jf, float *Mb, float *Jb, uint8_t *Mimg, long long BH, int T,
-                              int chunk, int anchors, int parts, int ndirs, int32_t *info,
-                              cudaStream_t st);
-// Bidirectional scan from Mc images and fp32 Jc (tensor cores, d = 128).
+                              int chunk, int anchors, int ndirs, int32_t *info, cudaStream_t st);
+// Both scans from Mc images and fp32 Jc (tensor cores, d = 128).
 cudaError_t launch_scan_tc(const uint8_t *Mimg, const float *Jf, const float *Jb, const float *S_T,
-                           float *F, float *G, long long BH, int C, int dir_mask, int32_t *info,
-                           cudaStream_t st);
+                           float *F, float *G, long long BH, int C, int32_t *info, cudaStream_t st);
 
 // Message returned by vdn_last_error() on this thread.
 void set_last_error(const char *msg);

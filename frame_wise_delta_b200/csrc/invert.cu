@@ -50,61 +50,61 @@ __global__ void __launch_bounds__(kThreads) invert_sweep_kernel(const float *__r
     }
 
   bool bad = false;
+  // Pivot block kb is a compile-time constant (outer loop unrolled), so the
+  // pivot row/column registers X[.][kb], X[kb][.] are addressed statically and
+  // only the lanes that own them act on them; the 8 pivots of a block run in
+  // an ordinary loop.
+#pragma unroll
+  for (int kb = 0; kb < R; ++kb) {
 #pragma unroll 1
-  for (int k = 0; k < D; ++k) {
-    float *c = cbuf[k & 1];
-    const int kb = k / kGrid, kr = k % kGrid;
-    // publish c_x = G[x][k] for all x (column k below/at the diagonal block,
-    // row k to its left)
+    for (int kr = 0; kr < kGrid; ++kr) {
+      const int k = kb * kGrid + kr;
+      float *c = cbuf[k & 1];
+      // publish c_x = G[x][k] for all x: column k at and below the diagonal
+      // block (lanes with cg == kr), row k to its left (lanes with rg == kr)
+      if (cg == kr) {
 #pragma unroll
-    for (int b = 0; b < R; ++b)
-      if (b == kb && cg == kr) {
+        for (int a = kb; a < R; ++a) c[rg * R + a] = X[a][kb];
+      }
+      if (rg == kr) {
 #pragma unroll
-        for (int a = b; a < R; ++a) c[rg * R + a] = X[a][b];
+        for (int b = 0; b < kb; ++b) c[cg * R + b] = X[kb][b];
+      }
+      __syncthreads();
+      const float piv = c[kr * R + kb];
+      bad |= !(piv > 0.f) || !isfinite(piv);
+      const float rp = 1.0f / piv;
+      float ci[R], cj[R];
+      if constexpr (R % 4 == 0) {
+#pragma unroll
+        for (int a = 0; a < R; a += 4) {
+          const float4 v = *reinterpret_cast<const float4 *>(&c[rg * R + a]);
+          ci[a] = v.x; ci[a + 1] = v.y; ci[a + 2] = v.z; ci[a + 3] = v.w;
+          const float4 w = *reinterpret_cast<const float4 *>(&c[cg * R + a]);
+          cj[a] = w.x * rp; cj[a + 1] = w.y * rp; cj[a + 2] = w.z * rp; cj[a + 3] = w.w * rp;
+        }
+      } else {
+#pragma unroll
+        for (int a = 0; a < R; ++a) {
+          ci[a] = c[rg * R + a];
+          cj[a] = c[cg * R + a] * rp;
+        }
       }
 #pragma unroll
-    for (int a = 0; a < R; ++a)
-      if (a == kb && rg == kr) {
+      for (int a = 0; a < R; ++a)
 #pragma unroll
-        for (int b = 0; b < a; ++b) c[cg * R + b] = X[a][b];
+        for (int b = 0; b <= a; ++b) X[a][b] = fmaf(-ci[a], cj[b], X[a][b]);
+      // row/column k: G[x][k] / piv, and the pivot -> -1/piv
+      if (cg == kr) {
+#pragma unroll
+        for (int a = kb; a < R; ++a) X[a][kb] = ci[a] * rp;
       }
-    __syncthreads();
-    const float piv = c[kr * R + kb];
-    bad |= !(piv > 0.f) || !isfinite(piv);
-    const float rp = 1.0f / piv;
-    float ci[R], cj[R];
-    if constexpr (R % 4 == 0) {
+      if (rg == kr) {
 #pragma unroll
-      for (int a = 0; a < R; a += 4) {
-        const float4 v = *reinterpret_cast<const float4 *>(&c[rg * R + a]);
-        ci[a] = v.x; ci[a + 1] = v.y; ci[a + 2] = v.z; ci[a + 3] = v.w;
-        const float4 w = *reinterpret_cast<const float4 *>(&c[cg * R + a]);
-        cj[a] = w.x * rp; cj[a + 1] = w.y * rp; cj[a + 2] = w.z * rp; cj[a + 3] = w.w * rp;
-      }
-    } else {
-#pragma unroll
-      for (int a = 0; a < R; ++a) {
-        ci[a] = c[rg * R + a];
-        cj[a] = c[cg * R + a] * rp;
+        for (int b = 0; b < kb; ++b) X[kb][b] = cj[b];
+        X[kb][kb] = (cg == kr) ? -rp : cj[kb];
       }
     }
-#pragma unroll
-    for (int a = 0; a < R; ++a)
-#pragma unroll
-      for (int b = 0; b <= a; ++b) X[a][b] = fmaf(-ci[a], cj[b], X[a][b]);
-    // row/column k: G[x][k] / piv, and the pivot -> -1/piv
-#pragma unroll
-    for (int b = 0; b < R; ++b)
-      if (b == kb && cg == kr) {
-#pragma unroll
-        for (int a = b; a < R; ++a) X[a][b] = ci[a] * rp;
-      }
-#pragma unroll
-    for (int a = 0; a < R; ++a)
-      if (a == kb && rg == kr) {
-#pragma unroll
-        for (int b = 0; b <= a; ++b) X[a][b] = (b == kb && cg == kr) ? -rp : cj[b];
-      }
   }
   if (bad && threadIdx.x == 0) report_frame_failure(info, f);
 

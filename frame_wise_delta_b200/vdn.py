@@ -195,11 +195,15 @@ def vdn_forward_workspace_bytes(s) -> int:
 
 def vdn_forward(s, Q, K, V, beta, alpha, Kx, Vx, beta_x, O, F, G, workspace, info, events=None,
                 stream=None):
-    """events: None or 7 torch.cuda.Event (enable_timing) recorded between the stages."""
+    """events: None or 7 torch.cuda.Event (enable_timing, already recorded once so
+    that their CUDA handles exist) recorded by the library between the stages."""
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     ev = None
     if events is not None:
-        arr = (ctypes.c_void_p * 7)(*[e.cuda_event if e is not None else None for e in events])
+        handles = [e.cuda_event if e is not None else None for e in events]
+        if any(e is not None and not h for e, h in zip(events, handles)):
+            raise VdnError(VDN_ERR_INVALID, "stage events must have been recorded once (no CUDA handle yet)")
+        arr = (ctypes.c_void_p * 7)(*handles)
         ev = ctypes.cast(arr, ctypes.c_void_p)
     _check(lib().vdn_forward(_shp(s), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(alpha), _ptr(Kx),
                              _ptr(Vx), _ptr(beta_x), _ptr(O), _ptr(F), _ptr(G), _ptr(workspace), nbytes,
