@@ -211,14 +211,18 @@ __global__ void __launch_bounds__(kThreads, 1) chain_tc_kernel(ChainArgs p) {
     if (MODE == kScan) {
       const float *st = p.S_T + bh * DD + m;
       float *o = (dir == 0 ? p.F + (bh * (p.C + 1)) * DD : p.G + (bh * (p.C + 1) + p.C) * DD) + m;
-#pragma unroll 1
-      for (int n0 = row0; n0 < row0 + kRows; n0 += 32) {
+      float x0[kRows];  // every load first: one memory latency, not one per block
+#pragma unroll
+      for (int e = 0; e < kRows; ++e) x0[e] = 0.5f * st[(row0 + e) * kD];
+#pragma unroll
+      for (int j = 0; j < kRows / 32; ++j) {
         float v[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = 0.5f * st[(n0 + e) * kD];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[(n0 + e) * kD] = v[e];
-        if (nsteps > 0) write_img32(eimg, m, n0, v, kImgRegion, kEHalf);
+        for (int e = 0; e < 32; ++e) {
+          v[e] = x0[32 * j + e];
+          o[(row0 + 32 * j + e) * kD] = v[e];
+        }
+        if (nsteps > 0) write_img32(eimg, m, row0 + 32 * j, v, kImgRegion, kEHalf);
       }
     } else {
       const long long cidx = bh * p.C + c_cmp;
@@ -233,17 +237,17 @@ __global__ void __launch_bounds__(kThreads, 1) chain_tc_kernel(ChainArgs p) {
       } else {
         const float al = p.alpha[(bh * p.T + frames[0]) * kD + m];
         const float *Bt = p.Bm + (bh * p.T + frames[0]) * DD + m;
-#pragma unroll 1
-        for (int n0 = 0; n0 < kD; n0 += 32) {
+        float b0[kD];  // every load first: one memory latency, not one per block
+        if (h == 1) {
+#pragma unroll
+          for (int e = 0; e < kD; ++e) b0[e] = Bt[e * kD];
+        }
+#pragma unroll
+        for (int j = 0; j < kD / 32; ++j) {
           float v[32];
-          if (h == 0) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = (n0 + e == m) ? al : 0.f;
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = Bt[(n0 + e) * kD];
-          }
-          write_img32(eimg, m, tcol0 + n0, v, kImgRegion, kEHalf);
+          for (int e = 0; e < 32; ++e) v[e] = h == 0 ? ((32 * j + e == m) ? al : 0.f) : b0[32 * j + e];
+          write_img32(eimg, m, tcol0 + 32 * j, v, kImgRegion, kEHalf);
         }
       }
     }

@@ -12,8 +12,9 @@
 // symmetric positive definite with eigenvalues >= 1, so every pivot is
 // positive and no pivoting is needed. The matrix stays symmetric, so only
 // the lower block-triangle is kept: 64 threads on an 8 x 8 grid own the
-// elements (rg + 8a, cg + 8b) with a >= b (136 registers each), which is
-// half the work of a full Gauss-Jordan and spreads it evenly. Each step
+// elements (rg + 8a, cg + 8b) with a >= b (136 values each, held as float2
+// pairs for the packed fp32x2 FMA of sm_100), which is half the work of a
+// full Gauss-Jordan and spreads it evenly. Each step
 // publishes pivot row k into a shared vector (stored interleaved so that a
 // thread's eight-apart entries are contiguous), applies one rank-1 update to
 // every owned element, then rewrites row/column k. A non-positive or
@@ -40,13 +41,19 @@ __global__ void __launch_bounds__(kThreads) invert_sweep_kernel(const float *__r
   const int rg = threadIdx.x / kGrid, cg = threadIdx.x % kGrid;
   const float *Af = A + f * (long long)D * D;
 
-  float X[R][R];  // only a >= b is used
+  // X(a, b) for a >= b: full pairs of block columns (b = 2q, 2q + 1 <= a) as
+  // float2, so the rank-1 update runs as packed fp32x2 FMAs, and the
+  // diagonal block of even rows (b = a) as a scalar: 136 values, no padding.
+  constexpr int P = (R + 1) / 2;
+  float2 XP[R][P];
+  float XS[P];
+#define XE(a, b) ((((a) & 1) == 0 && (b) == (a)) ? XS[(a) >> 1] : (((b) & 1) ? XP[a][(b) >> 1].y : XP[a][(b) >> 1].x))
 #pragma unroll
   for (int a = 0; a < R; ++a)
 #pragma unroll
     for (int b = 0; b <= a; ++b) {
       const int i = rg + kGrid * a, j = cg + kGrid * b;
-      X[a][b] = Af[i * D + j] + (i == j ? 1.f : 0.f);
+      XE(a, b) = Af[i * D + j] + (i == j ? 1.f : 0.f);
     }
 
   bool bad = false;
@@ -64,45 +71,51 @@ __global__ void __launch_bounds__(kThreads) invert_sweep_kernel(const float *__r
       // block (lanes with cg == kr), row k to its left (lanes with rg == kr)
       if (cg == kr) {
 #pragma unroll
-        for (int a = kb; a < R; ++a) c[rg * R + a] = X[a][kb];
+        for (int a = kb; a < R; ++a) c[rg * R + a] = XE(a, kb);
       }
       if (rg == kr) {
 #pragma unroll
-        for (int b = 0; b < kb; ++b) c[cg * R + b] = X[kb][b];
+        for (int b = 0; b < kb; ++b) c[cg * R + b] = XE(kb, b);
       }
       __syncthreads();
       const float piv = c[kr * R + kb];
       bad |= !(piv > 0.f) || !isfinite(piv);
       const float rp = 1.0f / piv;
-      float ci[R], cj[R];
+      // c_i for this thread's rows is read from shared memory where it is
+      // used (keeps the 144 matrix values plus cj2 within the register file)
+      const float *ci = &c[rg * R];
+      float2 cj2[P];  // c_j / piv for this thread's columns, as pairs
       if constexpr (R % 4 == 0) {
+        const float2 rp2 = make_float2(rp, rp);
 #pragma unroll
         for (int a = 0; a < R; a += 4) {
-          const float4 v = *reinterpret_cast<const float4 *>(&c[rg * R + a]);
-          ci[a] = v.x; ci[a + 1] = v.y; ci[a + 2] = v.z; ci[a + 3] = v.w;
           const float4 w = *reinterpret_cast<const float4 *>(&c[cg * R + a]);
-          cj[a] = w.x * rp; cj[a + 1] = w.y * rp; cj[a + 2] = w.z * rp; cj[a + 3] = w.w * rp;
+          cj2[a / 2] = __fmul2_rn(make_float2(w.x, w.y), rp2);
+          cj2[a / 2 + 1] = __fmul2_rn(make_float2(w.z, w.w), rp2);
         }
       } else {
 #pragma unroll
-        for (int a = 0; a < R; ++a) {
-          ci[a] = c[rg * R + a];
-          cj[a] = c[cg * R + a] * rp;
-        }
+        for (int q = 0; q < P; ++q)
+          cj2[q] = make_float2(c[cg * R + 2 * q] * rp, (2 * q + 1 < R) ? c[cg * R + 2 * q + 1] * rp : 0.f);
       }
+#define CJ(b) (((b) & 1) ? cj2[(b) >> 1].y : cj2[(b) >> 1].x)
 #pragma unroll
-      for (int a = 0; a < R; ++a)
+      for (int a = 0; a < R; ++a) {
+        const float nc = -ci[a];
+        const float2 na = make_float2(nc, nc);
 #pragma unroll
-        for (int b = 0; b <= a; ++b) X[a][b] = fmaf(-ci[a], cj[b], X[a][b]);
+        for (int q = 0; q < (a + 1) / 2; ++q) XP[a][q] = __ffma2_rn(na, cj2[q], XP[a][q]);
+        if ((a & 1) == 0) XS[a >> 1] = fmaf(nc, CJ(a), XS[a >> 1]);
+      }
       // row/column k: G[x][k] / piv, and the pivot -> -1/piv
       if (cg == kr) {
 #pragma unroll
-        for (int a = kb; a < R; ++a) X[a][kb] = ci[a] * rp;
+        for (int a = kb; a < R; ++a) XE(a, kb) = ci[a] * rp;
       }
       if (rg == kr) {
 #pragma unroll
-        for (int b = 0; b < kb; ++b) X[kb][b] = cj[b];
-        X[kb][kb] = (cg == kr) ? -rp : cj[kb];
+        for (int b = 0; b < kb; ++b) XE(kb, b) = CJ(b);
+        XE(kb, kb) = (cg == kr) ? -rp : CJ(kb);
       }
     }
   }
@@ -116,8 +129,8 @@ __global__ void __launch_bounds__(kThreads) invert_sweep_kernel(const float *__r
 #pragma unroll
       for (int b = 0; b <= a; ++b) {
         const int i = rg + kGrid * a, j = cg + kGrid * b;
-        Wf[i * D + j] = -X[a][b];
-        if (a != b) Wf[j * D + i] = -X[a][b];
+        Wf[i * D + j] = -XE(a, b);
+        if (a != b) Wf[j * D + i] = -XE(a, b);
       }
   }
   if constexpr (D == 128) {
@@ -128,11 +141,13 @@ __global__ void __launch_bounds__(kThreads) invert_sweep_kernel(const float *__r
 #pragma unroll
         for (int b = 0; b <= a; ++b) {
           const int i = rg + kGrid * a, j = cg + kGrid * b;
-          img_store(img, i, j, -X[a][b]);
-          if (a != b) img_store(img, j, i, -X[a][b]);
+          img_store(img, i, j, -XE(a, b));
+          if (a != b) img_store(img, j, i, -XE(a, b));
         }
     }
   }
+#undef CJ
+#undef XE
 }
 
 }  // namespace
