@@ -14,7 +14,7 @@
 //     X <- (X Diag(alpha_t) + [0 ; B_t]) W_t,    X_0 = [I ; 0]
 //  and ends as [Mc ; Jc]. This equals X M_t + [0 ; J_t] with
 //  M_t = Diag(alpha_t) W_t and J_t = B_t W_t, so the per-frame (M_t, J_t) are
-//  never materialised. One N = 256 MMA stream per step.
+//  never materialised. The M and J rows are independent groups of N = 128.
 //
 //  scan, one CTA per (b*h, direction): X <- X Mc_c + Jc_c over the chunks,
 //  from X = S_T / 2, writing every boundary state (N = 128).
@@ -30,8 +30,12 @@
 // consecutive floats of one state row).
 //
 // Roles (288 threads): warps 0..7 are the epilogue (warp w drains TMEM lanes
-// 32(w%4)..+31 for column half w/4); warp 8 allocates TMEM and one lane
-// issues the bulk copies and the MMAs. Every wait is bounded.
+// 32(w%4)..+31 for column half w/4; for the compose, half 0 is the M group and
+// half 1 the J group, each with its own TMEM accumulator and barriers, so the
+// epilogue of one group overlaps the MMAs of the other); warp 8 allocates TMEM
+// and one lane issues the bulk copies and the MMAs. The epilogue's fp32 work
+// and bf16 splits use packed fp32x2 / bf16x2 instructions. Every wait is
+// bounded.
 #include "common.cuh"
 #include "internal.h"
 
@@ -64,6 +68,17 @@ __device__ __forceinline__ void fail(volatile int *abort, int32_t *info) {
   if (info) atomicExch(info, VDN_INFO_TIMEOUT);
 }
 
+// bf16 hi/lo split of two values with packed instructions: hi = bf16x2(a, b),
+// lo = bf16x2 of the fp32 remainders.
+__device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t &lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const float2 hf = __bfloat1622float2(h);
+  const float2 r = __fadd2_rn(make_float2(a, b), make_float2(-hf.x, -hf.y));
+  const __nv_bfloat162 l = __floats2bfloat162_rn(r.x, r.y);
+  hi = *reinterpret_cast<const uint32_t *>(&h);
+  lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
 // Write 32 consecutive values (columns x0 .. x0+31 of image row rr) of an
 // MN-major hi/lo image in shared memory whose 64-column regions are `region`
 // bytes apart and whose hi and lo halves are `half` bytes apart.
@@ -71,16 +86,14 @@ __device__ __forceinline__ void write_img32(uint8_t *img, int rr, int x0, const 
                                             uint32_t region, uint32_t half) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    __nv_bfloat16 h[8], l[8];
+    uint32_t h[4], l[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) split_bf16(v[q * 8 + e], h[e], l[e]);
+    for (int e = 0; e < 4; ++e) split2(v[q * 8 + 2 * e], v[q * 8 + 2 * e + 1], h[e], l[e]);
     const int x = x0 + q * 8;
     const uint32_t off = (uint32_t)(x >> 6) * region + (uint32_t)rr * 128u +
                          ((((uint32_t)(x & 63) >> 3) ^ (uint32_t)(rr & 7)) << 4);
-    *reinterpret_cast<uint4 *>(img + off) =
-        make_uint4(pack2(h[0], h[1]), pack2(h[2], h[3]), pack2(h[4], h[5]), pack2(h[6], h[7]));
-    *reinterpret_cast<uint4 *>(img + half + off) =
-        make_uint4(pack2(l[0], l[1]), pack2(l[2], l[3]), pack2(l[4], l[5]), pack2(l[6], l[7]));
+    *reinterpret_cast<uint4 *>(img + off) = make_uint4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint4 *>(img + half + off) = make_uint4(l[0], l[1], l[2], l[3]);
   }
 }
 
@@ -95,10 +108,17 @@ __global__ void __launch_bounds__(kThreads, 1) chain_tc_kernel(ChainArgs p) {
   uint8_t *eimg = smem;                              // 2 * kEHalf bytes
   uint8_t *opbase = smem + 2 * kEHalf;               // compose: 1 buffer, scan: 2
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 3 * kImgBytes);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
   volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  const uint32_t ready = smem_u32(bars), done = ready + 8, drain = ready + 16;
-  const uint32_t opfull0 = ready + 24;  // opfull[b]
+  // Independent row groups: compose runs the M rows and the J rows as two
+  // groups (each N = 128) so one group's epilogue overlaps the other's MMAs;
+  // the scan is one group.
+  constexpr int NG = MODE == kCompose ? 2 : 1;
+  constexpr int kGroupWorkers = kWorkers / NG;
+  const uint32_t ready0 = smem_u32(bars);  // ready[g]
+  const uint32_t done0 = ready0 + 16;      // done[g]
+  const uint32_t opfull0 = ready0 + 32;    // opfull[b]
+  const uint32_t drain = ready0 + 48;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long DD = (long long)kD * kD;
@@ -130,11 +150,12 @@ __global__ void __launch_bounds__(kThreads, 1) chain_tc_kernel(ChainArgs p) {
   constexpr int kBufs = MODE == kCompose ? 1 : 2;
 
   if (threadIdx.x == 0) {
-    mbar_init(ready, kWorkers);
-    mbar_init(done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(ready0 + 8 * i, kGroupWorkers);
+      mbar_init(done0 + 8 * i, 1);
+      mbar_init(opfull0 + 8 * i, 1);
+    }
     mbar_init(drain, 1);
-    mbar_init(opfull0, 1);
-    mbar_init(opfull0 + 8, 1);
     *abort = 0;
     fence_barrier_init();
   }
@@ -146,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_tc_kernel(ChainArgs p) {
 
   if (warp == 8) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, N, true, true);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, true, true);
       const uint32_t e_hi = smem_u32(eimg), e_lo = e_hi + kEHalf;
       auto load = [&](int s) {
         const int b = s % kBufs;
@@ -160,31 +181,40 @@ __global__ void __launch_bounds__(kThreads, 1) chain_tc_kernel(ChainArgs p) {
       };
       int loads = 0;
       for (; loads < kBufs && loads < nsteps; ++loads) load(loads);
-      for (int s = 0; s < nsteps; ++s) {
+      bool ok = true;
+      for (int s = 0; ok && s < nsteps; ++s) {
         const int b = s % kBufs;
-        const uint32_t par = (uint32_t)((s / kBufs) & 1);
-        if (!mbar_wait(opfull0 + 8 * b, par, abort) || !mbar_wait(ready, (uint32_t)(s & 1), abort)) {
+        if (!mbar_wait(opfull0 + 8 * b, (uint32_t)((s / kBufs) & 1), abort)) {
           fail(abort, p.info);
           break;
         }
-        tc_fence_after();
         const uint32_t o_hi = smem_u32(opbase + b * kImgBytes), o_lo = o_hi + kImgHalf;
-#pragma unroll
-        for (int part = 0; part < 3; ++part) {
-          const uint32_t a0 = part == 2 ? o_lo : o_hi;
-          const uint32_t b0 = part == 1 ? e_lo : e_hi;
-#pragma unroll
-          for (int ks = 0; ks < kD / 16; ++ks) {
-            const uint64_t ad = smem_desc_sw128(a0 + ks * 2048, kImgRegion, 1024);
-            const uint64_t bd = smem_desc_sw128(b0 + ks * 2048, kImgRegion, 1024);
-            tc_mma_bf16(tmem_base, ad, bd, idesc, (part > 0 || ks > 0) ? 1u : 0u);
+        for (int g = 0; g < NG; ++g) {
+          if (!mbar_wait(ready0 + 8 * g, (uint32_t)(s & 1), abort)) {
+            fail(abort, p.info);
+            ok = false;
+            break;
           }
+          tc_fence_after();
+          // group g: state rows 128g.. (E image regions 2g, 2g+1), TMEM columns 128g..
+          const uint32_t eg_hi = e_hi + (uint32_t)(g * 2 * kImgRegion), eg_lo = e_lo + (uint32_t)(g * 2 * kImgRegion);
+#pragma unroll
+          for (int part = 0; part < 3; ++part) {
+            const uint32_t a0 = part == 2 ? o_lo : o_hi;
+            const uint32_t b0 = part == 1 ? eg_lo : eg_hi;
+#pragma unroll
+            for (int ks = 0; ks < kD / 16; ++ks) {
+              const uint64_t ad = smem_desc_sw128(a0 + ks * 2048, kImgRegion, 1024);
+              const uint64_t bd = smem_desc_sw128(b0 + ks * 2048, kImgRegion, 1024);
+              tc_mma_bf16(tmem_base + (uint32_t)(128 * g), ad, bd, idesc, (part > 0 || ks > 0) ? 1u : 0u);
+            }
+          }
+          tc_commit(done0 + 8 * g);
         }
-        tc_commit(done);
-        if (loads < nsteps) {
+        if (ok && loads < nsteps) {
           // the next load (step s + kBufs) reuses this step's buffer: wait for
-          // these MMAs to finish reading it
-          if (!mbar_wait(done, (uint32_t)(s & 1), abort)) {
+          // the MMAs of the last group (hence of every group) to finish
+          if (!mbar_wait(done0 + 8 * (NG - 1), (uint32_t)(s & 1), abort)) {
             fail(abort, p.info);
             break;
           }
@@ -201,7 +231,8 @@ __global__ void __launch_bounds__(kThreads, 1) chain_tc_kernel(ChainArgs p) {
   } else {
     // ---- epilogue: thread owns state column m (TMEM lane m) for column half h
     const int m = (warp & 3) * 32 + lane;
-    const int h = warp >> 2;                     // scan: rows 64h..64h+63; compose: part (0 M, 1 J)
+    const int h = warp >> 2;                     // scan: rows 64h..64h+63; compose: group (0 M, 1 J)
+    const int grp = MODE == kCompose ? h : 0;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     constexpr int kRows = MODE == kCompose ? 128 : 64;  // state rows handled per thread
     const int row0 = MODE == kCompose ? 0 : 64 * h;     // first state row of this thread
@@ -253,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_tc_kernel(ChainArgs p) {
     }
     if (nsteps > 0) {
       fence_proxy_async_smem();
-      mbar_arrive(ready);
+      mbar_arrive(ready0 + 8 * grp);
     }
 
     for (int s = 0; s < nsteps; ++s) {
@@ -281,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_tc_kernel(ChainArgs p) {
 #pragma unroll
         for (int e = 0; e < kRows; ++e) addv[e] = add[(row0 + e) * kD];
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(done, (uint32_t)(s & 1), abort))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(done0 + 8 * grp, (uint32_t)(s & 1), abort))) {
         fail(abort, p.info);
         break;
       }
@@ -299,7 +330,12 @@ __global__ void __launch_bounds__(kThreads, 1) chain_tc_kernel(ChainArgs p) {
           if (!last) write_img32(eimg, m, n0, v, kImgRegion, kEHalf);
         } else if (!last) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = v[e] * al + (add ? addv[32 * j + e] : 0.f);
+          for (int e = 0; e < 32; e += 2) {
+            const float2 r2 = __ffma2_rn(make_float2(v[e], v[e + 1]), make_float2(al, al),
+                                         add ? make_float2(addv[32 * j + e], addv[32 * j + e + 1]) : make_float2(0.f, 0.f));
+            v[e] = r2.x;
+            v[e + 1] = r2.y;
+          }
           write_img32(eimg, m, tcol0 + n0, v, kImgRegion, kEHalf);
         } else {
           if (o) {
@@ -315,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_tc_kernel(ChainArgs p) {
       if (!last) {
         tc_fence_before();
         fence_proxy_async_smem();
-        mbar_arrive(ready);
+        mbar_arrive(ready0 + 8 * grp);
       }
     }
   }
