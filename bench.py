@@ -31,8 +31,13 @@ FALLBACK_HBM_GBS = 6650.0
 # FP32 FMA peak: 148 SMs x 128 lanes x 2 flop x 1.965 GHz (max SM clock).
 ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum)
-# for the kernel as it stands; None until a capture of the current kernel.
-NCU_TRAFFIC = {}
+# at the H3 shape (profiles/launch_list_h3.md), keyed by stage, with the
+# sha256 prefix of the kernel source the counters were taken on; reported as
+# None as soon as that source changes.
+NCU_TRAFFIC = {
+    "frame_factor": {"bytes": 112.5e6 + 123.3e6, "source": "frame_wise_delta_b200/csrc/invert.cu",
+                     "sha256_16": "c731caa4fd644675", "workload": "h3"},
+}
 
 
 def parse():
@@ -412,7 +417,13 @@ def roofline(w, stage_ms, hbm_gbs, peak_src, bf16_tflops=1607.7):
         achieved = amount / sec / 1e12
         peak, unit = ALU_F32_TFLOPS, "TFLOP/s"
         src = "FP32 FMA: 148 SMs x 128 lanes x 2 flop x 1.965 GHz"
-    tr = NCU_TRAFFIC.get(name)
+    tr = None
+    rec = NCU_TRAFFIC.get(name)
+    if rec and rec["workload"] == w.name:
+        import hashlib
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest()[:16] == rec["sha256_16"]:
+                tr = rec["bytes"]
     return {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
             "frac": achieved / peak, "traffic": tr, "peak_source": src,
             "per_stage_ms": {k: round(v, 4) for k, v in stage_ms.items()}}
