@@ -228,6 +228,7 @@ def main():
     import torch.distributed as dist
 
     from frame_wise_delta_b200 import build, vdn
+    from frame_wise_delta_b200 import dist as vdist
 
     rank, world, local = dist_env()
     if world > 1:
@@ -291,13 +292,10 @@ def main():
     step_ms = [event_ms(e[0], e[6]) for e in evs]
     stage_ms = {name: statistics.mean(event_ms(e[j], e[j + 1]) for e in evs) for j, name in enumerate(stages)}
     total_ms = event_ms(evs[0][0], evs[-1][6])
-    t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = vdist.max_over_ranks(total_ms)  # the slowest rank's device time
     ms_per_step = total_ms / args.steps
     frames_all = world * B * T
-    value = frames_all / (ms_per_step / 1e3)
+    value = vdist.throughput(B * T, world, ms_per_step / 1e3)
 
     # ---- end to end: pinned host inputs -> device -> vdn_forward -> O to host
     e2e = e2e_measure(args, host, d, s, dev, stream, barrier, world, frames_all, dt) if not args.no_e2e else None
@@ -331,8 +329,8 @@ def e2e_measure(args, host, d, s, dev, stream, barrier, world, frames_all, dt):
     """Same metric through vdn_forward with the step's inputs copied from pinned
     host memory and O copied back, inside the timed region."""
     import torch
-    import torch.distributed as dist
 
+    from frame_wise_delta_b200 import dist as vdist
     from frame_wise_delta_b200 import vdn
 
     fwd = vdn.Forward(s, device=dev, keep_states=False)
@@ -359,11 +357,9 @@ def e2e_measure(args, host, d, s, dev, stream, barrier, world, frames_all, dt):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    te = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    te = vdist.max_over_ranks(e0.elapsed_time(e1))
     assert int(fwd.info.item()) == 0
-    return {"value": frames_all / (float(te.item()) / e2e_steps / 1e3), "unit": "frames/s",
+    return {"value": frames_all / (te / e2e_steps / 1e3), "unit": "frames/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
 
