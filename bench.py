@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--groups", type=int, default=1,
+                    help="head groups of vdn_forward_pipelined (tensor path); 0 = plain vdn_forward")
     return ap.parse_args()
 
 
@@ -258,17 +260,29 @@ def main():
     s = vdn.shape_for(w)
     B, H, T, U, D, C = w.B, w.H, w.T, w.U, w.d, w.C
     f32 = dict(dtype=torch.float32, device=dev)
-    fwd_dev = vdn.Forward(s, device=dev)
     stream = torch.cuda.current_stream()
 
     stages = ["text_state", "frame_grams", "frame_factor", "chunk_compose", "scan_bidir", "chunk_readout"]
     tensor_path = w.dtype == "bf16" and D == 128
+    G = min(args.groups, B * H) if tensor_path else 0
+
+    def make_forward(keep_states=True):
+        if G:
+            return vdn.PipelinedForward(s, groups=G, device=dev, keep_states=keep_states)
+        return vdn.Forward(s, device=dev, keep_states=keep_states)
+
+    fwd_dev = make_forward()
     # our kernels per step: text (gram, invert, injection chain) + gram +
-    # invert + compose (M and J chains) + scan + readout
-    launches_per_step = 9 if tensor_path else 7
+    # invert + compose (M and J chains) + scan + readout, per head group
+    launches_per_step = (6 + 2 * max(G, 1)) if tensor_path else 7
+    n_ev = 7 + 3 * G if G else 7
 
     def step(ev=None):
-        fwd_dev(d["Q"], d["K"], d["V"], d["beta"], d["alpha"], d["Kx"], d["Vx"], d["beta_x"], events=ev)
+        if G:
+            fwd_dev.events = ev if ev is not None else warm_ev
+        fwd_dev(d["Q"], d["K"], d["V"], d["beta"], d["alpha"], d["Kx"], d["Vx"], d["beta_x"],
+                events=None if G else ev)
+    warm_ev = fwd_dev.events if G else None
     info = fwd_dev.info
 
     for _ in range(max(3, args.warmup)):
@@ -276,7 +290,7 @@ def main():
     torch.cuda.synchronize()
     assert int(info.item()) == 0, f"device status {int(info.item())}"
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     for e in evs:  # torch creates the CUDA event on its first record
         for x in e:
             x.record(stream)
@@ -289,16 +303,23 @@ def main():
             step(evs[i])
         torch.cuda.synchronize()
     barrier()
-    step_ms = [event_ms(e[0], e[6]) for e in evs]
-    stage_ms = {name: statistics.mean(event_ms(e[j], e[j + 1]) for e in evs) for j, name in enumerate(stages)}
-    total_ms = event_ms(evs[0][0], evs[-1][6])
+    assert int(info.item()) == 0, f"device status {int(info.item())}"
+    first, last = 0, n_ev - 1
+    step_ms = [event_ms(e[first], e[last]) for e in evs]
+    if G:
+        stage_ms = {name: statistics.mean(pipelined_stage_ms(e, G)[name] for e in evs) for name in stages}
+    else:
+        stage_ms = {name: statistics.mean(event_ms(e[j], e[j + 1]) for e in evs)
+                    for j, name in enumerate(stages)}
+    total_ms = event_ms(evs[0][first], evs[-1][last])
     total_ms = vdist.max_over_ranks(total_ms)  # the slowest rank's device time
     ms_per_step = total_ms / args.steps
     frames_all = world * B * T
     value = vdist.throughput(B * T, world, ms_per_step / 1e3)
 
     # ---- end to end: pinned host inputs -> device -> vdn_forward -> O to host
-    e2e = e2e_measure(args, host, d, s, dev, stream, barrier, world, frames_all, dt) if not args.no_e2e else None
+    e2e = (e2e_measure(args, host, d, make_forward, stream, barrier, world, frames_all, dt)
+           if not args.no_e2e else None)
 
     if rank == 0:
         hbm_gbs, bf16_tflops, peak_src = load_peaks()
@@ -315,6 +336,7 @@ def main():
             "roofline": roof,
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
+            "head_groups": G,
             "clocks": clk.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -325,7 +347,23 @@ def main():
         dist.destroy_process_group()
 
 
-def e2e_measure(args, host, d, s, dev, stream, barrier, world, frames_all, dt):
+def pipelined_stage_ms(e, G):
+    """Per-stage device time of one vdn_forward_pipelined step from its 7 + 3 G
+    events, each stage timed on its own stream and summed over head groups;
+    the text state and the inverses run on the auxiliary stream beside the
+    Grams, so these overlap and add up to more than the step."""
+    t = 3 + 3 * G
+    out = {"text_state": event_ms(e[1], e[2]), "frame_grams": 0.0, "frame_factor": 0.0,
+           "chunk_compose": event_ms(e[t], e[t + 1]), "scan_bidir": event_ms(e[t + 1], e[t + 2]),
+           "chunk_readout": event_ms(e[t + 2], e[t + 3])}
+    for g in range(G):
+        b = 3 + 3 * g
+        out["frame_grams"] += event_ms(e[0] if g == 0 else e[b - 3], e[b])
+        out["frame_factor"] += event_ms(e[b + 1], e[b + 2])
+    return out
+
+
+def e2e_measure(args, host, d, make_forward, stream, barrier, world, frames_all, dt):
     """Same metric through vdn_forward with the step's inputs copied from pinned
     host memory and O copied back, inside the timed region."""
     import torch
@@ -333,7 +371,7 @@ def e2e_measure(args, host, d, s, dev, stream, barrier, world, frames_all, dt):
     from frame_wise_delta_b200 import dist as vdist
     from frame_wise_delta_b200 import vdn
 
-    fwd = vdn.Forward(s, device=dev, keep_states=False)
+    fwd = make_forward(keep_states=False)
     O_host = torch.empty(fwd.O.shape, dtype=dt).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = O_host.numel() * O_host.element_size()

@@ -480,4 +480,99 @@ vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K, const v
   return VDN_OK;
 }
 
+vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *K, const void *V,
+                                 const float *beta, const float *alpha, const void *Kx,
+                                 const void *Vx, const float *beta_x, void *O, float *F, float *G,
+                                 void *workspace, size_t workspace_bytes, int32_t *info,
+                                 int32_t groups, vdn_stream_t aux, const void *const *events,
+                                 vdn_stream_t stream) {
+  g_err[0] = 0;
+  Geo g;
+  VDN_TRY(check_shape(s, &g));
+  if (!tensor_path(g))
+    return fail(VDN_ERR_UNSUPPORTED, "the pipelined pass needs bf16 inputs and output and d = 128");
+  if (groups < 1 || groups > 64) return fail(VDN_ERR_INVALID, "groups = %d not in [1, 64]", groups);
+  if (!events) return fail(VDN_ERR_INVALID, "events is NULL");
+  for (int i = 0; i < 7 + 3 * groups; ++i)
+    if (!events[i]) return fail(VDN_ERR_INVALID, "events[%d] is NULL", i);
+  const bool frames = g.BH * g.T > 0;
+  VDN_TRY(need(Q, "Q", frames && g.U > 0));
+  VDN_TRY(need(K, "K", frames && g.U > 0));
+  VDN_TRY(need(V, "V", frames && g.U > 0));
+  VDN_TRY(need(beta, "beta", frames && g.U > 0));
+  VDN_TRY(need(alpha, "alpha", frames));
+  VDN_TRY(need(Kx, "Kx", g.BH > 0 && g.n_text > 0));
+  VDN_TRY(need(Vx, "Vx", g.BH > 0 && g.n_text > 0));
+  VDN_TRY(need(beta_x, "beta_x", g.BH > 0 && g.n_text > 0));
+  VDN_TRY(need(O, "O", frames && g.U > 0));
+  if ((F && !aligned16(F)) || (G && !aligned16(G)))
+    return fail(VDN_ERR_INVALID, "F/G not 16-byte aligned");
+  VDN_TRY(need(info, "info", true));
+  const FwdLayout L = fwd_layout(g);
+  VDN_TRY(need(workspace, "workspace", g.BH > 0));
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(VDN_ERR_INVALID, "workspace is not 256-byte aligned");
+  if (workspace_bytes < L.total)
+    return fail(VDN_ERR_INVALID, "workspace of %zu bytes < %zu required", workspace_bytes, L.total);
+
+  cudaStream_t st = (cudaStream_t)stream, ax = (cudaStream_t)aux;
+  auto ev = [&](int i) { return (cudaEvent_t)events[i]; };
+  char *w = (char *)workspace;
+  float *S_T = (float *)(w + L.st);
+  float *A = (float *)(w + L.a), *Bm = (float *)(w + L.b);
+  uint8_t *Wimg = (uint8_t *)(w + L.wimg), *Mimg = (uint8_t *)(w + L.mimg);
+  float *Jf = (float *)(w + L.jf), *Jb = (float *)(w + L.jb);
+  float *Fo = F ? F : (float *)(w + L.f);
+  float *Go = G ? G : (float *)(w + L.g);
+  const long long T = g.T, U = g.U, DD = (long long)g.D * g.D, D = g.D;
+  const int G_ = (int)(groups < g.BH ? groups : (g.BH > 0 ? g.BH : 1));
+  auto lo = [&](int gi) { return g.BH * gi / G_; };
+  auto tok = [&](const void *p, long long b0) { return (const char *)p + b0 * T * U * D * g.in_elem; };
+
+  VDN_CUDA(cudaMemsetAsync(info, 0, sizeof(int32_t), st), "memset info");
+  VDN_CUDA(cudaEventRecord(ev(0), st), "event record");
+  // the text state on the auxiliary stream, beside the first Grams
+  VDN_CUDA(cudaStreamWaitEvent(ax, ev(0), 0), "stream wait");
+  VDN_CUDA(cudaEventRecord(ev(1), ax), "event record");
+  VDN_TRY(run_text_state(g, Kx, Vx, beta_x, S_T, w + L.text, info, ax));
+  VDN_CUDA(cudaEventRecord(ev(2), ax), "event record");
+  // the Grams of every group on the main stream; each group's inverse on the
+  // auxiliary stream once its Grams are done, beside the next group's Grams
+  for (int gi = 0; gi < groups; ++gi) {
+    const int base = 3 + 3 * gi;
+    const bool run = gi < G_ && frames;
+    const long long b0 = run ? lo(gi) : 0, nbh = run ? lo(gi + 1) - b0 : 0;
+    if (run)
+      VDN_TRY(run_grams(g, tok(K, b0), tok(V, b0), beta + b0 * T, A + b0 * T * DD, Bm + b0 * T * DD, nbh * T,
+                        (int)U, info, st));
+    VDN_CUDA(cudaEventRecord(ev(base + 0), st), "event record");
+    VDN_CUDA(cudaStreamWaitEvent(ax, ev(base + 0), 0), "stream wait");
+    VDN_CUDA(cudaEventRecord(ev(base + 1), ax), "event record");
+    if (run)
+      VDN_CUDA(launch_invert_simt(A + b0 * T * DD, nullptr, Wimg + b0 * T * kImgBytes, info, nbh * T, g.D,
+                                  ax, b0 * T),
+               "invert");
+    VDN_CUDA(cudaEventRecord(ev(base + 2), ax), "event record");
+  }
+  // composition, scans and readout over all pairs once the auxiliary stream
+  // (text state and every inverse) is done: these are latency-bound chains
+  // whose time grows if they are split
+  const int tail = 3 + 3 * groups;
+  VDN_CUDA(cudaStreamWaitEvent(st, ev(tail - 1), 0), "stream wait");
+  VDN_CUDA(cudaEventRecord(ev(tail), st), "event record");
+  if (frames)
+    VDN_CUDA(launch_compose_tc(Wimg, Bm, alpha, nullptr, Jf, nullptr, Jb, Mimg, g.BH, g.T, g.chunk, g.anchors,
+                               2, info, st),
+             "compose");
+  VDN_CUDA(cudaEventRecord(ev(tail + 1), st), "event record");
+  if (frames)
+    VDN_CUDA(launch_scan_tc(Mimg, Jf, Jb, S_T, Fo, Go, g.BH, g.C, info, st), "scan");
+  else if (g.BH > 0)
+    VDN_CUDA(launch_scan_simt(nullptr, nullptr, nullptr, nullptr, S_T, Fo, Go, g.BH, g.C, g.D, 3, st), "scan");
+  VDN_CUDA(cudaEventRecord(ev(tail + 2), st), "event record");
+  if (frames) VDN_TRY(run_readout(g, Q, Fo, Go, O, info, st));
+  VDN_CUDA(cudaEventRecord(ev(tail + 3), st), "event record");
+  return VDN_OK;
+}
+
 }  // extern "C"

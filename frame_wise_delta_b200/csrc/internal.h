@@ -34,8 +34,9 @@ cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, voi
 
 // W = (I + A)^{-1} per frame (CUDA cores); W fp32 and/or Wimg (hi/lo MMA
 // images of kImgBytes per frame, d = 128 only), each optional.
+// frame_base: index of the first frame, for the failure index in *info.
 cudaError_t launch_invert_simt(const float *A, float *W, uint8_t *Wimg, int32_t *info,
-                               long long nframes, int D, cudaStream_t st);
+                               long long nframes, int D, cudaStream_t st, long long frame_base = 0);
 // Chunk maps from W images (tensor cores, d = 128): per (direction, b*h,
 // chunk) the M-chain (Mf/Mb, and their images if Mimg) and the J-chain
 // (Jf/Jb); any output pointer may be NULL. ndirs = 1 runs the forward

@@ -33,7 +33,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads) invert_sweep_kernel(const float *__restrict__ A,
                                                                 float *__restrict__ W,
                                                                 uint8_t *__restrict__ Wimg,
-                                                                int32_t *__restrict__ info) {
+                                                                int32_t *__restrict__ info,
+                                                                long long frame_base) {
   constexpr int R = D / kGrid;  // blocks per dimension
   // c[x] lives at slot (x % 8) * R + x / 8: a thread's entries rg + 8a are contiguous
   __shared__ __align__(16) float cbuf[2][D];
@@ -119,7 +120,7 @@ __global__ void __launch_bounds__(kThreads) invert_sweep_kernel(const float *__r
       }
     }
   }
-  if (bad && threadIdx.x == 0) report_frame_failure(info, f);
+  if (bad && threadIdx.x == 0) report_frame_failure(info, frame_base + f);
 
   // W = -X; write both triangles
   if (W) {
@@ -153,14 +154,14 @@ __global__ void __launch_bounds__(kThreads) invert_sweep_kernel(const float *__r
 }  // namespace
 
 cudaError_t launch_invert_simt(const float *A, float *W, uint8_t *Wimg, int32_t *info,
-                               long long nframes, int D, cudaStream_t st) {
+                               long long nframes, int D, cudaStream_t st, long long frame_base) {
   if (nframes <= 0) return cudaSuccess;
   if (Wimg && D != 128) return cudaErrorInvalidValue;
   switch (D) {
-    case 16: invert_sweep_kernel<16><<<(unsigned)nframes, kThreads, 0, st>>>(A, W, nullptr, info); break;
-    case 32: invert_sweep_kernel<32><<<(unsigned)nframes, kThreads, 0, st>>>(A, W, nullptr, info); break;
-    case 64: invert_sweep_kernel<64><<<(unsigned)nframes, kThreads, 0, st>>>(A, W, nullptr, info); break;
-    case 128: invert_sweep_kernel<128><<<(unsigned)nframes, kThreads, 0, st>>>(A, W, Wimg, info); break;
+    case 16: invert_sweep_kernel<16><<<(unsigned)nframes, kThreads, 0, st>>>(A, W, nullptr, info, frame_base); break;
+    case 32: invert_sweep_kernel<32><<<(unsigned)nframes, kThreads, 0, st>>>(A, W, nullptr, info, frame_base); break;
+    case 64: invert_sweep_kernel<64><<<(unsigned)nframes, kThreads, 0, st>>>(A, W, nullptr, info, frame_base); break;
+    case 128: invert_sweep_kernel<128><<<(unsigned)nframes, kThreads, 0, st>>>(A, W, Wimg, info, frame_base); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

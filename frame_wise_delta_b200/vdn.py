@@ -67,6 +67,7 @@ _SIGS = {
     "vdn_forward": [_P] * 13 + [ctypes.c_size_t, _P, _P, _P],
     "vdn_frame_invert": [_P, _P, _P, _P, _P],
     "vdn_text_state_noalloc": [_P, _P, _P, _P, _P, _P, _P],
+    "vdn_forward_pipelined": [_P] * 13 + [ctypes.c_size_t, _P, ctypes.c_int32, _P, _P, _P],
 }
 
 
@@ -210,6 +211,28 @@ def vdn_forward(s, Q, K, V, beta, alpha, Kx, Vx, beta_x, O, F, G, workspace, inf
                              _ptr(info), ev, _stream(stream)))
 
 
+def pipeline_events(groups: int):
+    """The 7 + 3 * groups timing events vdn_forward_pipelined records (created
+    here by torch and recorded once so that their CUDA handles exist)."""
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(7 + 3 * groups)]
+    for e in evs:
+        e.record()
+    return evs
+
+
+def vdn_forward_pipelined(s, Q, K, V, beta, alpha, Kx, Vx, beta_x, O, F, G, workspace, info, groups, aux,
+                          events, stream=None):
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    handles = [e.cuda_event for e in events]
+    if len(handles) < 7 + 3 * groups or not all(handles):
+        raise VdnError(VDN_ERR_INVALID, "need 7 + 3 * groups recorded events")
+    arr = (ctypes.c_void_p * len(handles))(*handles)
+    _check(lib().vdn_forward_pipelined(_shp(s), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(alpha), _ptr(Kx),
+                                       _ptr(Vx), _ptr(beta_x), _ptr(O), _ptr(F), _ptr(G), _ptr(workspace),
+                                       nbytes, _ptr(info), int(groups), _stream(aux),
+                                       ctypes.cast(arr, ctypes.c_void_p), _stream(stream)))
+
+
 def vdn_status_string(status: int) -> str:
     return lib().vdn_status_string(status).decode()
 
@@ -248,4 +271,19 @@ class Forward:
     def __call__(self, Q, K, V, beta, alpha, Kx, Vx, beta_x, events=None, stream=None):
         vdn_forward(self.s, Q, K, V, beta, alpha, Kx, Vx, beta_x, self.O, self.F, self.G, self.ws,
                     self.info, events, stream)
+        return self.O
+
+
+class PipelinedForward(Forward):
+    """vdn_forward_pipelined with its own auxiliary stream and events."""
+
+    def __init__(self, s: vdn_shape, groups: int = 3, device="cuda", keep_states=True):
+        super().__init__(s, device, keep_states)
+        self.groups = groups
+        self.aux = torch.cuda.Stream(device=device)
+        self.events = pipeline_events(groups)
+
+    def __call__(self, Q, K, V, beta, alpha, Kx, Vx, beta_x, events=None, stream=None):
+        vdn_forward_pipelined(self.s, Q, K, V, beta, alpha, Kx, Vx, beta_x, self.O, self.F, self.G, self.ws,
+                              self.info, self.groups, self.aux, self.events, stream)
         return self.O

@@ -116,3 +116,22 @@ def test_binding_refuses_host_tensors(L):
     x = torch.zeros(4)
     with pytest.raises(vdn.VdnError):
         vdn.vdn_frame_grams(s, x, x, x, x, x)
+
+
+def test_pipelined_validation(L):
+    s = _shape()  # float32, d = 16: not the tensor path
+    need = vdn.vdn_forward_workspace_bytes(s)
+    ev = (ctypes.c_void_p * 13)(*([16] * 13))
+    evp = ctypes.cast(ev, ctypes.c_void_p)
+    args = [_p(s)] + [16] * 11 + [256, need, 16]  # Q..O, F, G, workspace, bytes, info
+    assert L.vdn_forward_pipelined(*args, 2, None, evp, None) == vdn.VDN_ERR_UNSUPPORTED
+    s2 = _shape(d=128, in_dtype="bf16")
+    args[0] = _p(s2)
+    args[13] = vdn.vdn_forward_workspace_bytes(s2)
+    assert L.vdn_forward_pipelined(*args, 0, None, evp, None) == vdn.VDN_ERR_INVALID
+    assert "groups" in vdn.vdn_last_error()
+    assert L.vdn_forward_pipelined(*args, 2, None, None, None) == vdn.VDN_ERR_INVALID
+    assert "events" in vdn.vdn_last_error()
+    ev[9] = None  # 7 + 3 * 2 = 13 events, one missing
+    assert L.vdn_forward_pipelined(*args, 2, None, evp, None) == vdn.VDN_ERR_INVALID
+    assert "events[9]" in vdn.vdn_last_error()

@@ -1,0 +1,107 @@
+"""GPU parity of vdn_forward_pipelined: the fused pass split into head groups
+across two streams must give bit-for-bit the results of vdn_forward (every
+(b, h) pair runs the same kernels on the same data), and therefore the
+oracle's within the bf16 bound, for every group count, with ragged groups,
+degenerate shapes and a failing frame reported at its global index."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from frame_wise_delta_b200 import synth, vdn
+from vdn_testlib import TOL, device_fill, device_inputs, rel, run_forward
+
+pytestmark = pytest.mark.gpu
+
+
+def custom(name, **kw):
+    base = dict(name=name, index=50, B=1, H=5, T=12, U=300, d=128, n_text=40, dtype="bf16",
+                alpha_lo=0.9, anchors=1)
+    base.update(kw)
+    return synth.Workload(**base)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _build():
+    from frame_wise_delta_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+
+
+def _pipelined(w, dev, groups):
+    fw = vdn.PipelinedForward(vdn.shape_for(w), groups=groups)
+    fw(dev["Q"], dev["K"], dev["V"], dev["beta"], dev["alpha"], dev["Kx"], dev["Vx"], dev["beta_x"])
+    torch.cuda.synchronize()
+    return fw
+
+
+def _same(a, b):
+    return a is None and b is None or torch.equal(a, b)
+
+
+# 5 heads: groups 2 and 3 are ragged (3 + 2, 2 + 1 + 2), 7 > B*H clamps to one pair per group
+@pytest.mark.parametrize("groups", [1, 2, 3, 5, 7])
+def test_pipelined_equals_forward_and_oracle(groups):
+    w = custom("pipe5")
+    full = synth.generate_all(w)
+    dev = device_inputs(w, full)
+    ref = run_forward(w, dev)
+    fw = _pipelined(w, dev, groups)
+    assert int(fw.info.item()) == 0
+    assert torch.equal(fw.O, ref.O) and torch.equal(fw.F, ref.F) and torch.equal(fw.G, ref.G)
+    for h in range(w.H):
+        inp = {k: full[k][0, h] for k in full}
+        r = oracle.vda_head(inp, w.chunk, w.anchors)
+        assert rel(fw.O[0, h], r["O"]) <= TOL["bf16"]
+        assert rel(fw.F[0, h], r["F"]) <= TOL["bf16"] and rel(fw.G[0, h], r["G"]) <= TOL["bf16"]
+
+
+def test_pipelined_batches_and_near_duplicates():
+    w = custom("pipe_dup", index=51, B=3, H=2, T=23, U=200, n_text=17, near_dup=True)
+    full = synth.generate_all(w)
+    dev = device_inputs(w, full)
+    ref = run_forward(w, dev)
+    fw = _pipelined(w, dev, 4)
+    assert torch.equal(fw.O, ref.O) and torch.equal(fw.F, ref.F) and torch.equal(fw.G, ref.G)
+
+
+@pytest.mark.parametrize("kw", [dict(T=0), dict(U=0), dict(n_text=0), dict(B=0), dict(T=1), dict(T=3, U=1)],
+                         ids=lambda kw: "-".join(f"{k}{v}" for k, v in kw.items()))
+def test_pipelined_edge_shapes(kw):
+    w = custom("pipe_edge", index=52, **{"T": 7, "U": 33, "n_text": 6, **kw})
+    full = synth.generate_all(w)
+    dev = device_inputs(w, full)
+    ref = run_forward(w, dev)
+    fw = _pipelined(w, dev, 2)
+    assert int(fw.info.item()) == 0
+    assert torch.equal(fw.O, ref.O) and torch.equal(fw.F, ref.F) and torch.equal(fw.G, ref.G)
+
+
+def test_pipelined_reports_failing_frame_by_global_index():
+    # NaN keys in (b=0, h=3, t=4) make that frame's Gram NaN; with 5 heads in
+    # 3 groups the frame lies in the last group, whose inverse starts at frame
+    # 3 * 12, so the report must add that offset: 1 + (3 * 12 + 4)
+    w = custom("pipe_nan", index=53)
+    full = synth.generate_all(w)
+    full["K"][0, 3, 4, 7, 11] = np.nan
+    dev = device_inputs(w, full)
+    ref = run_forward(w, dev)
+    fw = _pipelined(w, dev, 3)
+    assert int(ref.info.item()) == 1 + 3 * 12 + 4
+    assert int(fw.info.item()) == int(ref.info.item())
+
+
+def test_pipelined_full_size_sampled_heads():
+    w = synth.WORKLOADS["h3"]
+    pairs = [(0, 0), (0, 9), (0, 23)]  # first, middle and last of three groups of eight
+    sampled = {(b, h): synth.generate_head(w, b, h) for b, h in pairs}
+    dev = device_fill(w, sampled, seed=w.seed)
+    fw = _pipelined(w, dev, 3)
+    assert int(fw.info.item()) == 0
+    for (b, h), inp in sampled.items():
+        r = oracle.vda_head(inp, w.chunk, w.anchors)
+        eo, ef, eg = rel(fw.O[b, h], r["O"]), rel(fw.F[b, h], r["F"]), rel(fw.G[b, h], r["G"])
+        print(f"h3 pipelined b{b} h{h}: O {eo:.2e} F {ef:.2e} G {eg:.2e}")
+        assert eo <= TOL["bf16"] and ef <= TOL["bf16"] and eg <= TOL["bf16"]
+    del dev, fw
+    torch.cuda.empty_cache()
