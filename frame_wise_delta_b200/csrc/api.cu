@@ -180,7 +180,7 @@ vdn_status run_text_state(const Geo &g, const void *Kx, const void *Vx, const fl
     // S_T is the injection of one "frame" made of the text tokens: invert,
     // then one J-chain step (B_x W_x) on the tensor cores.
     uint8_t *Wimg = (uint8_t *)(ws + L.wimg);
-    VDN_CUDA(launch_invert_simt(Ax, nullptr, Wimg, info, g.BH, g.D, st), "text invert");
+    VDN_CUDA(launch_invert_tc(Ax, nullptr, Wimg, info, g.BH, st), "text invert");
     VDN_CUDA(launch_compose_tc(Wimg, Bx, Ax, nullptr, S_T, nullptr, nullptr, nullptr, g.BH, 1, 1, 0,
                                /*ndirs=*/1, info, st),
              "text injection");
@@ -351,7 +351,10 @@ vdn_status vdn_frame_invert(const vdn_shape *s, const float *A, float *W, int32_
   VDN_TRY(need(info, "info", true));
   cudaStream_t st = (cudaStream_t)stream;
   VDN_CUDA(cudaMemsetAsync(info, 0, sizeof(int32_t), st), "memset info");
-  VDN_CUDA(launch_invert_simt(A, W, nullptr, info, g.BH * g.T, g.D, st), "invert");
+  if (tensor_path(g))
+    VDN_CUDA(launch_invert_tc(A, W, nullptr, info, g.BH * g.T, st), "invert");
+  else
+    VDN_CUDA(launch_invert_simt(A, W, nullptr, info, g.BH * g.T, g.D, st), "invert");
   return VDN_OK;
 }
 
@@ -449,7 +452,7 @@ vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K, const v
   VDN_TRY(mark(2));
   if (frames) {
     if (tc) {
-      VDN_CUDA(launch_invert_simt(A, nullptr, Wimg, info, g.BH * g.T, g.D, st), "invert");
+      VDN_CUDA(launch_invert_tc(A, nullptr, Wimg, info, g.BH * g.T, st), "invert");
     } else {
       // M and J overwrite A and Bm in place (each element is read and
       // written by the same thread).
@@ -549,8 +552,8 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
     VDN_CUDA(cudaStreamWaitEvent(ax, ev(base + 0), 0), "stream wait");
     VDN_CUDA(cudaEventRecord(ev(base + 1), ax), "event record");
     if (run)
-      VDN_CUDA(launch_invert_simt(A + b0 * T * DD, nullptr, Wimg + b0 * T * kImgBytes, info, nbh * T, g.D,
-                                  ax, b0 * T),
+      VDN_CUDA(launch_invert_tc(A + b0 * T * DD, nullptr, Wimg + b0 * T * kImgBytes, info, nbh * T, ax,
+                                b0 * T),
                "invert");
     VDN_CUDA(cudaEventRecord(ev(base + 2), ax), "event record");
   }

@@ -35,6 +35,10 @@ cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, voi
 // W = (I + A)^{-1} per frame (CUDA cores); W fp32 and/or Wimg (hi/lo MMA
 // images of kImgBytes per frame, d = 128 only), each optional.
 // frame_base: index of the first frame, for the failure index in *info.
+// (I + A)^{-1} of fp32 128 x 128 frames by the tensor-core block inverse, as
+// fp32 row-major W and/or hi/lo MMA images (either may be null)
+cudaError_t launch_invert_tc(const float *A, float *W, uint8_t *Wimg, int32_t *info, long long nframes,
+                             cudaStream_t st, long long frame_base = 0);
 cudaError_t launch_invert_simt(const float *A, float *W, uint8_t *Wimg, int32_t *info,
                                long long nframes, int D, cudaStream_t st, long long frame_base = 0);
 // Chunk maps from W images (tensor cores, d = 128): per (direction, b*h,

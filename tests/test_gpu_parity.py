@@ -125,9 +125,16 @@ def test_frame_invert(w):
     torch.cuda.synchronize()
     assert int(info.item()) == 0
     ref = np.linalg.inv(np.eye(w.d) + Ar)
-    assert rel(W, ref) <= 1e-5, rel(W, ref)
+    # the tensor-core block inverse (bf16 shapes, d = 128) multiplies hi/lo
+    # bf16 splits (each operand exact to ~2^-17): 1e-4, the fp32 bound; the
+    # fp32 sweep: 1e-5. Its off-diagonal blocks come from two separate
+    # products (-Y and -Y^T), so symmetry holds to rounding, not exactly.
+    tc = w.dtype == "bf16" and w.d == 128
+    e = rel(W, ref)
+    print(f"{w.name}: invert rel {e:.2e}")
+    assert e <= (1e-4 if tc else 1e-5), e
     Wc = W.double().cpu().numpy()
-    assert np.allclose(Wc, np.swapaxes(Wc, -1, -2), rtol=0, atol=1e-6)
+    assert np.allclose(Wc, np.swapaxes(Wc, -1, -2), rtol=0, atol=1e-5 if tc else 1e-6)
 
 
 def _maps_ref(w, full):
@@ -273,6 +280,30 @@ def test_nonpositive_pivot_is_reported_by_invert(d):
     vdn.vdn_frame_invert(s, to_dev(Ar), W, info)
     torch.cuda.synchronize()
     assert int(info.item()) == 1 + 13
+
+
+def test_nonpositive_pivot_is_reported_by_block_invert():
+    # bf16, d = 128: the tensor-core block inverse sweeps P (the leading 64 x 64
+    # block) and then the Schur complement S of the trailing block; a poisoned
+    # trailing diagonal makes S indefinite, a poisoned leading one P
+    w = custom("poison_tc", index=48, T=9, anchors=0)
+    full = _full(w)
+    Ar, _ = _stats_ref(w, full)
+    Ar[0, 1, 2, 100, 100] = -60.0   # (b=0, h=1, t=2): linear index 11, S fails
+    Ar[0, 1, 6, 3, 3] = -9.0        # (0, 1, 6): 15, P fails
+    s = vdn.shape_for(w)
+    W = torch.empty((w.B, w.H, w.T, w.d, w.d), device="cuda")
+    info = torch.zeros(1, dtype=torch.int32, device="cuda")
+    vdn.vdn_frame_invert(s, to_dev(Ar), W, info)
+    torch.cuda.synchronize()
+    assert int(info.item()) == 1 + 11
+    Ar[0, 1, 2, 100, 100] = 0.0
+    vdn.vdn_frame_invert(s, to_dev(Ar), W, info)
+    torch.cuda.synchronize()
+    assert int(info.item()) == 1 + 15
+    # the frames that were not poisoned are still exact
+    ref = np.linalg.inv(np.eye(w.d) + Ar[0, 0])
+    assert rel(W[0, 0], ref) <= 1e-4
 
 
 def test_nonpositive_pivot_is_reported():
