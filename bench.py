@@ -35,8 +35,8 @@ ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # sha256 prefix of the kernel source the counters were taken on; reported as
 # None as soon as that source changes.
 NCU_TRAFFIC = {
-    "frame_factor": {"bytes": 112.5e6 + 123.3e6, "source": "frame_wise_delta_b200/csrc/invert.cu",
-                     "sha256_16": "c731caa4fd644675", "workload": "h3"},
+    "frame_factor": {"bytes": 101.3e6 + 104.8e6, "source": "frame_wise_delta_b200/csrc/invert_tc.cu",
+                     "sha256_16": "71f8ec1c98c2a934", "workload": "h3"},
 }
 
 
@@ -415,8 +415,9 @@ def roofline(w, stage_ms, hbm_gbs, peak_src, bf16_tflops=1607.7):
     """Roofline of the dominant stage. Per-unit algorithmic figures:
     frame_grams: per frame reads K, V (2 U d bf16) and writes A, B (2 d^2 fp32);
     chunk_readout: per frame reads Q, writes O (2 U d bf16) plus two states per chunk;
-    frame_factor: d^3 flop per non-anchor frame on the tensor path (symmetric
-      sweep), 4 d^3 on the CUDA-core path (Gauss-Jordan on [I+A; B]);
+    frame_factor: on the tensor path the CUDA cores sweep two 64 x 64 blocks per
+      non-anchor frame (d^3 / 4 flop; the block products run on the tensor
+      cores), 4 d^3 on the CUDA-core path (Gauss-Jordan on [I+A; B]);
     chunk_compose: 4 d^3 flop per frame step (M and J chains), per direction;
     scan_bidir: 2 d^3 flop per chunk and direction."""
     B, H, T, U, d, C = w.B, w.H, w.T, w.U, w.d, w.C
@@ -432,7 +433,7 @@ def roofline(w, stage_ms, hbm_gbs, peak_src, bf16_tflops=1607.7):
     units = {
         "frame_grams": ("hbm", frames * (2 * U * d * e + 2 * d * d * 4)),
         "chunk_readout": ("hbm", frames * 2 * U * d * e + BH * C * 2 * d * d * 4),
-        "frame_factor": ("alu", live * (d ** 3 if tensor_path else 4 * d ** 3)),
+        "frame_factor": ("alu", live * (d ** 3 // 4 if tensor_path else 4 * d ** 3)),
         "chunk_compose": ("tensor" if tensor_path else "alu", BH * 2 * steps * 4 * d ** 3),
         "scan_bidir": ("tensor" if tensor_path else "alu", BH * 2 * C * 2 * d ** 3),
     }

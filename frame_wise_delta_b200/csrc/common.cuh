@@ -133,6 +133,15 @@ __device__ __forceinline__ void split_bf16(float v, __nv_bfloat16 &h, __nv_bfloa
   l = __float2bfloat16_rn(v - __bfloat162float(h));
 }
 
+// Two values at once: hi = bf16 pair (a, b) (a in the low half), lo = the pair
+// of residuals, each rounded to nearest like split_bf16.
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t &hi, uint32_t &lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(a - __low2float(h), b - __high2float(h));
+  hi = *reinterpret_cast<const uint32_t *>(&h);
+  lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
 __device__ __forceinline__ uint32_t pack2(__nv_bfloat16 a, __nv_bfloat16 b) {
   return (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
 }

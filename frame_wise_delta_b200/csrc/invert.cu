@@ -22,7 +22,7 @@ __global__ void __launch_bounds__(kSweepThreads) invert_sweep_kernel(const float
                                                                      long long frame_base) {
   using S = Sweep<D>;
   constexpr int R = S::R;
-  __shared__ __align__(16) float cbuf[2][D];
+  __shared__ __align__(16) float cbuf[2][2][D];
   const long long f = blockIdx.x;
   const int rg = threadIdx.x / kSweepGrid, cg = threadIdx.x % kSweepGrid;
   const float *Af = A + f * (long long)D * D;
@@ -35,7 +35,7 @@ __global__ void __launch_bounds__(kSweepThreads) invert_sweep_kernel(const float
       const int i = rg + kSweepGrid * a, j = cg + kSweepGrid * b;
       X.at(a, b) = Af[i * D + j] + (i == j ? 1.f : 0.f);
     }
-  const bool ok = X.run(cbuf, rg, cg, [] { __syncthreads(); });
+  const bool ok = X.run2(cbuf, rg, cg, [] { __syncthreads(); });
   if (!ok && threadIdx.x == 0) report_frame_failure(info, frame_base + f);
 
   // W = -X; write both triangles

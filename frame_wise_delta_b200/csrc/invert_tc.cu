@@ -16,9 +16,10 @@
 // TMEM. A pivot of P or S that is not positive (G not positive definite) is
 // reported in *info like the sweep does.
 //
-// One CTA of 128 threads per frame at a time (persistent over frames), four
-// CTAs per SM: warps 0-1 run the sweeps, warps 2-3 own TMEM lanes 64-127 and
-// do the loads, the epilogues and the output; thread 64 issues the MMAs.
+// One CTA of 128 threads works through frames (persistent), four CTAs per SM:
+// warps 0-1 run the sweeps, warps 2-3 own TMEM lanes 64-127 and do the loads,
+// the epilogues and the output; thread 64 issues the MMAs. The two pairs are
+// one frame apart where they can be (named-barrier hand-offs).
 // Every product keeps its 64 useful rows in lanes 64-127: the A operand's
 // descriptor starts 64 rows (8 KB) before the useful rows, so lanes 0-63
 // compute throw-away rows from whatever shared memory lies there.
@@ -30,6 +31,7 @@ namespace vdn {
 namespace {
 
 constexpr int kThreads = 128;
+constexpr int kCtasPerSm = 4;          // x 128 TMEM columns <= 512
 constexpr int kHalf = 64 * 128;         // one 64 x 64 bf16 tile, 128-byte rows: 8 KB
 constexpr int kTile = 2 * kHalf;        // hi + lo: 16 KB
 // shared memory slots (offsets from the 1024-aligned base)
@@ -49,28 +51,23 @@ __device__ __forceinline__ uint32_t tile_off(int row, int k) { return kmajor_sw1
 // physical 16-byte chunk of logical chunk c in row r (both tile and image layouts)
 __device__ __forceinline__ uint32_t chunk_pos(int r, int c) { return (uint32_t)((c ^ (r & 7)) << 4); }
 
-__device__ __forceinline__ uint4 pack8(const float *v, bool lo) {
-  uint32_t w[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    __nv_bfloat16 h0, l0, h1, l1;
-    split_bf16(v[2 * q], h0, l0);
-    split_bf16(v[2 * q + 1], h1, l1);
-    w[q] = lo ? pack2(l0, l1) : pack2(h0, h1);
-  }
-  return make_uint4(w[0], w[1], w[2], w[3]);
+// hi and lo 16-byte chunks of 8 values (times sign)
+__device__ __forceinline__ void pack8(const float *v, float sign, uint4 &h, uint4 &l) {
+  split_bf16x2(sign * v[0], sign * v[1], h.x, l.x);
+  split_bf16x2(sign * v[2], sign * v[3], h.y, l.y);
+  split_bf16x2(sign * v[4], sign * v[5], h.z, l.z);
+  split_bf16x2(sign * v[6], sign * v[7], h.w, l.w);
 }
 
 // Row r of a hi/lo tile (64 values) written from one thread.
 __device__ __forceinline__ void tile_row_store(uint8_t *tile, int r, const float *v, float sign) {
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
-    float s[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) s[e] = sign * v[8 * c + e];
+    uint4 h, l;
+    pack8(v + 8 * c, sign, h, l);
     const uint32_t o = (uint32_t)r * 128u + chunk_pos(r, c);
-    *reinterpret_cast<uint4 *>(tile + o) = pack8(s, false);
-    *reinterpret_cast<uint4 *>(tile + kHalf + o) = pack8(s, true);
+    *reinterpret_cast<uint4 *>(tile + o) = h;
+    *reinterpret_cast<uint4 *>(tile + kHalf + o) = l;
   }
 }
 
@@ -79,12 +76,11 @@ __device__ __forceinline__ void img_row_store(uint8_t *img, int region, int r, c
   uint8_t *base = img + region * kImgRegion + r * 128;
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
-    float s[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) s[e] = sign * v[8 * c + e];
+    uint4 h, l;
+    pack8(v + 8 * c, sign, h, l);
     const uint32_t o = chunk_pos(r, c);
-    *reinterpret_cast<uint4 *>(base + o) = pack8(s, false);
-    *reinterpret_cast<uint4 *>(base + kImgHalf + o) = pack8(s, true);
+    *reinterpret_cast<uint4 *>(base + o) = h;
+    *reinterpret_cast<uint4 *>(base + kImgHalf + o) = l;
   }
 }
 
@@ -109,6 +105,17 @@ __device__ __forceinline__ void mma_hilo(uint32_t d, uint32_t a_hi, uint32_t a_l
 __device__ __forceinline__ void bar_named(int id) {
   asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
 }
+// hand-offs between the sweep warps and the epilogue warps (128 threads:
+// the producers arrive, the consumers wait)
+__device__ __forceinline__ void handoff_arrive(int id) {
+  __threadfence_block();
+  asm volatile("bar.arrive %0, 128;" ::"r"(id) : "memory");
+}
+__device__ __forceinline__ void handoff_wait(int id) {
+  asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
+}
+constexpr int kBarSweep = 1, kBarEpi = 2;           // within each warp pair
+constexpr int kBarPiReady = 3, kBarTReady = 4, kBarSiReady = 5, kBarPiFree = 6;
 
 // v (+)= row r of a hi/lo tile, decoded to fp32
 __device__ __forceinline__ void tile_row_add(const uint8_t *tile, int r, float (&v)[64], bool add) {
@@ -166,7 +173,7 @@ __device__ __forceinline__ void store_swept(Sweep<64> &X, uint8_t *tile, int rg,
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 4)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     invert_tc_kernel(const float *__restrict__ A, float *__restrict__ W, uint8_t *__restrict__ Wimg,
                      int32_t *__restrict__ info, long long nframes, long long frame_base) {
   extern __shared__ uint8_t smem_raw[];
@@ -188,72 +195,96 @@ __global__ void __launch_bounds__(kThreads, 4)
   __syncthreads();
   tc_fence_after();
   const uint32_t acc0 = *tmem_slot, acc1 = acc0 + 64;
-  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-  const uint32_t a_pi = smem_u32(pi_t), a_s0 = smem_u32(s0), a_xt = smem_u32(xt);
-  const int rg = (tid & 63) / kSweepGrid, cg = tid % kSweepGrid;  // sweep grid (warps 0-1)
-  const int i = tid - 64;                                         // epilogue row (warps 2-3)
-  float *stage = reinterpret_cast<float *>(s0);                   // fp32 Q^T X, swizzled rows
-  uint32_t nwait = 0;
-  auto wait_mma = [&]() {
-    if (!mbar_wait(mbar, nwait & 1, abort)) fail(abort, info);
-    ++nwait;
-    tc_fence_after();
-  };
-  auto issue = [&](auto body) {  // thread 64, after the operands are visible to the tensor cores
-    if (tid == 64 && !*abort) {
-      tc_fence_after();
-      body();
-      tc_commit(mbar);
-    }
-  };
+  float *stage = reinterpret_cast<float *>(s0);  // fp32 Q^T X, rows with swizzled 16-byte chunks
 
-  for (long long f = blockIdx.x; f < nframes; f += gridDim.x) {
-    const float *Af = A + f * 128LL * 128;
-    uint8_t *img = Wimg ? Wimg + f * (long long)kImgBytes : nullptr;
-    float *Wf = W ? W + f * 128LL * 128 : nullptr;
-    bool ok = true;
-    if (tid < 64) {
-      // P^{-1} by the sweep
+  // The two warp pairs run their own loops over the same frames and meet at
+  // the hand-off barriers, so that the sweep of frame f + 1's P overlaps the
+  // last products and the output of frame f:
+  //   sweep warps:    P sweep -> [P^{-1} free] -> P^{-1} tile -> (PiReady)
+  //                   [TReady] -> S sweep -> S^{-1} tile -> (SiReady)
+  //   epilogue warps: Q^T tile -> [PiReady] -> X^T -> Q^T X staged -> (TReady)
+  //                   [SiReady] -> Y, Y^T -> Y X^T -> (P^{-1} free) -> output
+  if (tid < 64) {
+    const int rg = tid / kSweepGrid, cg = tid % kSweepGrid;
+    bool first = true;
+    for (long long f = blockIdx.x; f < nframes; f += gridDim.x) {
+      const float *Af = A + f * 128LL * 128;
       Sweep<64> X;
 #pragma unroll
       for (int a = 0; a < Sweep<64>::R; ++a)
 #pragma unroll
         for (int b = 0; b <= a; ++b) {
           const int r = rg + kSweepGrid * a, c = cg + kSweepGrid * b;
-          X.at(a, b) = Af[r * 128 + c] + (r == c ? 1.f : 0.f);
+          X.at(a, b) = __ldg(Af + r * 128 + c) + (r == c ? 1.f : 0.f);
         }
-      ok = X.run(cbuf, rg, cg, [] { bar_named(1); });
+      bool ok = X.run(cbuf, rg, cg, [] { bar_named(kBarSweep); });
+      if (!first) handoff_wait(kBarPiFree);  // the previous frame's last product has read P^{-1}
+      first = false;
       store_swept(X, pi_t, rg, cg);
-    } else {
+      fence_proxy_async_smem();
+      handoff_arrive(kBarPiReady);
+      handoff_wait(kBarTReady);
+      // S = R - Q^T X and S^{-1} by the sweep; S^{-1} replaces the staging
+      // (every thread has read its part before the sweep's first barrier)
+#pragma unroll
+      for (int a = 0; a < Sweep<64>::R; ++a)
+#pragma unroll
+        for (int b = 0; b <= a; ++b) {
+          const int r = rg + kSweepGrid * a, c = cg + kSweepGrid * b;
+          X.at(a, b) = __ldg(Af + (64 + r) * 128 + 64 + c) + (r == c ? 1.f : 0.f) -
+                       stage[r * 64 + (((c >> 2) ^ (r & 15)) << 2) + (c & 3)];
+        }
+      ok = X.run(cbuf, rg, cg, [] { bar_named(kBarSweep); }) && ok;
+      store_swept(X, s0, rg, cg);
+      fence_proxy_async_smem();
+      handoff_arrive(kBarSiReady);
+      if (!ok && tid == 0) report_frame_failure(info, frame_base + f);
+    }
+  } else {
+    const int i = tid - 64;  // TMEM lane 64 + i, row i of every product
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t a_pi = smem_u32(pi_t), a_s0 = smem_u32(s0), a_xt = smem_u32(xt);
+    uint32_t nwait = 0;
+    auto wait_mma = [&]() {
+      if (!mbar_wait(mbar, nwait & 1, abort)) fail(abort, info);
+      ++nwait;
+      tc_fence_after();
+    };
+    auto issue = [&](auto body) {  // thread 64, once the operands are visible to the tensor cores
+      if (tid == 64 && !*abort) {
+        tc_fence_after();
+        body();
+        tc_commit(mbar);
+      }
+    };
+    for (long long f = blockIdx.x; f < nframes; f += gridDim.x) {
+      const float *Af = A + f * 128LL * 128;
+      uint8_t *img = Wimg ? Wimg + f * (long long)kImgBytes : nullptr;
+      float *Wf = W ? W + f * 128LL * 128 : nullptr;
       // Q^T = G[64 + r][0 .. 63] as a hi/lo tile, read row-contiguously
-      const int e = i;
 #pragma unroll 4
       for (int it = 0; it < 16; ++it) {
-        const int r = it * 4 + (e >> 4), c4 = e & 15;
+        const int r = it * 4 + (i >> 4), c4 = i & 15;
         const float4 x = __ldg(reinterpret_cast<const float4 *>(Af + (64 + r) * 128 + 4 * c4));
-        __nv_bfloat16 h[4], l[4];
-        split_bf16(x.x, h[0], l[0]);
-        split_bf16(x.y, h[1], l[1]);
-        split_bf16(x.z, h[2], l[2]);
-        split_bf16(x.w, h[3], l[3]);
+        uint2 h, l;
+        split_bf16x2(x.x, x.y, h.x, l.x);
+        split_bf16x2(x.z, x.w, h.y, l.y);
         const uint32_t o = tile_off(r, 4 * c4);
-        *reinterpret_cast<uint2 *>(s0 + o) = make_uint2(pack2(h[0], h[1]), pack2(h[2], h[3]));
-        *reinterpret_cast<uint2 *>(s0 + kHalf + o) = make_uint2(pack2(l[0], l[1]), pack2(l[2], l[3]));
+        *reinterpret_cast<uint2 *>(s0 + o) = h;
+        *reinterpret_cast<uint2 *>(s0 + kHalf + o) = l;
       }
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    // X^T = Q^T P^{-1}
-    issue([&] { mma_hilo(acc0, a_s0 - kHalf, a_s0, a_pi, a_pi + kHalf, false, false, 16, kIdesc); });
-    if (tid >= 64) {
+      fence_proxy_async_smem();
+      handoff_wait(kBarPiReady);
+      // X^T = Q^T P^{-1}
+      issue([&] { mma_hilo(acc0, a_s0 - kHalf, a_s0, a_pi, a_pi + kHalf, false, false, 16, kIdesc); });
       float v[64];
       wait_mma();
       tmem_row64(acc0 + lane_off, v);
       tile_row_store(xt, i, v, 1.f);
       fence_proxy_async_smem();
       tc_fence_before();
-      bar_named(2);
-      // Q^T X (B = Q read from the Q^T tile K-major)
+      bar_named(kBarEpi);
+      // Q^T X (B = Q read from the Q^T tile K-major), staged in fp32 for the S sweep
       issue([&] { mma_hilo(acc0, a_xt - kHalf, a_xt, a_s0, a_s0 + kHalf, false, false, 16, kIdesc); });
       wait_mma();
       tmem_row64(acc0 + lane_off, v);
@@ -262,35 +293,15 @@ __global__ void __launch_bounds__(kThreads, 4)
         *reinterpret_cast<float4 *>(stage + i * 64 + ((c ^ (i & 15)) << 2)) =
             make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
       tc_fence_before();
-    }
-    __syncthreads();
-    if (tid < 64) {
-      // S = R - Q^T X and S^{-1} by the sweep; S^{-1} replaces the staging
-      // (every thread has read its part before the sweep's first barrier)
-      Sweep<64> X;
-#pragma unroll
-      for (int a = 0; a < Sweep<64>::R; ++a)
-#pragma unroll
-        for (int b = 0; b <= a; ++b) {
-          const int r = rg + kSweepGrid * a, c = cg + kSweepGrid * b;
-          X.at(a, b) = Af[(64 + r) * 128 + 64 + c] + (r == c ? 1.f : 0.f) -
-                       stage[r * 64 + (((c >> 2) ^ (r & 15)) << 2) + (c & 3)];
-        }
-      ok = X.run(cbuf, rg, cg, [] { bar_named(1); }) && ok;
-      store_swept(X, s0, rg, cg);
-      fence_proxy_async_smem();
-      if (!ok && tid == 0) report_frame_failure(info, frame_base + f);
-    }
-    __syncthreads();
-    issue([&] {
-      // Y = X S^{-1}: A = X, the X^T tile read MN-major as the second 64-row
-      // block (lanes 64-127) of a descriptor that starts one tile earlier
-      mma_hilo(acc0, a_xt - kTile, a_xt + kHalf - kTile, a_s0, a_s0 + kHalf, true, false, kTile, kIdescAmn);
-      // Y^T = S^{-1} X^T: B = X^T read MN-major
-      mma_hilo(acc1, a_s0 - kHalf, a_s0, a_xt, a_xt + kHalf, false, true, 16, kIdescBmn);
-    });
-    if (tid >= 64) {
-      float v[64];
+      handoff_arrive(kBarTReady);
+      handoff_wait(kBarSiReady);
+      issue([&] {
+        // Y = X S^{-1}: A = X, the X^T tile read MN-major as the second 64-row
+        // block (lanes 64-127) of a descriptor that starts one tile earlier
+        mma_hilo(acc0, a_xt - kTile, a_xt + kHalf - kTile, a_s0, a_s0 + kHalf, true, false, kTile, kIdescAmn);
+        // Y^T = S^{-1} X^T: B = X^T read MN-major
+        mma_hilo(acc1, a_s0 - kHalf, a_s0, a_xt, a_xt + kHalf, false, true, 16, kIdescBmn);
+      });
       wait_mma();
       tmem_row64(acc0 + lane_off, v);  // row i of Y
       // top-right block: -Y
@@ -319,21 +330,20 @@ __global__ void __launch_bounds__(kThreads, 4)
       if (Wf) w_row_store(Wf, 0, 64 + i, v, -1.f);
       fence_proxy_async_smem();
       tc_fence_before();
-      bar_named(2);
+      bar_named(kBarEpi);
       // Y X^T
       issue([&] { mma_hilo(acc0, a_s0 - kHalf, a_s0, a_xt, a_xt + kHalf, false, true, 16, kIdescBmn); });
       wait_mma();
       tmem_row64(acc0 + lane_off, v);
-      // top-left block: P^{-1} + Y X^T, P^{-1} from its hi/lo tile
+      // top-left block: P^{-1} + Y X^T; once every row of P^{-1} is read the
+      // sweep warps may overwrite it with the next frame's
       tile_row_add(pi_t, i, v, true);
+      if (f + gridDim.x < nframes) handoff_arrive(kBarPiFree);
       if (img) img_row_store(img, 0, i, v, 1.f);
       if (Wf) w_row_store(Wf, 0, i, v, 1.f);
       tc_fence_before();
     }
-    __syncthreads();
-    if (*abort) break;
   }
-  tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
@@ -349,8 +359,7 @@ cudaError_t launch_invert_tc(const float *A, float *W, uint8_t *Wimg, int32_t *i
   cudaError_t e = cudaFuncSetAttribute(invert_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  // four CTAs per SM: 4 x 128 TMEM columns fill the SM's 512
-  const long long cap = 4LL * device_sm_count();
+  const long long cap = (long long)kCtasPerSm * device_sm_count();
   const long long grid = nframes < cap ? nframes : cap;
   invert_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(A, W, Wimg, info, nframes, frame_base);
   return cudaGetLastError();

@@ -63,7 +63,7 @@ struct Sweep {
         sync();
         const float piv = c[kr * R + kb];
         bad |= !(piv > 0.f) || !isfinite(piv);
-        const float rp = 1.0f / piv;
+        const float rp = __frcp_rn(piv);
         // c_i for this thread's rows is read from shared memory where it is used
         const float *ci = &c[rg * R];
         float2 cj2[P];  // c_j / piv for this thread's columns, as pairs
@@ -100,6 +100,90 @@ struct Sweep {
           at(kb, kb) = (cg == kr) ? -rp : VDN_CJ(kb);
         }
 #undef VDN_CJ
+      }
+    }
+    return !bad;
+  }
+
+  // The same result two pivots at a time: sweeping the pair K = {k, k + 1}
+  // at once maps G_KK -> -G_KK^{-1}, G_iK -> G_iK G_KK^{-1} and
+  // G_ij -> G_ij - G_iK G_KK^{-1} G_Kj (sweeps compose, so this equals
+  // sweeping k and then k + 1). One barrier and one reciprocal (of the 2 x 2
+  // block's determinant) per pair. `cbuf` is 2 x 2 x D floats here.
+  template <class Sync>
+  __device__ __forceinline__ bool run2(float (*cbuf)[2][D], int rg, int cg, Sync sync) {
+    static_assert(kSweepGrid % 2 == 0, "pivot pairs stay inside a block of 8");
+    bool bad = false;
+#pragma unroll
+    for (int kb = 0; kb < R; ++kb) {
+#pragma unroll 1
+      for (int kr = 0; kr < kSweepGrid; kr += 2) {
+        float *c0 = cbuf[(kr >> 1) & 1][0], *c1 = cbuf[(kr >> 1) & 1][1];
+        // publish columns k and k + 1 (slot (x % 8) * R + x / 8 as in run)
+        if (cg == kr || cg == kr + 1) {
+          float *c = cg == kr ? c0 : c1;
+#pragma unroll
+          for (int a = kb; a < R; ++a) c[rg * R + a] = at(a, kb);
+        }
+        if (rg == kr || rg == kr + 1) {
+          float *c = rg == kr ? c0 : c1;
+#pragma unroll
+          for (int b = 0; b < kb; ++b) c[cg * R + b] = at(kb, b);
+        }
+        sync();
+        const float p00 = c0[kr * R + kb], p01 = c0[(kr + 1) * R + kb], p11 = c1[(kr + 1) * R + kb];
+        const float det = fmaf(p00, p11, -p01 * p01);
+        bad |= !(p00 > 0.f) || !(det > 0.f) || !isfinite(p00) || !isfinite(det);
+        const float rd = __frcp_rn(det);
+        const float q00 = p11 * rd, q01 = -p01 * rd, q11 = p00 * rd;  // G_KK^{-1}
+        const float *ci0 = &c0[rg * R], *ci1 = &c1[rg * R];
+        // e_j = G_KK^{-1} (c0_j, c1_j) for this thread's columns, as pairs
+        float2 e0[P], e1[P];
+        {
+          const float2 Q00 = make_float2(q00, q00), Q01 = make_float2(q01, q01), Q11 = make_float2(q11, q11);
+#pragma unroll
+          for (int q = 0; q < P; ++q) {
+            float2 x0, x1;
+            if constexpr (R % 2 == 0) {
+              x0 = *reinterpret_cast<const float2 *>(&c0[cg * R + 2 * q]);
+              x1 = *reinterpret_cast<const float2 *>(&c1[cg * R + 2 * q]);
+            } else {
+              x0 = make_float2(c0[cg * R + 2 * q], (2 * q + 1 < R) ? c0[cg * R + 2 * q + 1] : 0.f);
+              x1 = make_float2(c1[cg * R + 2 * q], (2 * q + 1 < R) ? c1[cg * R + 2 * q + 1] : 0.f);
+            }
+            e0[q] = __ffma2_rn(Q01, x1, __fmul2_rn(Q00, x0));
+            e1[q] = __ffma2_rn(Q11, x1, __fmul2_rn(Q01, x0));
+          }
+        }
+#define VDN_E(e, b) (((b) & 1) ? e[(b) >> 1].y : e[(b) >> 1].x)
+#pragma unroll
+        for (int a = 0; a < R; ++a) {
+          const float n0 = -ci0[a], n1 = -ci1[a];
+          const float2 m0 = make_float2(n0, n0), m1 = make_float2(n1, n1);
+#pragma unroll
+          for (int q = 0; q < (a + 1) / 2; ++q) XP[a][q] = __ffma2_rn(m1, e1[q], __ffma2_rn(m0, e0[q], XP[a][q]));
+          if ((a & 1) == 0) XS[a >> 1] = fmaf(n1, VDN_E(e1, a), fmaf(n0, VDN_E(e0, a), XS[a >> 1]));
+        }
+        // columns k, k + 1 (rows at and below the diagonal block): c_i^T G_KK^{-1}
+        if (cg == kr || cg == kr + 1) {
+          const float u0 = cg == kr ? q00 : q01, u1 = cg == kr ? q01 : q11;
+#pragma unroll
+          for (int a = kb; a < R; ++a) at(a, kb) = fmaf(ci1[a], u1, ci0[a] * u0);
+        }
+        // rows k, k + 1 (left of and in the diagonal block): G_KK^{-1} c_j, and
+        // -G_KK^{-1} on the pair itself
+        if (rg == kr || rg == kr + 1) {
+          const bool r0 = rg == kr;
+#pragma unroll
+          for (int b = 0; b < kb; ++b) at(kb, b) = r0 ? VDN_E(e0, b) : VDN_E(e1, b);
+          if (cg == kr || cg == kr + 1) {
+            const bool c0k = cg == kr;
+            at(kb, kb) = r0 ? (c0k ? -q00 : -q01) : (c0k ? -q01 : -q11);
+          } else {
+            at(kb, kb) = r0 ? VDN_E(e0, kb) : VDN_E(e1, kb);
+          }
+        }
+#undef VDN_E
       }
     }
     return !bad;
