@@ -5,7 +5,7 @@
 // and "Method steps" step (5):
 //   R_c = F[max(c-1,0)] + G[min(c+2,C)],   o_{t,u} = R_c q_{t,u}.
 //
-// D = R Q_tile^T with M = 128 (value channel i), N = 128 tokens, K = 128 key
+// D = Q_tile R^T with M = 128 tokens, N = 128 (value channel i), K = 128 key
 // channels. The fp32 state R is split into bf16 hi + lo parts (R = hi + lo to
 // ~2^-17 relative) and both products accumulate into one fp32 TMEM tile, so
 // the readout keeps fp32-state accuracy while Q is read once, as bf16.
@@ -17,7 +17,8 @@
 // rebuilt only when the chunk changes.
 //   warp 0     : TMA producer (two 16 KB loads per 128-token stage)
 //   warp 1     : TMEM allocator and single-thread MMA issuer
-//   warps 2..5 : R builder and epilogue (TMEM -> bf16 stores; anchor frames
+//   warps 2..5 : R builder and epilogue (TMEM -> bf16 tile in shared memory ->
+//                TMA store, double-buffered; anchor frames
 //                are written as zeros without touching the tensor cores)
 #include <cudaTypedefs.h>
 
@@ -29,16 +30,18 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kNT = 128;                      // tokens per tile (MMA N)
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kStageBytes = kNT * 128 * 2;    // two 64-channel regions
 constexpr int kRegionQ = kNT * 128;           // 16 KB
 constexpr int kRBytes = kD * 128 * 2;         // one bf16 R operand, 2 regions
 constexpr int kRegionR = kD * 128;
+constexpr int kOBytes = kNT * 128 * 2;        // one bf16 O tile, two 64-channel regions
+constexpr int kRegionO = kNT * 128;
 constexpr int kAcc = 4;                       // TMEM accumulators (128 columns each)
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBarBytes = 8 * (2 * kStages + 2 * kAcc + 2);
-constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 2 * kRBytes + kBarBytes + 16;
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 2 * kRBytes + 2 * kOBytes + kBarBytes + 16;
 
 struct ReadoutArgs {
   const float *F;
@@ -64,20 +67,21 @@ __device__ __forceinline__ long long chunk_key(const ReadoutArgs &p, long long f
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(a));
-  const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(b));
-  return lo | (hi << 16);
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);  // a in the low half
+  return *reinterpret_cast<const uint32_t *>(&h);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    readout_tc_kernel(const __grid_constant__ CUtensorMap tmQ, ReadoutArgs p) {
+    readout_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+                      ReadoutArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
   uint8_t *stages = smem;
   uint8_t *Rhi = smem + kStages * kStageBytes;
   uint8_t *Rlo = Rhi + kRBytes;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(Rlo + kRBytes);
+  uint8_t *Obuf = Rlo + kRBytes;  // two O staging tiles
+  uint64_t *bars = reinterpret_cast<uint64_t *>(Obuf + 2 * kOBytes);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(bars) + kBarBytes);
   volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -185,8 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int ks = 0; ks < kD / 16; ++ks) {
               const uint32_t koff = (uint32_t)(ks & 3) * 32;  // 16 bf16 = 32 B inside the swizzle atom
-              const uint64_t adesc = smem_desc_sw128(r + (ks >> 2) * kRegionR + koff, 16, 1024);
-              const uint64_t bdesc = smem_desc_sw128(q + (ks >> 2) * kRegionQ + koff, 16, 1024);
+              const uint64_t adesc = smem_desc_sw128(q + (ks >> 2) * kRegionQ + koff, 16, 1024);
+              const uint64_t bdesc = smem_desc_sw128(r + (ks >> 2) * kRegionR + koff, 16, 1024);
               tc_mma_bf16(dcol, adesc, bdesc, idesc, (part > 0 || ks > 0) ? 1u : 0u);
             }
           }
@@ -205,9 +209,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     const int et = threadIdx.x - 64;  // 0..127
     const int sub = warp & 3;
-    const int row = sub * 32 + lane;  // value channel i held by this thread
+    const int row = sub * 32 + lane;  // token of the tile held by this thread (TMEM lane)
     uint32_t tile = 0;
     long long cur = -1;
+    bool ok = true;  // after a failed wait: keep every barrier, skip the work
     for (long long f = f_begin; f < f_end; ++f) {
       __nv_bfloat16 *Of = p.O + f * (long long)p.U * kD;
       if (is_anchor(p, f)) {
@@ -233,54 +238,61 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float4 a0 = f4[0], a1 = f4[1], b0 = g4[0], b1 = g4[1];
           const float r[8] = {a0.x + b0.x, a0.y + b0.y, a0.z + b0.z, a0.w + b0.w,
                               a1.x + b1.x, a1.y + b1.y, a1.z + b1.z, a1.w + b1.w};
-          float h[8], l[8];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            h[q] = __bfloat162float(__float2bfloat16_rn(r[q]));
-            l[q] = r[q] - h[q];
-          }
+          uint4 h, l;
+          split_bf16x2(r[0], r[1], h.x, l.x);
+          split_bf16x2(r[2], r[3], h.y, l.y);
+          split_bf16x2(r[4], r[5], h.z, l.z);
+          split_bf16x2(r[6], r[7], h.w, l.w);
           const uint32_t off = kmajor_sw128_offset(i, k0, kD);
-          *reinterpret_cast<uint4 *>(Rhi + off) =
-              make_uint4(pack_bf16(h[0], h[1]), pack_bf16(h[2], h[3]), pack_bf16(h[4], h[5]),
-                         pack_bf16(h[6], h[7]));
-          *reinterpret_cast<uint4 *>(Rlo + off) =
-              make_uint4(pack_bf16(l[0], l[1]), pack_bf16(l[2], l[3]), pack_bf16(l[4], l[5]),
-                         pack_bf16(l[6], l[7]));
+          *reinterpret_cast<uint4 *>(Rhi + off) = h;
+          *reinterpret_cast<uint4 *>(Rlo + off) = l;
         }
         fence_proxy_async_smem();
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (et == 0) mbar_arrive(rfull);
       }
-      bool ok = true;
       for (int j = 0; j < p.ntiles; ++j, ++tile) {
         const int buf = (int)(tile % kAcc);
         const uint32_t use = tile / kAcc;
-        if (!__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * buf, use & 1, abort))) {
+        uint8_t *ob = Obuf + (tile & 1) * kOBytes;
+        // the TMA store that last read this staging tile (two tiles ago) is done
+        if (et == 0) bulk_wait_read<1>();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (ok && !__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * buf, use & 1, abort))) {
           fail(abort, p.info);
           ok = false;
-          break;
         }
-        tc_fence_after();
-#pragma unroll 1
-        for (int cc = 0; cc < kNT / 32; ++cc) {
-          float v[32];
-          tmem_ld32(tmem_base + (uint32_t)(buf * kNT + cc * 32) + ((uint32_t)(sub * 32) << 16), v);
-          const int u0 = j * kNT + cc * 32;
-          __nv_bfloat16 *dst = Of + (long long)u0 * kD + row;
-          if (u0 + 32 <= p.U) {
+        if (ok) {
+          tc_fence_after();
+          // row `row` of the tile: 128 channels -> bf16, 16-byte chunks swizzled
+          // as the tensor map's 128-byte swizzle expects
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj) dst[jj * kD] = __float2bfloat16_rn(v[jj]);
-          } else {
+          for (int cc = 0; cc < kD / 32; ++cc) {
+            float v[32];
+            tmem_ld32(tmem_base + (uint32_t)(buf * kNT + cc * 32) + ((uint32_t)(sub * 32) << 16), v);
+            uint8_t *rb = ob + (cc >> 1) * kRegionO + row * 128;
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj)
-              if (u0 + jj < p.U) dst[jj * kD] = __float2bfloat16_rn(v[jj]);
+            for (int q = 0; q < 4; ++q) {
+              const int ch = (cc & 1) * 4 + q;
+              *reinterpret_cast<uint4 *>(rb + ((ch ^ (row & 7)) << 4)) =
+                  make_uint4(pack_bf16(v[8 * q], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                             pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+            }
           }
+          tc_fence_before();
+          mbar_arrive(tempty0 + 8 * buf);
         }
-        tc_fence_before();
-        mbar_arrive(tempty0 + 8 * buf);
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (ok && et == 0) {
+          // rows past U fall outside the tensor and are not written
+          tma_store_3d(&tmO, smem_u32(ob), 0, j * kNT, (int)f);
+          tma_store_3d(&tmO, smem_u32(ob + kRegionO), 64, j * kNT, (int)f);
+          bulk_commit();
+        }
       }
-      if (!ok) break;
     }
+    if (et == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -304,8 +316,9 @@ cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, voi
                               int T, int U, int chunk, int anchors, int32_t *info, cudaStream_t st) {
   const long long nframes = BH * T;
   if (nframes <= 0) return cudaSuccess;
-  CUtensorMap tmQ;
-  if (!make_rows_map(&tmQ, Q, nframes, U, kNT)) return cudaErrorInvalidValue;
+  CUtensorMap tmQ, tmO;
+  if (!make_rows_map(&tmQ, Q, nframes, U, kNT) || !make_rows_map(&tmO, O, nframes, U, kNT))
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(readout_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
@@ -313,7 +326,7 @@ cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, voi
   const long long grid = nframes < sms ? nframes : sms;
   ReadoutArgs a{F, G, (__nv_bfloat16 *)O, info, nframes, T, U, chunk, anchors,
                 (T + chunk - 1) / chunk, (U + kNT - 1) / kNT};
-  readout_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(tmQ, a);
+  readout_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(tmQ, tmO, a);
   return cudaGetLastError();
 }
 
