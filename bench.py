@@ -206,8 +206,9 @@ def run_reference(args, w):
 
 
 def workload_config(w):
+    gates = "per-token write gates" if w.beta_per_token else "per-frame write gates"
     return {"workload": f"{w.name}: B={w.B} H={w.H} T={w.T} U={w.U} d_k=d_v={w.d} n_text={w.n_text} "
-                        f"chunk={w.chunk} anchors={w.anchors} {w.dtype} inputs, fp32 state",
+                        f"chunk={w.chunk} anchors={w.anchors} {w.dtype} inputs, fp32 state, {gates}",
             "global_batch": w.B, "frames": w.B * w.T, "tokens": w.B * w.T * w.U,
             "l2": "inputs larger than L2 (Q+K+V bf16 = %.2f GB > 126 MB)" % (3 * w.B * w.H * w.T * w.U * w.d * 2 / 1e9),
             "parallelism": "heads independent; one full problem per rank"}
@@ -403,11 +404,12 @@ def e2e_measure(args, host, d, make_forward, stream, barrier, world, frames_all,
 
 def alg_bytes(w):
     """Algorithmic HBM bytes of the whole pass: Q, K, V read, O written (bf16),
-    text keys/values read, gates read."""
+    text keys/values read, gates read (write gates per frame or per token)."""
     e = 2 if w.dtype == "bf16" else 4
     qkvo = 4 * w.B * w.H * w.T * w.U * w.d * e
     text = 2 * w.B * w.H * w.n_text * w.d * e
-    gates = w.B * w.H * w.T * (w.d + 1) * 4
+    tb = getattr(w, "beta_per_token", False)
+    gates = w.B * w.H * (w.T * (w.d + (w.U if tb else 1)) + (w.n_text if tb else 1)) * 4
     return qkvo + text + gates
 
 
@@ -431,7 +433,7 @@ def roofline(w, stage_ms, hbm_gbs, peak_src, bf16_tflops=1607.7):
         fr = [t for t in range(5 * c, min(5 * c + 5, T)) if not (w.anchors and t in (0, T - 1))]
         steps += len(fr) if tensor_path else max(0, len(range(5 * c, min(5 * c + 5, T))) - 1)
     units = {
-        "frame_grams": ("hbm", frames * (2 * U * d * e + 2 * d * d * 4)),
+        "frame_grams": ("hbm", frames * (2 * U * d * e + 2 * d * d * 4 + (U * 4 if w.beta_per_token else 0))),
         "chunk_readout": ("hbm", frames * 2 * U * d * e + BH * C * 2 * d * d * 4),
         "frame_factor": ("alu", live * (d ** 3 // 4 if tensor_path else 4 * d ** 3)),
         "chunk_compose": ("tensor" if tensor_path else "alu", BH * 2 * steps * 4 * d ** 3),

@@ -55,7 +55,7 @@ vdn_status cuda_fail(cudaError_t e, const char *where) {
 
 struct Geo {
   long long BH;
-  int T, U, D, C, chunk, anchors, n_text, in_dtype, out_dtype;
+  int T, U, D, C, chunk, anchors, n_text, in_dtype, out_dtype, tokb;
   size_t in_elem, out_elem;
 };
 
@@ -69,6 +69,8 @@ vdn_status check_shape(const vdn_shape *s, Geo *g) {
     return fail(VDN_ERR_UNSUPPORTED, "d = %d not in {16, 32, 64, 128}", s->dk);
   if (s->chunk < 1 || s->chunk > 16) return fail(VDN_ERR_INVALID, "chunk = %d not in [1, 16]", s->chunk);
   if (s->anchors != 0 && s->anchors != 1) return fail(VDN_ERR_INVALID, "anchors must be 0 or 1");
+  if (s->beta_per_token != 0 && s->beta_per_token != 1)
+    return fail(VDN_ERR_INVALID, "beta_per_token must be 0 or 1");
   if ((s->in_dtype != VDN_F32 && s->in_dtype != VDN_BF16) ||
       (s->out_dtype != VDN_F32 && s->out_dtype != VDN_BF16))
     return fail(VDN_ERR_INVALID, "dtype must be VDN_F32 or VDN_BF16");
@@ -82,6 +84,7 @@ vdn_status check_shape(const vdn_shape *s, Geo *g) {
   g->n_text = s->n_text;
   g->in_dtype = s->in_dtype;
   g->out_dtype = s->out_dtype;
+  g->tokb = s->beta_per_token;
   g->in_elem = s->in_dtype == VDN_BF16 ? 2 : 4;
   g->out_elem = s->out_dtype == VDN_BF16 ? 2 : 4;
   if (g->BH * (long long)(g->T > 0 ? g->T : 1) > 0x7fffffffLL)
@@ -127,9 +130,10 @@ vdn_status run_grams(const Geo &g, const void *K, const void *V, const float *be
     return VDN_OK;
   }
   if (gram_tc_supported(g.in_dtype, g.D, U)) {
-    VDN_CUDA(launch_gram_tc(K, V, beta, A, Bm, nframes, U, info, st), "gram_tc");
+    VDN_CUDA(launch_gram_tc(K, V, beta, g.tokb != 0, A, Bm, nframes, U, info, st), "gram_tc");
   } else {
-    VDN_CUDA(launch_gram_simt(K, V, g.in_dtype, beta, A, Bm, nframes, U, g.D, st), "gram_simt");
+    VDN_CUDA(launch_gram_simt(K, V, g.in_dtype, beta, g.tokb != 0, A, Bm, nframes, U, g.D, st),
+             "gram_simt");
   }
   return VDN_OK;
 }
@@ -546,7 +550,7 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
     const bool run = gi < G_ && frames;
     const long long b0 = run ? lo(gi) : 0, nbh = run ? lo(gi + 1) - b0 : 0;
     if (run)
-      VDN_TRY(run_grams(g, tok(K, b0), tok(V, b0), beta + b0 * T, A + b0 * T * DD, Bm + b0 * T * DD, nbh * T,
+      VDN_TRY(run_grams(g, tok(K, b0), tok(V, b0), beta + b0 * T * (g.tokb ? U : 1), A + b0 * T * DD, Bm + b0 * T * DD, nbh * T,
                         (int)U, info, st));
     VDN_CUDA(cudaEventRecord(ev(base + 0), st), "event record");
     VDN_CUDA(cudaStreamWaitEvent(ax, ev(base + 0), 0), "stream wait");

@@ -1,7 +1,7 @@
 // Frame statistics on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
 // Paper: "Video DeltaNet: A Video-Native Hybrid Attention for Livestream
 // Video Generation" (summary page), "Method steps" step (3):
-//   A_t = beta_t K_t^T K_t,   B_t = beta_t V_t^T K_t   (bf16 in, fp32 out, d = 128).
+//   A_t = K_t^T Diag(beta_t) K_t,   B_t = V_t^T Diag(beta_t) K_t   (bf16 in, fp32 out, d = 128).
 //
 // One MMA stream per frame computes D = K^T [K | V] (M = 128, N = 256,
 // contraction over the frame's U tokens): columns 0..127 of D are A_t and
@@ -11,10 +11,17 @@
 // index, channel = M/N index). K-block stride 1024 B per 8 tokens, M/N-block
 // stride 8 KB.
 //
-// Persistent kernel, one CTA per SM, 6 warps:
+// With one gate per frame, beta_t scales the fp32 sums in the epilogue. With
+// one gate per token ("Core method": beta_{t,u}), four more warps write a
+// copy of each K tile with row u scaled by beta_{t,u}, split into bf16 hi and
+// lo parts (hi + lo = beta k to ~2^-17), and two MMAs per step compute
+// (Diag(beta) K)^T [K | V] instead.
+//
+// Persistent kernel, one CTA per SM, 6 warps (10 with per-token gates):
 //   warp 0     : TMA producer (4 loads of 8 KB per 64-token stage)
 //   warp 1     : TMEM allocator and single-thread MMA issuer
-//   warps 2..5 : epilogue: TMEM -> registers -> scaled fp32 stores
+//   warps 2..5 : epilogue: TMEM -> registers -> fp32 stores
+//   warps 6..9 : (per-token gates) the scaled K tile of each stage
 // TMEM holds two 256-column accumulators so a frame's epilogue overlaps the
 // next frame's MMAs. Every wait is bounded (see common.cuh).
 #include <cudaTypedefs.h>
@@ -27,13 +34,17 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kUT = 64;                          // tokens per pipeline stage
-constexpr int kStages = 4;
-constexpr int kStageBytes = 4 * kUT * 128;       // K lo, K hi, V lo, V hi blocks
+constexpr int kStagesMax = 4;
 constexpr int kBlockBytes = kUT * 128;           // one 64-channel block
-constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kBarBytes = 8 * (2 * kStages + 2 + 2 + 1);
-constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + kBarBytes + 16;
+constexpr int kBarBytes = 8 * (3 * kStagesMax + 2 + 2 + 1);
+// per stage: the K and V blocks of channels 0..63 and 64..127 (+ the scaled
+// K blocks: hi part of both, then lo part of both)
+template <bool TOKB> constexpr int kStagesT = TOKB ? 3 : 4;
+template <bool TOKB> constexpr int kStageBytesT = (TOKB ? 8 : 4) * kBlockBytes;
+template <bool TOKB> constexpr int kThreadsT = TOKB ? 320 : 192;
+template <bool TOKB>
+constexpr size_t kSmemBytesT = 1024 + (size_t)kStagesT<TOKB> * kStageBytesT<TOKB> + kBarBytes + 16;
 
 struct GramArgs {
   float *A;
@@ -42,6 +53,7 @@ struct GramArgs {
   int32_t *info;
   long long nframes;
   int ntiles;
+  int U;
 };
 
 __device__ __forceinline__ void fail(volatile int *abort, int32_t *info) {
@@ -49,9 +61,12 @@ __device__ __forceinline__ void fail(volatile int *abort, int32_t *info) {
   if (info) atomicExch(info, VDN_INFO_TIMEOUT);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool TOKB>
+__global__ void __launch_bounds__(kThreadsT<TOKB>, 1)
     gram_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    GramArgs p) {
+  constexpr int kStageBytes = kStageBytesT<TOKB>;
+  constexpr int kStages = kStagesT<TOKB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -66,6 +81,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tfull0 = empty0 + 8 * kStages;
   const uint32_t tempty0 = tfull0 + 16;
   const uint32_t drain = tempty0 + 16;
+  const uint32_t scaled0 = drain + 8;  // per stage: the scaled K tile is written
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -77,6 +93,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(tempty0 + 8 * b, 128);
     }
     mbar_init(drain, 1);
+    if (TOKB)
+      for (int s = 0; s < kStages; ++s) mbar_init(scaled0 + 8 * s, 128);
     *abort = 0;
     fence_barrier_init();
   }
@@ -104,7 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t dst = smem_u32(stages + stage * kStageBytes);
           const uint32_t fb = full0 + 8 * stage;
-          mbar_arrive_expect_tx(fb, kStageBytes);
+          mbar_arrive_expect_tx(fb, 4 * kBlockBytes);  // the four TMA blocks
           armed_parity[stage] = (int)phase;
           const int y = j * kUT, z = (int)f;
           tma_load_3d(dst + 0 * kBlockBytes, &tmK, fb, 0, y, z);
@@ -140,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t dcol = tmem_base + (uint32_t)(buf * 256);
         for (int j = 0; j < p.ntiles; ++j) {
-          if (!mbar_wait(full0 + 8 * stage, phase, abort)) {
+          if (!mbar_wait((TOKB ? scaled0 : full0) + 8 * stage, phase, abort)) {
             fail(abort, p.info);
             ok = false;
             break;
@@ -149,8 +167,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t base = smem_u32(stages + stage * kStageBytes);
 #pragma unroll
           for (int ks = 0; ks < kUT / 16; ++ks) {
-            const uint64_t desc = smem_desc_sw128(base + ks * 2048, kBlockBytes, 1024);
-            tc_mma_bf16(dcol, desc, desc, idesc, (j > 0 || ks > 0) ? 1u : 0u);
+            const uint64_t bdesc = smem_desc_sw128(base + ks * 2048, kBlockBytes, 1024);
+            if (TOKB) {
+              // (Diag(beta) K)^T as its hi and lo parts
+#pragma unroll
+              for (int part = 0; part < 2; ++part) {
+                const uint32_t abase = base + (4 + 2 * part) * kBlockBytes;
+                const uint64_t adesc = smem_desc_sw128(abase + ks * 2048, kBlockBytes, 1024);
+                tc_mma_bf16(dcol, adesc, bdesc, idesc, (j > 0 || ks > 0 || part > 0) ? 1u : 0u);
+              }
+            } else {
+              tc_mma_bf16(dcol, bdesc, bdesc, idesc, (j > 0 || ks > 0) ? 1u : 0u);
+            }
           }
           tc_commit(empty0 + 8 * stage);
           if (++stage == kStages) {
@@ -164,6 +192,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(drain);
       volatile int never = 0;
       mbar_wait(drain, 0, &never);
+    }
+  } else if (TOKB && warp >= 6) {
+    // scaled copy of each K tile: row u (token j * 64 + u) times beta_{t,u},
+    // split into bf16 hi and lo, at the same offsets (the swizzle permutes
+    // 16-byte chunks inside a row, so a row is its 128-byte line)
+    const int st_ = threadIdx.x - 192;         // 0..127
+    const int blk = st_ >> 6, r = st_ & 63;    // one 128-byte row (token r) of one K block
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (long long f = blockIdx.x; ok && f < p.nframes; f += gridDim.x) {
+      const float *bf = p.beta + f * (long long)p.U;
+      for (int j = 0; j < p.ntiles; ++j) {
+        const int u = j * kUT + r;
+        const float b = u < p.U ? __ldg(bf + u) : 0.f;  // in flight during the wait
+        if (!mbar_wait(full0 + 8 * stage, phase, abort)) {
+          fail(abort, p.info);
+          ok = false;
+          break;
+        }
+        uint8_t *row = stages + stage * kStageBytes + blk * kBlockBytes + r * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          // rotate the chunk order by row so a warp's 16-byte accesses spread over the banks
+          const int off = ((c + r) & 7) * 16;
+          const uint4 x = *reinterpret_cast<const uint4 *>(row + off);
+          const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            split_bf16x2(b * __uint_as_float(w[e] << 16), b * __uint_as_float(w[e] & 0xFFFF0000u), hi[e], lo[e]);
+          *reinterpret_cast<uint4 *>(row + 4 * kBlockBytes + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4 *>(row + 6 * kBlockBytes + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(scaled0 + 8 * stage);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
     }
   } else {
     // epilogue warps 2..5 -> TMEM sub-partitions 2, 3, 0, 1
@@ -181,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const float bt = p.beta[f];
+      const float bt = TOKB ? 1.f : p.beta[f];
       float *Af = p.A + f * (long long)(kD * kD);
       float *Bf = p.Bm + f * (long long)(kD * kD);
 #pragma unroll 1
@@ -227,20 +296,25 @@ bool make_rows_map(CUtensorMap *m, const void *base, long long frames, int rows,
   return r == CUDA_SUCCESS;
 }
 
-cudaError_t launch_gram_tc(const void *K, const void *V, const float *beta, float *A, float *Bm,
-                           long long nframes, int U, int32_t *info, cudaStream_t st) {
+template <bool TOKB>
+cudaError_t launch_gram_t(const CUtensorMap &tmK, const CUtensorMap &tmV, const GramArgs &a, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(gram_tc_kernel<TOKB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBytesT<TOKB>);
+  if (e != cudaSuccess) return e;
+  const int sms = device_sm_count();
+  const long long grid = a.nframes < sms ? a.nframes : sms;
+  gram_tc_kernel<TOKB><<<(unsigned)grid, kThreadsT<TOKB>, kSmemBytesT<TOKB>, st>>>(tmK, tmV, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gram_tc(const void *K, const void *V, const float *beta, bool per_token, float *A,
+                           float *Bm, long long nframes, int U, int32_t *info, cudaStream_t st) {
   if (nframes <= 0) return cudaSuccess;
   CUtensorMap tmK, tmV;
   if (!make_rows_map(&tmK, K, nframes, U, kUT) || !make_rows_map(&tmV, V, nframes, U, kUT))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBytes);
-  if (e != cudaSuccess) return e;
-  const int sms = device_sm_count();
-  const long long grid = nframes < sms ? nframes : sms;
-  GramArgs a{A, Bm, beta, info, nframes, (U + kUT - 1) / kUT};
-  gram_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(tmK, tmV, a);
-  return cudaGetLastError();
+  GramArgs a{A, Bm, beta, info, nframes, (U + kUT - 1) / kUT, U};
+  return per_token ? launch_gram_t<true>(tmK, tmV, a, st) : launch_gram_t<false>(tmK, tmV, a, st);
 }
 
 }  // namespace vdn

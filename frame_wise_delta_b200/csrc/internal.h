@@ -9,8 +9,9 @@
 namespace vdn {
 
 // Generic CUDA-core kernels: any d in {16, 32, 64, 128}, float32 or bf16 inputs.
-cudaError_t launch_gram_simt(const void *K, const void *V, int in_dtype, const float *beta, float *A,
-                             float *Bm, long long nframes, int U, int D, cudaStream_t st);
+// beta: one gate per frame ([nframes]) or, with per_token, per token ([nframes, U])
+cudaError_t launch_gram_simt(const void *K, const void *V, int in_dtype, const float *beta, bool per_token,
+                             float *A, float *Bm, long long nframes, int U, int D, cudaStream_t st);
 cudaError_t launch_factor_simt(const float *A, const float *Bm, const float *alpha, float *M,
                                float *J, int32_t *info, long long nframes, int T, int anchors, int D,
                                cudaStream_t st);
@@ -26,8 +27,8 @@ cudaError_t launch_readout_simt(const void *Q, int in_dtype, const float *F, con
 
 // Tensor-core kernels (tcgen05 + TMA), bf16 inputs, d = 128.
 bool gram_tc_supported(int in_dtype, int D, int U);
-cudaError_t launch_gram_tc(const void *K, const void *V, const float *beta, float *A, float *Bm,
-                           long long nframes, int U, int32_t *info, cudaStream_t st);
+cudaError_t launch_gram_tc(const void *K, const void *V, const float *beta, bool per_token, float *A,
+                           float *Bm, long long nframes, int U, int32_t *info, cudaStream_t st);
 bool readout_tc_supported(int in_dtype, int out_dtype, int D, int U);
 cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, void *O, long long BH,
                               int T, int U, int chunk, int anchors, int32_t *info, cudaStream_t st);

@@ -81,6 +81,9 @@ extern "C" vdn_status vdn_text_state_noalloc(const vdn_shape *s, const void *Kx,
     return fail(VDN_ERR_UNSUPPORTED, "need dk == dv in {16, 32, 64, 128}");
   if (s->in_dtype != VDN_F32 && s->in_dtype != VDN_BF16)
     return fail(VDN_ERR_INVALID, "in_dtype must be VDN_F32 or VDN_BF16");
+  if (s->beta_per_token != 0 && s->beta_per_token != 1)
+    return fail(VDN_ERR_INVALID, "beta_per_token must be 0 or 1");
+  const bool tokb = s->beta_per_token != 0;
   const long long BH = (long long)s->B * s->H;
   const int D = s->dk;
   const size_t per = (size_t)BH * D * D;  // floats of one Gram matrix set
@@ -111,9 +114,9 @@ extern "C" vdn_status vdn_text_state_noalloc(const vdn_shape *s, const void *Kx,
   float *Ax = scratch;
   float *Bx = scratch + per;
   if (gram_tc_supported(s->in_dtype, D, s->n_text))
-    e = launch_gram_tc(Kx, Vx, beta_x, Ax, Bx, BH, s->n_text, info, st);
+    e = launch_gram_tc(Kx, Vx, beta_x, tokb, Ax, Bx, BH, s->n_text, info, st);
   else
-    e = launch_gram_simt(Kx, Vx, s->in_dtype, beta_x, Ax, Bx, BH, s->n_text, D, st);
+    e = launch_gram_simt(Kx, Vx, s->in_dtype, beta_x, tokb, Ax, Bx, BH, s->n_text, D, st);
   if (e != cudaSuccess) return fail(VDN_ERR_CUDA, "text gram: %s", cudaGetErrorString(e));
   e = launch_factor_simt(Ax, Bx, nullptr, nullptr, S_T, info, BH, 1, 0, D, st);
   if (e != cudaSuccess) return fail(VDN_ERR_CUDA, "text factor: %s", cudaGetErrorString(e));

@@ -24,6 +24,7 @@ template <int D, typename Tin>
 __global__ void __launch_bounds__(kThreads) gram_simt_kernel(const Tin *__restrict__ K,
                                                             const Tin *__restrict__ V,
                                                             const float *__restrict__ beta,
+                                                            bool per_token,
                                                             float *__restrict__ A,
                                                             float *__restrict__ Bm, int U) {
   constexpr int R = D / 16;
@@ -48,6 +49,7 @@ __global__ void __launch_bounds__(kThreads) gram_simt_kernel(const Tin *__restri
       if (u < U) {
         xv = to_f32(Xf[(long long)u * D + c]);
         kv = to_f32(Kf[(long long)u * D + c]);
+        if (per_token) kv *= beta[f * U + u];  // K^T Diag(beta) [K | V]
       }
       Xs[uu][c] = xv;
       Ks[uu][c] = kv;
@@ -67,7 +69,7 @@ __global__ void __launch_bounds__(kThreads) gram_simt_kernel(const Tin *__restri
     }
     __syncthreads();
   }
-  const float bt = beta[f];
+  const float bt = per_token ? 1.f : beta[f];
   float *out = (which == 0 ? A : Bm) + f * (long long)D * D;
 #pragma unroll
   for (int a = 0; a < R; ++a)
@@ -401,15 +403,15 @@ __global__ void __launch_bounds__(kThreads) readout_simt_kernel(
 }
 
 template <int D>
-cudaError_t gram_d(const void *K, const void *V, int in_dtype, const float *beta, float *A,
+cudaError_t gram_d(const void *K, const void *V, int in_dtype, const float *beta, bool per_token, float *A,
                    float *Bm, long long nframes, int U, cudaStream_t st) {
   dim3 grid((unsigned)nframes, 2);
   if (in_dtype == VDN_BF16)
     gram_simt_kernel<D, __nv_bfloat16><<<grid, kThreads, 0, st>>>(
-        (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V, beta, A, Bm, U);
+        (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V, beta, per_token, A, Bm, U);
   else
     gram_simt_kernel<D, float><<<grid, kThreads, 0, st>>>((const float *)K, (const float *)V, beta,
-                                                          A, Bm, U);
+                                                          per_token, A, Bm, U);
   return cudaGetLastError();
 }
 
@@ -478,10 +480,10 @@ cudaError_t readout_d(const void *Q, int in_dtype, const float *F, const float *
     default: return cudaErrorInvalidValue;     \
   }
 
-cudaError_t launch_gram_simt(const void *K, const void *V, int in_dtype, const float *beta, float *A,
-                             float *Bm, long long nframes, int U, int D, cudaStream_t st) {
+cudaError_t launch_gram_simt(const void *K, const void *V, int in_dtype, const float *beta, bool per_token,
+                             float *A, float *Bm, long long nframes, int U, int D, cudaStream_t st) {
   if (nframes <= 0) return cudaSuccess;
-  VDN_DISPATCH_D(D, gram_d<DD_>(K, V, in_dtype, beta, A, Bm, nframes, U, st))
+  VDN_DISPATCH_D(D, gram_d<DD_>(K, V, in_dtype, beta, per_token, A, Bm, nframes, U, st))
 }
 
 cudaError_t launch_factor_simt(const float *A, const float *Bm, const float *alpha, float *M,

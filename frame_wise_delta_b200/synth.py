@@ -25,7 +25,7 @@ import numpy as np
 BASE_SEED = 20260917
 
 # tensor ids used to key the per-(b, h) random streams
-_TID = {"Q": 0, "K": 1, "V": 2, "Kx": 3, "Vx": 4, "beta": 5, "alpha": 6, "proto": 7}
+_TID = {"Q": 0, "K": 1, "V": 2, "Kx": 3, "Vx": 4, "beta": 5, "alpha": 6, "proto": 7, "beta_x": 8}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -39,6 +39,8 @@ class Workload:
     anchors: 1 when the first and last frames are softmax anchors that the
     linear branch skips.
     near_dup: keys of a frame cluster around a few prototypes (cosine 0.99).
+    beta_per_token: one write gate per token, beta [T, U] and beta_x
+    [n_text] ~ U(beta_lo, 1); otherwise beta [T] per frame and beta_x = 1.
     """
 
     name: str
@@ -55,6 +57,7 @@ class Workload:
     near_dup: bool = False
     chunk: int = 5
     beta_lo: float = 0.1
+    beta_per_token: bool = False
 
     @property
     def seed(self) -> int:
@@ -86,6 +89,11 @@ WORKLOADS = {
                  alpha_lo=0.95, anchors=1),
         Workload("batched", 4, B=4, H=24, T=102, U=1920, d=128, n_text=256, dtype="bf16",
                  alpha_lo=0.95, anchors=1, near_dup=True),
+        # per-token write gates beta_{t,u} ("Core method" objective)
+        Workload("small_tb", 5, B=1, H=4, T=20, U=256, d=64, n_text=64, dtype="f32",
+                 alpha_lo=0.9, anchors=1, beta_per_token=True),
+        Workload("h3_tb", 6, B=1, H=24, T=102, U=1008, d=128, n_text=512, dtype="bf16",
+                 alpha_lo=0.95, anchors=1, beta_per_token=True),
     ]
 }
 
@@ -152,9 +160,12 @@ def generate_head(w: Workload, b: int, h: int, parts=ALL_PARTS) -> dict:
         "V": lambda: _store(w, _rng(w, b, h, "V").standard_normal((T, U, d), dtype=np.float32)),
         "Kx": lambda: _store(w, _unit_rows(_rng(w, b, h, "Kx").standard_normal((w.n_text, d), dtype=np.float32))),
         "Vx": lambda: _store(w, _rng(w, b, h, "Vx").standard_normal((w.n_text, d), dtype=np.float32)),
-        "beta": lambda: _rng(w, b, h, "beta").uniform(w.beta_lo, 1.0, size=T).astype(np.float32),
+        "beta": lambda: _rng(w, b, h, "beta").uniform(
+            w.beta_lo, 1.0, size=(T, U) if w.beta_per_token else T).astype(np.float32),
         "alpha": lambda: _rng(w, b, h, "alpha").uniform(w.alpha_lo, 1.0, size=(T, d)).astype(np.float32),
-        "beta_x": lambda: np.float32(1.0),
+        # per-token gates also gate the text tokens; otherwise beta_x = 1
+        "beta_x": lambda: (_rng(w, b, h, "beta_x").uniform(w.beta_lo, 1.0, size=w.n_text).astype(np.float32)
+                           if w.beta_per_token else np.float32(1.0)),
     }
     return {k: make[k]() for k in parts}
 
@@ -168,9 +179,9 @@ def generate_all(w: Workload, threads: int = 8) -> dict:
         "V": np.empty((w.B, w.H, w.T, w.U, w.d), np.float32),
         "Kx": np.empty((w.B, w.H, w.n_text, w.d), np.float32),
         "Vx": np.empty((w.B, w.H, w.n_text, w.d), np.float32),
-        "beta": np.empty((w.B, w.H, w.T), np.float32),
+        "beta": np.empty((w.B, w.H, w.T, w.U) if w.beta_per_token else (w.B, w.H, w.T), np.float32),
         "alpha": np.empty((w.B, w.H, w.T, w.d), np.float32),
-        "beta_x": np.empty((w.B, w.H), np.float32),
+        "beta_x": np.empty((w.B, w.H, w.n_text) if w.beta_per_token else (w.B, w.H), np.float32),
     }
 
     def fill(bh):

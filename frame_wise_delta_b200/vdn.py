@@ -33,23 +33,25 @@ class VdnError(RuntimeError):
 
 class vdn_shape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
-                ("B", "H", "T", "U", "dk", "dv", "n_text", "chunk", "anchors", "in_dtype", "out_dtype")]
+                ("B", "H", "T", "U", "dk", "dv", "n_text", "chunk", "anchors", "in_dtype", "out_dtype",
+                 "beta_per_token")]
 
     @property
     def C(self) -> int:
         return -(-self.T // self.chunk) if self.T > 0 else 0
 
 
-def make_shape(B, H, T, U, d, n_text, chunk=5, anchors=0, in_dtype="bf16", out_dtype=None) -> vdn_shape:
+def make_shape(B, H, T, U, d, n_text, chunk=5, anchors=0, in_dtype="bf16", out_dtype=None,
+               beta_per_token=False) -> vdn_shape:
     in_dt = _DTYPES[in_dtype]
     out_dt = in_dt if out_dtype is None else _DTYPES[out_dtype]
-    return vdn_shape(B, H, T, U, d, d, n_text, chunk, anchors, in_dt, out_dt)
+    return vdn_shape(B, H, T, U, d, d, n_text, chunk, anchors, in_dt, out_dt, int(bool(beta_per_token)))
 
 
 def shape_for(w, B=None, H=None) -> vdn_shape:
     """Shape of a synth.Workload (optionally with other batch/head counts)."""
     return make_shape(w.B if B is None else B, w.H if H is None else H, w.T, w.U, w.d, w.n_text,
-                      w.chunk, w.anchors, w.dtype)
+                      w.chunk, w.anchors, w.dtype, beta_per_token=w.beta_per_token)
 
 
 _lib = None

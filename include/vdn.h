@@ -73,14 +73,24 @@ typedef struct {
   int32_t anchors;    /* 1: frames 0 and T-1 are anchors (no write, no read) */
   int32_t in_dtype;   /* vdn_dtype of Q, K, V, Kx, Vx */
   int32_t out_dtype;  /* vdn_dtype of O */
+  int32_t beta_per_token; /* 0: one write gate per frame, beta [B,H,T] and
+                             beta_x [B,H]; 1: one per token ("Core method":
+                             beta_{t,u}), beta [B,H,T,U] and beta_x
+                             [B,H,n_text] */
 } vdn_shape;
 
 /*
  * Frame statistics. Paper: "Method steps", step (3):
  *   A_t = K_t^T Diag(beta_t) K_t   [d_k, d_k]   (symmetric)
  *   B_t = V_t^T Diag(beta_t) K_t   [d_v, d_k]
- * with one scalar write gate beta_t per (b, h, t).
- * In : K [B,H,T,U,dk], V [B,H,T,U,dv] (in_dtype); beta [B,H,T] float32.
+ * with one scalar write gate beta_t per (b, h, t), or (shape.beta_per_token)
+ * one gate beta_{t,u} per token.
+ * In : K [B,H,T,U,dk], V [B,H,T,U,dv] (in_dtype); beta [B,H,T] or
+ *      [B,H,T,U] float32.
+ * Precision of the tensor-core path (bf16, d = 128) with per-token gates:
+ * beta_{t,u} k_{t,u} is rounded to bf16 before the product (2^-9 relative per
+ * term); with one gate per frame the products are exact and beta_t scales the
+ * fp32 sums.
  * Out: A [B,H,T,dk,dk], Bm [B,H,T,dv,dk] float32 (fully overwritten).
  * Every frame, anchors included, is computed (the factor step skips anchors).
  * info: optional device int32 (may be NULL) that receives VDN_INFO_TIMEOUT if
@@ -181,7 +191,9 @@ vdn_status vdn_chunk_readout(const vdn_shape *s, const void *Q, const float *F,
  * state S^T that initialises both scans). Reading: one VDA update from the
  * zero state over the n_text text tokens, with gate beta_x and no decay:
  *   S_T = beta_x V_x^T K_x (I + beta_x K_x^T K_x)^{-1}.
- * In : Kx [B,H,n_text,dk], Vx [B,H,n_text,dv] (in_dtype); beta_x [B,H] float32.
+ * In : Kx [B,H,n_text,dk], Vx [B,H,n_text,dv] (in_dtype); beta_x [B,H]
+ *      float32, or [B,H,n_text] with shape.beta_per_token (then beta_x is a
+ *      per-token vector in the formula above: K_x^T Diag(beta_x) K_x).
  * Out: S_T [B,H,dv,dk] float32; *info as for vdn_frame_factor.
  * workspace: device scratch of at least vdn_text_state_workspace_bytes(s)
  * bytes, 256-byte aligned, not read before it is written.
@@ -216,7 +228,8 @@ vdn_status vdn_text_state_noalloc(const vdn_shape *s, const void *Kx,
  * The whole linear branch in one call: text state, frame statistics,
  * factor, chunk composition, both scans and the chunk readout.
  * In : Q, K, V [B,H,T,U,d] and Kx, Vx [B,H,n_text,d] (in_dtype);
- *      beta [B,H,T], alpha [B,H,T,dk], beta_x [B,H] float32.
+ *      beta [B,H,T], alpha [B,H,T,dk], beta_x [B,H] float32 (beta
+ *      [B,H,T,U] and beta_x [B,H,n_text] with shape.beta_per_token).
  * Out: O [B,H,T,U,dv] (out_dtype). If F and G are not NULL they receive the
  *      boundary states [B,H,C+1,dv,dk]; *info as for vdn_frame_factor.
  * workspace: at least vdn_forward_workspace_bytes(s) bytes, 256-byte aligned.

@@ -135,3 +135,17 @@ def test_pipelined_validation(L):
     ev[9] = None  # 7 + 3 * 2 = 13 events, one missing
     assert L.vdn_forward_pipelined(*args, 2, None, evp, None) == vdn.VDN_ERR_INVALID
     assert "events[9]" in vdn.vdn_last_error()
+
+
+def test_beta_per_token_flag_is_checked(L):
+    s = _shape()
+    s.beta_per_token = 2
+    assert L.vdn_frame_grams(_p(s), 16, 16, 16, 16, 16, None, None) == vdn.VDN_ERR_INVALID
+    assert "beta_per_token" in vdn.vdn_last_error()
+    assert L.vdn_text_state_noalloc(_p(s), 16, 16, 16, 16, 16, None) == vdn.VDN_ERR_INVALID
+    assert vdn.shape_for(vdn_synth().WORKLOADS["h3_tb"]).beta_per_token == 1
+
+
+def vdn_synth():
+    from frame_wise_delta_b200 import synth
+    return synth

@@ -35,7 +35,12 @@ BF16_D64 = custom("bf16_d64", index=42, d=64, U=130, T=17)
 # float32 with d = 32, no anchors, ragged chunk
 F32_D32 = custom("f32_d32", index=43, dtype="f32", d=32, U=70, T=13, anchors=0, n_text=5)
 
-SMALL_CASES = [W["tiny"], W["small"], TC_SMALL, TC_DUP, BF16_D64, F32_D32]
+# per-token write gates beta_{t,u}: the tensor-core Gram (scaled K tiles), the
+# CUDA-core Gram on bf16 and on float32 inputs
+TC_TB = custom("tc_tb", index=56, B=1, H=3, T=13, U=200, n_text=40, beta_per_token=True)
+BF16_D64_TB = custom("bf16_d64_tb", index=57, d=64, U=130, T=11, beta_per_token=True)
+
+SMALL_CASES = [W["tiny"], W["small"], TC_SMALL, TC_DUP, BF16_D64, F32_D32, W["small_tb"], TC_TB, BF16_D64_TB]
 
 
 def _full(w):
@@ -322,7 +327,8 @@ def test_nonpositive_pivot_is_reported():
 
 
 # ------------------------------------------------------------ full size
-FULL = [("h3", [(0, 0), (0, 23)]), ("long", [(0, 5)]), ("batched", [(0, 0), (3, 17)])]
+FULL = [("h3", [(0, 0), (0, 23)]), ("long", [(0, 5)]), ("batched", [(0, 0), (3, 17)]),
+        ("h3_tb", [(0, 7)])]
 
 
 @pytest.mark.parametrize("name,pairs", FULL, ids=[f[0] for f in FULL])

@@ -341,3 +341,59 @@ def test_synthetic_workloads_have_the_stated_statistics():
     assert np.all(inp["alpha"] >= 0.95) and np.all(inp["alpha"] <= 1.0)
     # bf16 storage: the low 16 bits are clear
     assert not np.any(inp["Q"].view(np.uint32) & 0xFFFF)
+
+
+# --- per-token write gates beta_{t,u} ("Core method" objective) -------------
+def test_zero_token_gates_drop_those_tokens():
+    # a token whose gate is 0 has no term in the frame objective, so the
+    # statistics equal those of the frame without it
+    rng = _rng(40)
+    K, V = _frame(rng, 9, 5, 4)
+    beta = rng.uniform(0.1, 1.0, 9)
+    keep = np.array([1, 0, 1, 1, 0, 0, 1, 1, 0], bool)
+    A, B = oracle.frame_stats(K, V, np.where(keep, beta, 0.0))
+    A2, B2 = oracle.frame_stats(K[keep], V[keep], beta[keep])
+    np.testing.assert_allclose(A, A2, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(B, B2, rtol=1e-13, atol=1e-13)
+
+
+def test_equal_token_gates_are_the_frame_gate():
+    w = synth.Workload("eq", 90, B=1, H=1, T=12, U=6, d=4, n_text=5, dtype="f32", alpha_lo=0.9,
+                       anchors=1)
+    inp = synth.generate_head(w, 0, 0)
+    tok = dict(inp)
+    tok["beta"] = np.repeat(inp["beta"][:, None], w.U, axis=1)
+    tok["beta_x"] = np.full(w.n_text, inp["beta_x"])
+    a, b = oracle.vda_head(inp, w.chunk, w.anchors), oracle.vda_head(tok, w.chunk, w.anchors)
+    for k in ("S_T", "F", "G", "O"):
+        np.testing.assert_allclose(b[k], a[k], rtol=1e-12, atol=1e-12)
+
+
+def test_per_token_scan_matches_frame_by_frame_brute_force():
+    # forward boundary states from the stacked least-squares solve of each
+    # frame's objective (per-token weights), chained by hand
+    rng = _rng(41)
+    T, U, d, chunk = 7, 3, 3, 2
+    K = np.stack([_frame(rng, U, d, d)[0] for _ in range(T)])
+    V = rng.standard_normal((T, U, d))
+    beta = rng.uniform(0.0, 1.5, (T, U))
+    alpha = rng.uniform(0.6, 1.0, (T, d))
+    S_T = rng.standard_normal((d, d))
+    F, G = oracle.scan_states(K, V, beta, alpha, S_T, chunk, anchors=0)
+    S = 0.5 * S_T
+    ref = [S]
+    for t in range(T):
+        S = _brute_frame(S * alpha[t][None, :], K[t], V[t], beta[t])
+        if (t + 1) % chunk == 0 or t == T - 1:
+            ref.append(S)
+    np.testing.assert_allclose(F, np.stack(ref), rtol=1e-9, atol=1e-9)
+
+
+def test_per_token_synthetic_gates():
+    w = synth.WORKLOADS["small_tb"]
+    inp = synth.generate_head(w, 0, 2)
+    assert inp["beta"].shape == (w.T, w.U) and inp["beta_x"].shape == (w.n_text,)
+    for x in (inp["beta"], inp["beta_x"]):
+        assert x.min() >= w.beta_lo and x.max() <= 1.0 and x.std() > 0.2
+    # the per-frame workloads keep their gates: the stream of beta is unchanged
+    assert synth.generate_head(synth.WORKLOADS["small"], 0, 2)["beta"].shape == (w.T,)

@@ -76,13 +76,18 @@ def device_fill(w: synth.Workload, sampled: dict, seed: int) -> dict:
             t[b].copy_(x.to(dt))
             del x
         dev[k] = t
-    dev["beta"] = torch.rand((B, H, T), generator=g, device="cuda") * 0.9 + 0.1
+    tb = w.beta_per_token
+    dev["beta"] = torch.rand((B, H, T, U) if tb else (B, H, T), generator=g, device="cuda") * 0.9 + 0.1
     dev["alpha"] = torch.rand((B, H, T, d), generator=g, device="cuda") * (1 - w.alpha_lo) + w.alpha_lo
-    dev["beta_x"] = torch.ones((B, H), device="cuda")
+    dev["beta_x"] = (torch.rand((B, H, w.n_text), generator=g, device="cuda") * 0.9 + 0.1 if tb
+                     else torch.ones((B, H), device="cuda"))
     for (b, h), inp in sampled.items():
         for k in ("Q", "K", "V", "Kx", "Vx"):
             dev[k][b, h].copy_(to_dev(inp[k], dt))
         for k in ("beta", "alpha"):
             dev[k][b, h].copy_(to_dev(inp[k]))
-        dev["beta_x"][b, h] = float(inp["beta_x"])
+        if tb:
+            dev["beta_x"][b, h].copy_(to_dev(inp["beta_x"]))
+        else:
+            dev["beta_x"][b, h] = float(inp["beta_x"])
     return dev
