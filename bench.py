@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--gated", action="store_true",
+                    help="time the pass with the readout epilogue (RMSNorm + sigmoid gate, synthetic gates)")
     ap.add_argument("--groups", type=int, default=1,
                     help="head groups of vdn_forward_pipelined (tensor path); 0 = plain vdn_forward")
     return ap.parse_args()
@@ -205,8 +207,10 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(w):
+def workload_config(w, gated=False):
     gates = "per-token write gates" if w.beta_per_token else "per-frame write gates"
+    if gated:
+        gates += ", gated RMSNorm readout epilogue"
     return {"workload": f"{w.name}: B={w.B} H={w.H} T={w.T} U={w.U} d_k=d_v={w.d} n_text={w.n_text} "
                         f"chunk={w.chunk} anchors={w.anchors} {w.dtype} inputs, fp32 state, {gates}",
             "global_batch": w.B, "frames": w.B * w.T, "tokens": w.B * w.T * w.U,
@@ -257,7 +261,14 @@ def main():
         host[k] = torch.from_numpy(full[k]).to(dt).pin_memory()
     for k in ("beta", "alpha", "beta_x"):
         host[k] = torch.from_numpy(np.ascontiguousarray(full[k])).pin_memory()
+    if args.gated:
+        # gate logits ~ N(0, 4) in the input dtype, RMSNorm weights ~ U(0.5, 1.5)
+        grng = np.random.default_rng(w.seed + 1000)
+        host["gate"] = torch.from_numpy(
+            (2.0 * grng.standard_normal((w.B, w.H, w.T, w.U, w.d), dtype=np.float32))).to(dt).pin_memory()
+        host["norm_w"] = torch.from_numpy(grng.uniform(0.5, 1.5, (w.H, w.d)).astype(np.float32)).pin_memory()
     d = {k: v.to(dev) for k, v in host.items()}
+    og = vdn.out_gate(d["gate"], d["norm_w"], 1e-6) if args.gated else None
     s = vdn.shape_for(w)
     B, H, T, U, D, C = w.B, w.H, w.T, w.U, w.d, w.C
     f32 = dict(dtype=torch.float32, device=dev)
@@ -282,7 +293,7 @@ def main():
         if G:
             fwd_dev.events = ev if ev is not None else warm_ev
         fwd_dev(d["Q"], d["K"], d["V"], d["beta"], d["alpha"], d["Kx"], d["Vx"], d["beta_x"],
-                events=None if G else ev)
+                events=None if G else ev, og=og)
     warm_ev = fwd_dev.events if G else None
     info = fwd_dev.info
 
@@ -319,7 +330,7 @@ def main():
     value = vdist.throughput(B * T, world, ms_per_step / 1e3)
 
     # ---- end to end: pinned host inputs -> device -> vdn_forward -> O to host
-    e2e = (e2e_measure(args, host, d, make_forward, stream, barrier, world, frames_all, dt)
+    e2e = (e2e_measure(args, host, d, make_forward, stream, barrier, world, frames_all, dt, og)
            if not args.no_e2e else None)
 
     if rank == 0:
@@ -329,9 +340,9 @@ def main():
             "metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "state_dtype": "f32",
-            "data": "synthetic", "config": workload_config(w),
+            "data": "synthetic", "config": workload_config(w, args.gated),
             "tokens_per_s": value * U,
-            "hbm_frac_whole_pass": alg_bytes(w) * world / (ms_per_step / 1e3) / (hbm_gbs * 1e9),
+            "hbm_frac_whole_pass": alg_bytes(w, args.gated) * world / (ms_per_step / 1e3) / (hbm_gbs * 1e9),
             "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
             "step_ms_min_max": [min(step_ms), max(step_ms)],
             "roofline": roof,
@@ -364,7 +375,7 @@ def pipelined_stage_ms(e, G):
     return out
 
 
-def e2e_measure(args, host, d, make_forward, stream, barrier, world, frames_all, dt):
+def e2e_measure(args, host, d, make_forward, stream, barrier, world, frames_all, dt, og=None):
     """Same metric through vdn_forward with the step's inputs copied from pinned
     host memory and O copied back, inside the timed region."""
     import torch
@@ -380,7 +391,7 @@ def e2e_measure(args, host, d, make_forward, stream, barrier, world, frames_all,
     def e2e_step():
         for k in host:
             d[k].copy_(host[k], non_blocking=True)
-        fwd(d["Q"], d["K"], d["V"], d["beta"], d["alpha"], d["Kx"], d["Vx"], d["beta_x"])
+        fwd(d["Q"], d["K"], d["V"], d["beta"], d["alpha"], d["Kx"], d["Vx"], d["beta_x"], og=og)
         O_host.copy_(fwd.O, non_blocking=True)
 
     for _ in range(2):
@@ -402,7 +413,7 @@ def e2e_measure(args, host, d, make_forward, stream, barrier, world, frames_all,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
 
-def alg_bytes(w):
+def alg_bytes(w, gated=False):
     """Algorithmic HBM bytes of the whole pass: Q, K, V read, O written (bf16),
     text keys/values read, gates read (write gates per frame or per token)."""
     e = 2 if w.dtype == "bf16" else 4
@@ -410,6 +421,8 @@ def alg_bytes(w):
     text = 2 * w.B * w.H * w.n_text * w.d * e
     tb = getattr(w, "beta_per_token", False)
     gates = w.B * w.H * (w.T * (w.d + (w.U if tb else 1)) + (w.n_text if tb else 1)) * 4
+    if gated:  # gate logits read once (input dtype) + RMSNorm weights
+        gates += w.B * w.H * w.T * w.U * w.d * e + w.H * w.d * 4
     return qkvo + text + gates
 
 

@@ -55,7 +55,7 @@ vdn_status cuda_fail(cudaError_t e, const char *where) {
 
 struct Geo {
   long long BH;
-  int T, U, D, C, chunk, anchors, n_text, in_dtype, out_dtype, tokb;
+  int H, T, U, D, C, chunk, anchors, n_text, in_dtype, out_dtype, tokb;
   size_t in_elem, out_elem;
 };
 
@@ -75,6 +75,7 @@ vdn_status check_shape(const vdn_shape *s, Geo *g) {
       (s->out_dtype != VDN_F32 && s->out_dtype != VDN_BF16))
     return fail(VDN_ERR_INVALID, "dtype must be VDN_F32 or VDN_BF16");
   g->BH = (long long)s->B * s->H;
+  g->H = s->H;
   g->T = s->T;
   g->U = s->U;
   g->D = s->dk;
@@ -138,17 +139,31 @@ vdn_status run_grams(const Geo &g, const void *K, const void *V, const float *be
   return VDN_OK;
 }
 
+// og: the readout epilogue (step (5)), or nullptr
 vdn_status run_readout(const Geo &g, const void *Q, const float *F, const float *G, void *O,
-                       int32_t *info, cudaStream_t st) {
+                       int32_t *info, cudaStream_t st, const OutGate *og = nullptr) {
   if (g.BH * g.T * g.U == 0) return VDN_OK;
   if (readout_tc_supported(g.in_dtype, g.out_dtype, g.D, g.U)) {
-    VDN_CUDA(launch_readout_tc(Q, F, G, O, g.BH, g.T, g.U, g.chunk, g.anchors, info, st),
+    VDN_CUDA(launch_readout_tc(Q, F, G, O, g.BH, g.T, g.U, g.chunk, g.anchors, info, st, og),
              "readout_tc");
   } else {
     VDN_CUDA(launch_readout_simt(Q, g.in_dtype, F, G, O, g.out_dtype, g.BH, g.T, g.U, g.chunk,
-                                 g.anchors, g.D, st),
+                                 g.anchors, g.D, st, og),
              "readout_simt");
   }
+  return VDN_OK;
+}
+
+// Validates a caller's vdn_out_gate (NULL allowed when `optional`) into *out.
+vdn_status check_gate(const Geo &g, const vdn_out_gate *og, bool optional, OutGate *out, const OutGate **use) {
+  *use = nullptr;
+  if (!og) return optional ? VDN_OK : fail(VDN_ERR_INVALID, "og is NULL");
+  const bool any = g.BH * g.T * g.U > 0;
+  VDN_TRY(need(og->gate, "og->gate", any));
+  VDN_TRY(need(og->norm_weight, "og->norm_weight", any));
+  if (!(og->eps > 0.f) || !(og->eps < 3.0e38f)) return fail(VDN_ERR_INVALID, "og->eps must be positive and finite");
+  *out = OutGate{og->gate, og->norm_weight, og->eps, g.H > 0 ? g.H : 1};
+  *use = out;
   return VDN_OK;
 }
 
@@ -315,6 +330,22 @@ vdn_status vdn_chunk_readout(const vdn_shape *s, const void *Q, const float *F, 
   return run_readout(g, Q, F, G, O, info, (cudaStream_t)stream);
 }
 
+vdn_status vdn_chunk_readout_gated(const vdn_shape *s, const void *Q, const float *F, const float *G,
+                                   const vdn_out_gate *og, void *O, int32_t *info, vdn_stream_t stream) {
+  g_err[0] = 0;
+  Geo g;
+  VDN_TRY(check_shape(s, &g));
+  const bool any = g.BH * g.T * g.U > 0;
+  VDN_TRY(need(Q, "Q", any));
+  VDN_TRY(need(F, "F", any));
+  VDN_TRY(need(G, "G", any));
+  VDN_TRY(need(O, "O", any));
+  OutGate og_;
+  const OutGate *use;
+  VDN_TRY(check_gate(g, og, false, &og_, &use));
+  return run_readout(g, Q, F, G, O, info, (cudaStream_t)stream, use);
+}
+
 size_t vdn_text_state_workspace_bytes(const vdn_shape *s) {
   Geo g;
   if (check_shape(s, &g) != VDN_OK) return 0;
@@ -403,7 +434,7 @@ vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K, const v
                        const float *beta, const float *alpha, const void *Kx, const void *Vx,
                        const float *beta_x, void *O, float *F, float *G, void *workspace,
                        size_t workspace_bytes, int32_t *info, const void *const *stage_events,
-                       vdn_stream_t stream) {
+                       const vdn_out_gate *og, vdn_stream_t stream) {
   g_err[0] = 0;
   Geo g;
   VDN_TRY(check_shape(s, &g));
@@ -420,6 +451,9 @@ vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K, const v
   if ((F && !aligned16(F)) || (G && !aligned16(G)))
     return fail(VDN_ERR_INVALID, "F/G not 16-byte aligned");
   VDN_TRY(need(info, "info", true));
+  OutGate gate_;
+  const OutGate *gate;
+  VDN_TRY(check_gate(g, og, true, &gate_, &gate));
   const FwdLayout L = fwd_layout(g);
   VDN_TRY(need(workspace, "workspace", g.BH > 0));
   if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
@@ -482,7 +516,7 @@ vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K, const v
     VDN_CUDA(launch_scan_simt(Mf, Jf, Mb, Jb, S_T, Fo, Go, g.BH, g.C, g.D, 3, st), "scan");
   }
   VDN_TRY(mark(5));
-  if (frames) VDN_TRY(run_readout(g, Q, Fo, Go, O, info, st));
+  if (frames) VDN_TRY(run_readout(g, Q, Fo, Go, O, info, st, gate));
   VDN_TRY(mark(6));
   return VDN_OK;
 }
@@ -492,7 +526,7 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
                                  const void *Vx, const float *beta_x, void *O, float *F, float *G,
                                  void *workspace, size_t workspace_bytes, int32_t *info,
                                  int32_t groups, vdn_stream_t aux, const void *const *events,
-                                 vdn_stream_t stream) {
+                                 const vdn_out_gate *og, vdn_stream_t stream) {
   g_err[0] = 0;
   Geo g;
   VDN_TRY(check_shape(s, &g));
@@ -515,6 +549,9 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
   if ((F && !aligned16(F)) || (G && !aligned16(G)))
     return fail(VDN_ERR_INVALID, "F/G not 16-byte aligned");
   VDN_TRY(need(info, "info", true));
+  OutGate gate_;
+  const OutGate *gate;
+  VDN_TRY(check_gate(g, og, true, &gate_, &gate));
   const FwdLayout L = fwd_layout(g);
   VDN_TRY(need(workspace, "workspace", g.BH > 0));
   if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
@@ -577,7 +614,7 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
   else if (g.BH > 0)
     VDN_CUDA(launch_scan_simt(nullptr, nullptr, nullptr, nullptr, S_T, Fo, Go, g.BH, g.C, g.D, 3, st), "scan");
   VDN_CUDA(cudaEventRecord(ev(tail + 2), st), "event record");
-  if (frames) VDN_TRY(run_readout(g, Q, Fo, Go, O, info, st));
+  if (frames) VDN_TRY(run_readout(g, Q, Fo, Go, O, info, st, gate));
   VDN_CUDA(cudaEventRecord(ev(tail + 3), st), "event record");
   return VDN_OK;
 }

@@ -21,9 +21,17 @@ cudaError_t launch_compose_simt(const float *M, const float *J, float *Mf, float
 cudaError_t launch_scan_simt(const float *Mf, const float *Jf, const float *Mb, const float *Jb,
                              const float *S_T, float *F, float *G, long long BH, int C, int D,
                              int dir_mask, cudaStream_t st);
+// Readout epilogue of step (5): y = o / sqrt(mean o^2 + eps) * w[h] * sigmoid(gate),
+// per token over its d channels; gate == nullptr leaves o as it is.
+struct OutGate {
+  const void *gate;  // [B,H,T,U,d], the input dtype
+  const float *w;    // [H, d]
+  float eps;
+  int H;
+};
 cudaError_t launch_readout_simt(const void *Q, int in_dtype, const float *F, const float *G, void *O,
                                 int out_dtype, long long BH, int T, int U, int chunk, int anchors,
-                                int D, cudaStream_t st);
+                                int D, cudaStream_t st, const OutGate *og = nullptr);
 
 // Tensor-core kernels (tcgen05 + TMA), bf16 inputs, d = 128.
 bool gram_tc_supported(int in_dtype, int D, int U);
@@ -31,7 +39,8 @@ cudaError_t launch_gram_tc(const void *K, const void *V, const float *beta, bool
                            float *Bm, long long nframes, int U, int32_t *info, cudaStream_t st);
 bool readout_tc_supported(int in_dtype, int out_dtype, int D, int U);
 cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, void *O, long long BH,
-                              int T, int U, int chunk, int anchors, int32_t *info, cudaStream_t st);
+                              int T, int U, int chunk, int anchors, int32_t *info, cudaStream_t st,
+                              const OutGate *og = nullptr);
 
 // W = (I + A)^{-1} per frame (CUDA cores); W fp32 and/or Wimg (hi/lo MMA
 // images of kImgBytes per frame, d = 128 only), each optional.

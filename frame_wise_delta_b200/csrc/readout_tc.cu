@@ -12,13 +12,19 @@
 // Operands are K-major and 128-byte swizzled: Q tiles come from TMA, R is
 // written by the CTA into the same layout.
 //
-// Persistent kernel, one CTA per SM, 6 warps; each CTA walks a contiguous
+// Optional epilogue ("Method steps" step (5): RMSNorm, then a sigmoid gate):
+// y = o / sqrt(mean o^2 + eps) * w[h] * sigmoid(g) per token, in two passes
+// over the token's TMEM row (mean square, then scale), with the tile's gate
+// logits brought by TMA into the staging tile that then receives y.
+//
+// Persistent kernel, one CTA per SM, 10 warps; each CTA walks a contiguous
 // range of frames so consecutive frames usually share a chunk and R is
 // rebuilt only when the chunk changes.
 //   warp 0     : TMA producer (two 16 KB loads per 128-token stage)
 //   warp 1     : TMEM allocator and single-thread MMA issuer
-//   warps 2..5 : R builder and epilogue (TMEM -> bf16 tile in shared memory ->
-//                TMA store, double-buffered; anchor frames
+//   warps 2..9 : R builder and epilogue in two groups of four warps that take
+//                alternate tiles (TMEM -> bf16 tile in the group's staging
+//                buffer in shared memory -> TMA store); anchor frames
 //                are written as zeros without touching the tensor cores)
 #include <cudaTypedefs.h>
 
@@ -38,9 +44,9 @@ constexpr int kRegionR = kD * 128;
 constexpr int kOBytes = kNT * 128 * 2;        // one bf16 O tile, two 64-channel regions
 constexpr int kRegionO = kNT * 128;
 constexpr int kAcc = 4;                       // TMEM accumulators (128 columns each)
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kBarBytes = 8 * (2 * kStages + 2 * kAcc + 2);
+constexpr int kBarBytes = 8 * (2 * kStages + 2 * kAcc + 2 + 2);
 constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 2 * kRBytes + 2 * kOBytes + kBarBytes + 16;
 
 struct ReadoutArgs {
@@ -50,6 +56,10 @@ struct ReadoutArgs {
   int32_t *info;
   long long nframes;
   int T, U, chunk, anchors, C, ntiles;
+  // gated RMSNorm epilogue (step (5))
+  const float *gw;  // [H, 128] RMSNorm weights, nullptr = no epilogue (gate logits through tmG)
+  float eps;
+  int H;
 };
 
 __device__ __forceinline__ void fail(volatile int *abort, int32_t *info) {
@@ -66,6 +76,13 @@ __device__ __forceinline__ long long chunk_key(const ReadoutArgs &p, long long f
   return (f / p.T) * p.C + (f % p.T) / p.chunk;
 }
 
+// tanh by the hardware approximation (PTX tanh.approx.f32, ~2^-11 relative)
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);  // a in the low half
   return *reinterpret_cast<const uint32_t *>(&h);
@@ -73,7 +90,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 
 __global__ void __launch_bounds__(kThreads, 1)
     readout_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
-                      ReadoutArgs p) {
+                      const __grid_constant__ CUtensorMap tmG, ReadoutArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -92,6 +109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tempty0 = tfull0 + 8 * kAcc;
   const uint32_t rfull = tempty0 + 8 * kAcc;
   const uint32_t drain = rfull + 8;
+  const uint32_t gfull0 = drain + 8;  // a group's gate tile has landed in its staging tile
 
   // contiguous, balanced frame range of this CTA
   const long long f_begin = p.nframes * blockIdx.x / gridDim.x;
@@ -108,6 +126,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(rfull, 1);
     mbar_init(drain, 1);
+    mbar_init(gfull0, 1);
+    mbar_init(gfull0 + 8, 1);
     *abort = 0;
     fence_barrier_init();
   }
@@ -207,31 +227,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(drain, 0, &never);
     }
   } else {
-    const int et = threadIdx.x - 64;  // 0..127
-    const int sub = warp & 3;
-    const int row = sub * 32 + lane;  // token of the tile held by this thread (TMEM lane)
+    const int et = threadIdx.x - 64;       // 0..255 over both groups
+    const int grp = (warp - 2) >> 2;        // tiles with (tile & 1) == grp
+    const int gt = et & 127;                // thread of the group
+    const int sub = warp & 3;               // TMEM sub-partition
+    const int row = sub * 32 + lane;        // token of the tile held by this thread (TMEM lane)
+    const int gbar = 1 + grp;               // the group's named barrier
+    uint8_t *ob = Obuf + grp * kOBytes;     // the group's staging tile
     uint32_t tile = 0;
     long long cur = -1;
     bool ok = true;  // after a failed wait: keep every barrier, skip the work
+    const bool gated = p.gw != nullptr;
+    const uint32_t gfull = gfull0 + 8 * grp;
+    uint32_t guse = 0;      // gate tiles this group has loaded
+    bool garmed = false;    // a gate load is armed and not yet waited for
     for (long long f = f_begin; f < f_end; ++f) {
       __nv_bfloat16 *Of = p.O + f * (long long)p.U * kD;
       if (is_anchor(p, f)) {
         uint4 z = make_uint4(0, 0, 0, 0);
         uint4 *o4 = reinterpret_cast<uint4 *>(Of);
         const long long n16 = (long long)p.U * kD / 8;
-        for (long long e = et; e < n16; e += 128) o4[e] = z;
+        for (long long e = et; e < n16; e += 256) o4[e] = z;
         continue;
       }
       const long long key = chunk_key(p, f);
       if (key != cur) {
-        // All MMAs that read the previous R have completed: every one of
-        // their tiles was drained below before we got here.
+        // Both groups have drained every tile of the previous chunk (their
+        // MMAs, which read the previous R, have completed) once they meet here.
+        asm volatile("bar.sync 3, 256;" ::: "memory");
         cur = key;
         const long long bh = f / p.T;
         const int c = (int)((f % p.T) / p.chunk);
         const float *Fs = p.F + (bh * (p.C + 1) + max(c - 1, 0)) * (long long)(kD * kD);
         const float *Gs = p.G + (bh * (p.C + 1) + min(c + 2, p.C)) * (long long)(kD * kD);
-        for (int e8 = et; e8 < kD * kD / 8; e8 += 128) {
+        for (int e8 = et; e8 < kD * kD / 8; e8 += 256) {
           const int i = e8 >> 4, k0 = (e8 & 15) * 8;
           const float4 *f4 = reinterpret_cast<const float4 *>(Fs + i * kD + k0);
           const float4 *g4 = reinterpret_cast<const float4 *>(Gs + i * kD + k0);
@@ -248,21 +277,80 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4 *>(Rlo + off) = l;
         }
         fence_proxy_async_smem();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 3, 256;" ::: "memory");
         if (et == 0) mbar_arrive(rfull);
       }
       for (int j = 0; j < p.ntiles; ++j, ++tile) {
+        if ((int)(tile & 1) != grp) continue;
         const int buf = (int)(tile % kAcc);
         const uint32_t use = tile / kAcc;
-        uint8_t *ob = Obuf + (tile & 1) * kOBytes;
-        // the TMA store that last read this staging tile (two tiles ago) is done
-        if (et == 0) bulk_wait_read<1>();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        // the group's previous TMA store has finished reading the staging tile
+        if (gt == 0) bulk_wait_read<0>();
+        asm volatile("bar.sync %0, 128;" ::"r"(gbar) : "memory");
+        // the tile's gate logits into the staging tile (same layout as O),
+        // coalesced by TMA while the MMA and pass 1 run
+        if (gated && ok && gt == 0) {
+          mbar_arrive_expect_tx(gfull, kOBytes);
+          tma_load_3d(smem_u32(ob), &tmG, gfull, 0, j * kNT, (int)f);
+          tma_load_3d(smem_u32(ob + kRegionO), &tmG, gfull, 64, j * kNT, (int)f);
+          garmed = true;
+        }
         if (ok && !__all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * buf, use & 1, abort))) {
           fail(abort, p.info);
           ok = false;
         }
-        if (ok) {
+        float rs = 0.f;
+        if (ok && gated) {
+          tc_fence_after();
+          // pass 1: this token's mean square over its 128 channels
+          float ss[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+          for (int cc = 0; cc < kD / 32; ++cc) {
+            float v[32];
+            tmem_ld32(tmem_base + (uint32_t)(buf * kNT + cc * 32) + ((uint32_t)(sub * 32) << 16), v);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ss[e & 3] = fmaf(v[e], v[e], ss[e & 3]);
+          }
+          rs = rsqrtf((ss[0] + ss[1] + ss[2] + ss[3]) * (1.0f / kD) + p.eps);
+          const bool gok = __all_sync(0xffffffffu, mbar_wait(gfull, guse & 1, abort));
+          ++guse;
+          if (gt == 0) garmed = false;
+          if (!gok) {
+            fail(abort, p.info);
+            ok = false;
+          }
+        }
+        if (ok && gated) {
+          // pass 2: y = o * rs * w * sigmoid(g), sigmoid(g) = (1 + tanh(g / 2)) / 2
+          const float *wv = p.gw + ((f / p.T) % p.H) * kD;
+#pragma unroll
+          for (int cc = 0; cc < kD / 32; ++cc) {
+            float v[32];
+            tmem_ld32(tmem_base + (uint32_t)(buf * kNT + cc * 32) + ((uint32_t)(sub * 32) << 16), v);
+            uint8_t *rb = ob + (cc >> 1) * kRegionO + row * 128;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int ch = (cc & 1) * 4 + q;
+              uint4 *slot = reinterpret_cast<uint4 *>(rb + ((ch ^ (row & 7)) << 4));
+              const uint4 g8 = *slot;
+              const uint32_t gw4[4] = {g8.x, g8.y, g8.z, g8.w};
+              const float4 w0 = *reinterpret_cast<const float4 *>(wv + cc * 32 + 8 * q);
+              const float4 w1 = *reinterpret_cast<const float4 *>(wv + cc * 32 + 8 * q + 4);
+              const float wq[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+              uint32_t y[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float g0 = __uint_as_float(gw4[e] << 16), g1 = __uint_as_float(gw4[e] & 0xFFFF0000u);
+                const float y0 = v[8 * q + 2 * e] * rs * wq[2 * e] * fmaf(0.5f, tanh_approx(0.5f * g0), 0.5f);
+                const float y1 = v[8 * q + 2 * e + 1] * rs * wq[2 * e + 1] * fmaf(0.5f, tanh_approx(0.5f * g1), 0.5f);
+                y[e] = pack_bf16(y0, y1);
+              }
+              *slot = make_uint4(y[0], y[1], y[2], y[3]);
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(tempty0 + 8 * buf);
+        } else if (ok) {
           tc_fence_after();
           // row `row` of the tile: 128 channels -> bf16, 16-byte chunks swizzled
           // as the tensor map's 128-byte swizzle expects
@@ -283,8 +371,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(tempty0 + 8 * buf);
         }
         fence_proxy_async_smem();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (ok && et == 0) {
+        asm volatile("bar.sync %0, 128;" ::"r"(gbar) : "memory");
+        if (ok && gt == 0) {
           // rows past U fall outside the tensor and are not written
           tma_store_3d(&tmO, smem_u32(ob), 0, j * kNT, (int)f);
           tma_store_3d(&tmO, smem_u32(ob + kRegionO), 64, j * kNT, (int)f);
@@ -292,7 +380,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (et == 0) bulk_wait_all();
+    if (gt == 0) {
+      bulk_wait_all();
+      // never leave with a gate load in flight (only after a failed wait)
+      volatile int never = 0;
+      if (garmed) mbar_wait(gfull, guse & 1, &never);
+    }
   }
 
   tc_fence_before();
@@ -313,11 +406,14 @@ bool readout_tc_supported(int in_dtype, int out_dtype, int D, int U) {
 }
 
 cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, void *O, long long BH,
-                              int T, int U, int chunk, int anchors, int32_t *info, cudaStream_t st) {
+                              int T, int U, int chunk, int anchors, int32_t *info, cudaStream_t st,
+                              const OutGate *og) {
   const long long nframes = BH * T;
   if (nframes <= 0) return cudaSuccess;
-  CUtensorMap tmQ, tmO;
-  if (!make_rows_map(&tmQ, Q, nframes, U, kNT) || !make_rows_map(&tmO, O, nframes, U, kNT))
+  CUtensorMap tmQ, tmO, tmG;
+  const bool gated = og && og->gate;
+  if (!make_rows_map(&tmQ, Q, nframes, U, kNT) || !make_rows_map(&tmO, O, nframes, U, kNT) ||
+      !make_rows_map(&tmG, gated ? og->gate : Q, nframes, U, kNT))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(readout_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
@@ -325,8 +421,9 @@ cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, voi
   const int sms = device_sm_count();
   const long long grid = nframes < sms ? nframes : sms;
   ReadoutArgs a{F, G, (__nv_bfloat16 *)O, info, nframes, T, U, chunk, anchors,
-                (T + chunk - 1) / chunk, (U + kNT - 1) / kNT};
-  readout_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(tmQ, tmO, a);
+                (T + chunk - 1) / chunk, (U + kNT - 1) / kNT,
+                gated ? og->w : nullptr, gated ? og->eps : 0.f, gated ? og->H : 1};
+  readout_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(tmQ, tmO, tmG, a);
   return cudaGetLastError();
 }
 

@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(kThreads) scan_simt_kernel(
 template <int D, typename Tin, typename Tout>
 __global__ void __launch_bounds__(kThreads) readout_simt_kernel(
     const Tin *__restrict__ Q, const float *__restrict__ F, const float *__restrict__ G,
-    Tout *__restrict__ O, int T, int U, int chunk, int anchors, int C) {
+    Tout *__restrict__ O, int T, int U, int chunk, int anchors, int C, OutGate og) {
   constexpr int TU = 64;
   constexpr int RB = D / 16;
   constexpr int LD = D + 1;
@@ -391,6 +391,28 @@ __global__ void __launch_bounds__(kThreads) readout_simt_kernel(
     for (int a = 0; a < 4; ++a)
 #pragma unroll
       for (int b = 0; b < RB; ++b) acc[a][b] = fmaf(q[a], rr[b], acc[a][b]);
+  }
+  if (og.gate) {
+    // RMSNorm over each token's D channels (held by the 16 lanes tx of its
+    // half-warp), then the per-channel sigmoid gate
+    const Tin *Gf = static_cast<const Tin *>(og.gate) + f * (long long)U * D;
+    const float *w = og.w + (bh % og.H) * D;
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int u = u0 + ty + 16 * a;
+      float ss = 0.f;
+#pragma unroll
+      for (int b = 0; b < RB; ++b) ss = fmaf(acc[a][b], acc[a][b], ss);
+#pragma unroll
+      for (int m = 8; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+      const float rs = 1.0f / sqrtf(ss / D + og.eps);
+#pragma unroll
+      for (int b = 0; b < RB; ++b) {
+        const int ch = tx + 16 * b;
+        const float gv = u < U ? to_f32(Gf[(long long)u * D + ch]) : 0.f;
+        acc[a][b] *= rs * w[ch] / (1.0f + expf(-gv));
+      }
+    }
   }
 #pragma unroll
   for (int a = 0; a < 4; ++a) {
@@ -443,7 +465,7 @@ cudaError_t scan_d(const float *Mf, const float *Jf, const float *Mb, const floa
 
 template <int D, typename Tin, typename Tout>
 cudaError_t readout_dt(const void *Q, const float *F, const float *G, void *O, long long BH, int T,
-                       int U, int chunk, int anchors, cudaStream_t st) {
+                       int U, int chunk, int anchors, cudaStream_t st, const OutGate &og) {
   const int C = (T + chunk - 1) / chunk;
   const size_t smem = (size_t)(D * (D + 1) + 64 * D) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(readout_simt_kernel<D, Tin, Tout>,
@@ -451,22 +473,22 @@ cudaError_t readout_dt(const void *Q, const float *F, const float *G, void *O, l
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)(BH * T), (unsigned)((U + 63) / 64));
   readout_simt_kernel<D, Tin, Tout><<<grid, kThreads, smem, st>>>(
-      (const Tin *)Q, F, G, (Tout *)O, T, U, chunk, anchors, C);
+      (const Tin *)Q, F, G, (Tout *)O, T, U, chunk, anchors, C, og);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t readout_d(const void *Q, int in_dtype, const float *F, const float *G, void *O,
                       int out_dtype, long long BH, int T, int U, int chunk, int anchors,
-                      cudaStream_t st) {
+                      cudaStream_t st, const OutGate &og) {
   if (in_dtype == VDN_BF16) {
     if (out_dtype == VDN_BF16)
-      return readout_dt<D, __nv_bfloat16, __nv_bfloat16>(Q, F, G, O, BH, T, U, chunk, anchors, st);
-    return readout_dt<D, __nv_bfloat16, float>(Q, F, G, O, BH, T, U, chunk, anchors, st);
+      return readout_dt<D, __nv_bfloat16, __nv_bfloat16>(Q, F, G, O, BH, T, U, chunk, anchors, st, og);
+    return readout_dt<D, __nv_bfloat16, float>(Q, F, G, O, BH, T, U, chunk, anchors, st, og);
   }
   if (out_dtype == VDN_BF16)
-    return readout_dt<D, float, __nv_bfloat16>(Q, F, G, O, BH, T, U, chunk, anchors, st);
-  return readout_dt<D, float, float>(Q, F, G, O, BH, T, U, chunk, anchors, st);
+    return readout_dt<D, float, __nv_bfloat16>(Q, F, G, O, BH, T, U, chunk, anchors, st, og);
+  return readout_dt<D, float, float>(Q, F, G, O, BH, T, U, chunk, anchors, st, og);
 }
 
 }  // namespace
@@ -515,9 +537,11 @@ cudaError_t launch_scan_simt(const float *Mf, const float *Jf, const float *Mb, 
 
 cudaError_t launch_readout_simt(const void *Q, int in_dtype, const float *F, const float *G, void *O,
                                 int out_dtype, long long BH, int T, int U, int chunk, int anchors,
-                                int D, cudaStream_t st) {
+                                int D, cudaStream_t st, const OutGate *og) {
   if (BH <= 0 || T <= 0 || U <= 0) return cudaSuccess;
-  VDN_DISPATCH_D(D, readout_d<DD_>(Q, in_dtype, F, G, O, out_dtype, BH, T, U, chunk, anchors, st))
+  const OutGate none{nullptr, nullptr, 0.f, 1};
+  const OutGate &g = og ? *og : none;
+  VDN_DISPATCH_D(D, readout_d<DD_>(Q, in_dtype, F, G, O, out_dtype, BH, T, U, chunk, anchors, st, g))
 }
 
 }  // namespace vdn

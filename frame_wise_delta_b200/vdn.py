@@ -54,6 +54,21 @@ def shape_for(w, B=None, H=None) -> vdn_shape:
                       w.chunk, w.anchors, w.dtype, beta_per_token=w.beta_per_token)
 
 
+class vdn_out_gate(ctypes.Structure):
+    _fields_ = [("gate", ctypes.c_void_p), ("norm_weight", ctypes.c_void_p), ("eps", ctypes.c_float)]
+
+
+def out_gate(gate, norm_weight, eps=1e-6):
+    """The readout epilogue's arguments: gate logits [B,H,T,U,dv] (input dtype),
+    RMSNorm weights [H,dv] float32, eps. Returns a vdn_out_gate (keep the
+    tensors alive while it is in use)."""
+    return vdn_out_gate(_ptr(gate), _ptr(norm_weight), float(eps))
+
+
+def _og(og):
+    return None if og is None else ctypes.cast(ctypes.pointer(og), _P)
+
+
 _lib = None
 
 _P = ctypes.c_void_p
@@ -66,10 +81,11 @@ _SIGS = {
     "vdn_scan_bidir": [_P, _P, _P, _P, _P, _P, _P, _P, _P],
     "vdn_chunk_readout": [_P, _P, _P, _P, _P, _P, _P],
     "vdn_text_state": [_P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P],
-    "vdn_forward": [_P] * 13 + [ctypes.c_size_t, _P, _P, _P],
+    "vdn_forward": [_P] * 13 + [ctypes.c_size_t, _P, _P, _P, _P],
     "vdn_frame_invert": [_P, _P, _P, _P, _P],
     "vdn_text_state_noalloc": [_P, _P, _P, _P, _P, _P, _P],
-    "vdn_forward_pipelined": [_P] * 13 + [ctypes.c_size_t, _P, ctypes.c_int32, _P, _P, _P],
+    "vdn_forward_pipelined": [_P] * 13 + [ctypes.c_size_t, _P, ctypes.c_int32, _P, _P, _P, _P],
+    "vdn_chunk_readout_gated": [_P] * 8,
 }
 
 
@@ -197,9 +213,10 @@ def vdn_forward_workspace_bytes(s) -> int:
 
 
 def vdn_forward(s, Q, K, V, beta, alpha, Kx, Vx, beta_x, O, F, G, workspace, info, events=None,
-                stream=None):
+                stream=None, og=None):
     """events: None or 7 torch.cuda.Event (enable_timing, already recorded once so
-    that their CUDA handles exist) recorded by the library between the stages."""
+    that their CUDA handles exist) recorded by the library between the stages.
+    og: None or an out_gate(...) for the gated RMSNorm readout epilogue."""
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     ev = None
     if events is not None:
@@ -210,7 +227,7 @@ def vdn_forward(s, Q, K, V, beta, alpha, Kx, Vx, beta_x, O, F, G, workspace, inf
         ev = ctypes.cast(arr, ctypes.c_void_p)
     _check(lib().vdn_forward(_shp(s), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(alpha), _ptr(Kx),
                              _ptr(Vx), _ptr(beta_x), _ptr(O), _ptr(F), _ptr(G), _ptr(workspace), nbytes,
-                             _ptr(info), ev, _stream(stream)))
+                             _ptr(info), ev, _og(og), _stream(stream)))
 
 
 def pipeline_events(groups: int):
@@ -223,7 +240,7 @@ def pipeline_events(groups: int):
 
 
 def vdn_forward_pipelined(s, Q, K, V, beta, alpha, Kx, Vx, beta_x, O, F, G, workspace, info, groups, aux,
-                          events, stream=None):
+                          events, stream=None, og=None):
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     handles = [e.cuda_event for e in events]
     if len(handles) < 7 + 3 * groups or not all(handles):
@@ -232,7 +249,12 @@ def vdn_forward_pipelined(s, Q, K, V, beta, alpha, Kx, Vx, beta_x, O, F, G, work
     _check(lib().vdn_forward_pipelined(_shp(s), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(alpha), _ptr(Kx),
                                        _ptr(Vx), _ptr(beta_x), _ptr(O), _ptr(F), _ptr(G), _ptr(workspace),
                                        nbytes, _ptr(info), int(groups), _stream(aux),
-                                       ctypes.cast(arr, ctypes.c_void_p), _stream(stream)))
+                                       ctypes.cast(arr, ctypes.c_void_p), _og(og), _stream(stream)))
+
+
+def vdn_chunk_readout_gated(s, Q, F, G, og, O, info=None, stream=None):
+    _check(lib().vdn_chunk_readout_gated(_shp(s), _ptr(Q), _ptr(F), _ptr(G), _og(og), _ptr(O), _ptr(info),
+                                         _stream(stream)))
 
 
 def vdn_status_string(status: int) -> str:
@@ -270,9 +292,9 @@ class Forward:
             self.G = torch.empty_like(self.F)
         del BH
 
-    def __call__(self, Q, K, V, beta, alpha, Kx, Vx, beta_x, events=None, stream=None):
+    def __call__(self, Q, K, V, beta, alpha, Kx, Vx, beta_x, events=None, stream=None, og=None):
         vdn_forward(self.s, Q, K, V, beta, alpha, Kx, Vx, beta_x, self.O, self.F, self.G, self.ws,
-                    self.info, events, stream)
+                    self.info, events, stream, og)
         return self.O
 
 
@@ -285,7 +307,7 @@ class PipelinedForward(Forward):
         self.aux = torch.cuda.Stream(device=device)
         self.events = pipeline_events(groups)
 
-    def __call__(self, Q, K, V, beta, alpha, Kx, Vx, beta_x, events=None, stream=None):
+    def __call__(self, Q, K, V, beta, alpha, Kx, Vx, beta_x, events=None, stream=None, og=None):
         vdn_forward_pipelined(self.s, Q, K, V, beta, alpha, Kx, Vx, beta_x, self.O, self.F, self.G, self.ws,
-                              self.info, self.groups, self.aux, self.events, stream)
+                              self.info, self.groups, self.aux, self.events, stream, og)
         return self.O

@@ -187,6 +187,29 @@ vdn_status vdn_chunk_readout(const vdn_shape *s, const void *Q, const float *F,
                              vdn_stream_t stream);
 
 /*
+ * Readout epilogue. Paper: "Method steps", step (5) ("after the readout,
+ * RMSNorm and a sigmoid gate") and "Core method" (the linear branch is gated
+ * with an RMSNorm first). Every token's readout o (d_v channels) becomes
+ *   y_i = o_i / sqrt(mean_j o_j^2 + eps) * norm_weight[h][i] * sigmoid(gate_i),
+ * and anchor rows stay 0.
+ */
+typedef struct {
+  const void *gate;         /* [B,H,T,U,dv] in_dtype: gate logits per token and channel */
+  const float *norm_weight; /* [H, dv] float32: RMSNorm weight of each head */
+  float eps;                /* > 0, finite */
+} vdn_out_gate;
+
+/*
+ * vdn_chunk_readout followed by the epilogue above, in the same kernel (the
+ * ungated O is never written). og must not be NULL; gate and norm_weight are
+ * device pointers, 16-byte aligned. Same errors as vdn_chunk_readout, plus
+ * VDN_ERR_INVALID for a bad og.
+ */
+vdn_status vdn_chunk_readout_gated(const vdn_shape *s, const void *Q, const float *F,
+                                   const float *G, const vdn_out_gate *og, void *O,
+                                   int32_t *info, vdn_stream_t stream);
+
+/*
  * Text state. Paper: "Core method" (the text prompt is summarised into a text
  * state S^T that initialises both scans). Reading: one VDA update from the
  * zero state over the n_text text tokens, with gate beta_x and no decay:
@@ -240,6 +263,8 @@ vdn_status vdn_text_state_noalloc(const vdn_shape *s, const void *Kx,
  * run on the tensor-core path (per-frame inverses W_t, then
  * X <- (X Diag(alpha_t) + B_t) W_t chains, which equal X M_t + J_t); other
  * shapes use the CUDA-core kernels of the stage calls above.
+ * og: NULL for O as read out, or the readout epilogue of
+ *      vdn_chunk_readout_gated (O then holds y).
  */
 size_t vdn_forward_workspace_bytes(const vdn_shape *s);
 vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K,
@@ -247,7 +272,8 @@ vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K,
                        const void *Kx, const void *Vx, const float *beta_x,
                        void *O, float *F, float *G, void *workspace,
                        size_t workspace_bytes, int32_t *info,
-                       const void *const *stage_events, vdn_stream_t stream);
+                       const void *const *stage_events, const vdn_out_gate *og,
+                       vdn_stream_t stream);
 
 /*
  * The fused pass of vdn_forward (bf16 inputs and output, d = 128 only) on two
@@ -273,7 +299,8 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
                                  float *F, float *G, void *workspace,
                                  size_t workspace_bytes, int32_t *info,
                                  int32_t groups, vdn_stream_t aux,
-                                 const void *const *events, vdn_stream_t stream);
+                                 const void *const *events, const vdn_out_gate *og,
+                                 vdn_stream_t stream);
 
 /* Name of a status code (static string). */
 const char *vdn_status_string(vdn_status st);

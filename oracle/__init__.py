@@ -8,6 +8,7 @@ from .vda import (  # noqa: F401
     chunk_readout,
     frame_stats,
     frame_update,
+    gated_rmsnorm,
     is_anchor,
     num_chunks,
     readout_state,

@@ -168,6 +168,18 @@ def chunk_readout(Q, F, G, chunk: int = 5, anchors: int = 0):
     return O
 
 
+def gated_rmsnorm(O, weight, gate, eps: float = 1e-6):
+    """Readout epilogue of "Method steps" step (5): RMSNorm of every token's
+    readout over its d_v channels, then a sigmoid gate, channel by channel:
+        y = o / sqrt(mean_i o_i^2 + eps) * weight * sigmoid(gate).
+    O, gate: [..., d_v]; weight: [d_v] (one RMSNorm weight vector per head).
+    """
+    O = _f64(O)
+    g = _f64(gate)
+    rms = np.sqrt(np.mean(O * O, axis=-1, keepdims=True) + eps)
+    return O / rms * _f64(weight) * (1.0 / (1.0 + np.exp(-g)))
+
+
 def chunk_maps(K, V, beta, alpha, chunk: int = 5, anchors: int = 0):
     """Affine map S -> S M_c + J_c that each chunk's frames apply, per direction.
 
@@ -204,12 +216,16 @@ def vda_head(inp: dict, chunk: int = 5, anchors: int = 0) -> dict:
     """The whole linear branch for one (batch, head) pair.
 
     inp holds Q, K, V [T, U, d], Kx, Vx [n_text, d], beta [T], alpha [T, d]
-    and beta_x. Returns S_T, F, G and O (all float64).
+    and beta_x; with gate [T, U, d] and norm_w [d] also the gated RMSNorm
+    output Y. Returns S_T, F, G, O (and Y), all float64.
     """
     S_T = text_state(inp["Kx"], inp["Vx"], inp.get("beta_x", 1.0))
     F, G = scan_states(inp["K"], inp["V"], inp["beta"], inp["alpha"], S_T, chunk, anchors)
     O = chunk_readout(inp["Q"], F, G, chunk, anchors)
-    return {"S_T": S_T, "F": F, "G": G, "O": O}
+    out = {"S_T": S_T, "F": F, "G": G, "O": O}
+    if "gate" in inp:  # gated RMSNorm epilogue (step (5))
+        out["Y"] = gated_rmsnorm(O, inp["norm_w"], inp["gate"], inp.get("eps", 1e-6))
+    return out
 
 
 def rel_frobenius(x, ref) -> float:

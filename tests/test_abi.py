@@ -90,9 +90,9 @@ def test_workspace_checks(L):
     need = vdn.vdn_forward_workspace_bytes(s)
     assert need > 0 and need % 256 == 0
     args = [_p(s)] + [16] * 9 + [16, 16, 256]  # Q..O, F, G, workspace
-    st = L.vdn_forward(*args[:13], need - 1, 16, None, None)
+    st = L.vdn_forward(*args[:13], need - 1, 16, None, None, None)
     assert st == vdn.VDN_ERR_INVALID and "workspace" in vdn.vdn_last_error()
-    st = L.vdn_forward(*args[:12], 0x1010, need, 16, None, None)
+    st = L.vdn_forward(*args[:12], 0x1010, need, 16, None, None, None)
     assert st == vdn.VDN_ERR_INVALID and "256-byte" in vdn.vdn_last_error()
     assert vdn.vdn_text_state_workspace_bytes(s) == 2 * 2 * 16 * 16 * 4
     # bf16, d = 128: the tensor path also keeps one 64 KB inverse image per (b, h)
@@ -124,16 +124,16 @@ def test_pipelined_validation(L):
     ev = (ctypes.c_void_p * 13)(*([16] * 13))
     evp = ctypes.cast(ev, ctypes.c_void_p)
     args = [_p(s)] + [16] * 11 + [256, need, 16]  # Q..O, F, G, workspace, bytes, info
-    assert L.vdn_forward_pipelined(*args, 2, None, evp, None) == vdn.VDN_ERR_UNSUPPORTED
+    assert L.vdn_forward_pipelined(*args, 2, None, evp, None, None) == vdn.VDN_ERR_UNSUPPORTED
     s2 = _shape(d=128, in_dtype="bf16")
     args[0] = _p(s2)
     args[13] = vdn.vdn_forward_workspace_bytes(s2)
-    assert L.vdn_forward_pipelined(*args, 0, None, evp, None) == vdn.VDN_ERR_INVALID
+    assert L.vdn_forward_pipelined(*args, 0, None, evp, None, None) == vdn.VDN_ERR_INVALID
     assert "groups" in vdn.vdn_last_error()
-    assert L.vdn_forward_pipelined(*args, 2, None, None, None) == vdn.VDN_ERR_INVALID
+    assert L.vdn_forward_pipelined(*args, 2, None, None, None, None) == vdn.VDN_ERR_INVALID
     assert "events" in vdn.vdn_last_error()
     ev[9] = None  # 7 + 3 * 2 = 13 events, one missing
-    assert L.vdn_forward_pipelined(*args, 2, None, evp, None) == vdn.VDN_ERR_INVALID
+    assert L.vdn_forward_pipelined(*args, 2, None, evp, None, None) == vdn.VDN_ERR_INVALID
     assert "events[9]" in vdn.vdn_last_error()
 
 
@@ -149,3 +149,17 @@ def test_beta_per_token_flag_is_checked(L):
 def vdn_synth():
     from frame_wise_delta_b200 import synth
     return synth
+
+
+def test_gated_readout_validation(L):
+    s = _shape()
+    og = vdn.vdn_out_gate(16, 16, 1e-6)
+    ogp = ctypes.cast(ctypes.pointer(og), ctypes.c_void_p)
+    assert L.vdn_chunk_readout_gated(_p(s), 16, 16, 16, None, 16, None, None) == vdn.VDN_ERR_INVALID
+    assert "og is NULL" in vdn.vdn_last_error()
+    og.eps = 0.0
+    assert L.vdn_chunk_readout_gated(_p(s), 16, 16, 16, ogp, 16, None, None) == vdn.VDN_ERR_INVALID
+    assert "eps" in vdn.vdn_last_error()
+    og.eps, og.gate = 1e-6, 0x1004
+    assert L.vdn_chunk_readout_gated(_p(s), 16, 16, 16, ogp, 16, None, None) == vdn.VDN_ERR_INVALID
+    assert "og->gate" in vdn.vdn_last_error()

@@ -397,3 +397,29 @@ def test_per_token_synthetic_gates():
         assert x.min() >= w.beta_lo and x.max() <= 1.0 and x.std() > 0.2
     # the per-frame workloads keep their gates: the stream of beta is unchanged
     assert synth.generate_head(synth.WORKLOADS["small"], 0, 2)["beta"].shape == (w.T,)
+
+
+# --- readout epilogue: RMSNorm then a sigmoid gate (step (5)) ----------------
+def test_gated_rmsnorm_is_the_library_rmsnorm_times_sigmoid():
+    import torch
+    rng = _rng(50)
+    O = rng.standard_normal((3, 7, 16))
+    w = rng.uniform(0.5, 1.5, 16)
+    g = rng.standard_normal((3, 7, 16)) * 2
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(O), (16,), torch.from_numpy(w), eps=1e-6)
+    ref = (ref * torch.sigmoid(torch.from_numpy(g))).numpy()
+    np.testing.assert_allclose(oracle.gated_rmsnorm(O, w, g, 1e-6), ref, rtol=1e-12, atol=1e-12)
+
+
+def test_gated_rmsnorm_invariants():
+    rng = _rng(51)
+    O = rng.standard_normal((5, 32)) * 3
+    w = np.ones(32)
+    # an open gate leaves unit RMS; a zero logit halves it exactly
+    y = oracle.gated_rmsnorm(O, w, np.full_like(O, 60.0), 0.0)
+    np.testing.assert_allclose(np.sqrt(np.mean(y * y, axis=-1)), 1.0, rtol=1e-12)
+    np.testing.assert_allclose(oracle.gated_rmsnorm(O, w, np.zeros_like(O), 0.0), 0.5 * y, rtol=1e-12)
+    # scale invariance (eps = 0) and a zero row (anchor) stays zero
+    np.testing.assert_allclose(oracle.gated_rmsnorm(7.5 * O, w, O, 0.0), oracle.gated_rmsnorm(O, w, O, 0.0),
+                               rtol=1e-12)
+    assert not np.any(oracle.gated_rmsnorm(np.zeros((2, 32)), w, O[:2], 1e-6))
