@@ -113,6 +113,12 @@ __device__ __forceinline__ void tma_store_3d(const void *desc, uint32_t src, int
       : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Untiled bulk copy shared -> global (16-byte aligned, size multiple of 16),
+// tracked by this thread's bulk async-groups.
+__device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+               : "memory");
+}
 // Wait until at most N of this thread's bulk groups still read shared memory.
 template <int N>
 __device__ __forceinline__ void bulk_wait_read() {

@@ -71,19 +71,6 @@ __device__ __forceinline__ void tile_row_store(uint8_t *tile, int r, const float
   }
 }
 
-// Row r, columns 64 * region .. + 63 of a global 128 x 128 hi/lo image.
-__device__ __forceinline__ void img_row_store(uint8_t *img, int region, int r, const float *v, float sign) {
-  uint8_t *base = img + region * kImgRegion + r * 128;
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    uint4 h, l;
-    pack8(v + 8 * c, sign, h, l);
-    const uint32_t o = chunk_pos(r, c);
-    *reinterpret_cast<uint4 *>(base + o) = h;
-    *reinterpret_cast<uint4 *>(base + kImgHalf + o) = l;
-  }
-}
-
 // the 12 MMAs (3 hi/lo parts x 4 k-steps) of one 64-deep product
 __device__ __forceinline__ void mma_hilo(uint32_t d, uint32_t a_hi, uint32_t a_lo, uint32_t b_hi,
                                          uint32_t b_lo, bool a_mn, bool b_mn, uint32_t a_lbo,
@@ -304,46 +291,62 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       });
       wait_mma();
       tmem_row64(acc0 + lane_off, v);  // row i of Y
-      // top-right block: -Y
-      if (img) img_row_store(img, 1, i, v, -1.f);
-      if (Wf) w_row_store(Wf, 1, i, v, -1.f);
-      // bottom-right block: row i of the S^{-1} tile; the image copies it chunk
-      // by chunk (row 64 + i of the image has the same swizzle as row i of the tile)
-      if (img) {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t o = (uint32_t)i * 128u + (uint32_t)c * 16u;
-          uint8_t *dst = img + kImgRegion + (64 + i) * 128 + c * 16;
-          *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(s0 + o);
-          *reinterpret_cast<uint4 *>(dst + kImgHalf) = *reinterpret_cast<const uint4 *>(s0 + kHalf + o);
-        }
-      }
       if (Wf) {
+        w_row_store(Wf, 1, i, v, -1.f);  // top-right block: -Y
         float u[64];
         tile_row_add(s0, i, u, false);
-        w_row_store(Wf, 1, 64 + i, u, 1.f);
+        w_row_store(Wf, 1, 64 + i, u, 1.f);  // bottom-right block: S^{-1}
       }
-      tile_row_store(s0, i, v, 1.f);  // the Y tile, A of the last product
-      tmem_row64(acc1 + lane_off, v);  // row i of Y^T
-      // bottom-left block: -Y^T
-      if (img) img_row_store(img, 0, 64 + i, v, -1.f);
-      if (Wf) w_row_store(Wf, 0, 64 + i, v, -1.f);
+      // The image is written as four 64 x 64 blocks by bulk copies of the
+      // tiles (rows 64 + i of an image region have the swizzle of rows i of a
+      // tile). Bottom-right: the S^{-1} tile as it stands.
+      if (img && i == 0) {
+        bulk_store(img + kImgRegion + 64 * 128, a_s0, kHalf);
+        bulk_store(img + kImgHalf + kImgRegion + 64 * 128, a_s0 + kHalf, kHalf);
+        bulk_commit();
+        bulk_wait_read<0>();
+      }
+      bar_named(kBarEpi);  // the S^{-1} tile has been read; it becomes -Y
+      tile_row_store(s0, i, v, -1.f);  // -Y: the top-right block and A of the last product
       fence_proxy_async_smem();
       tc_fence_before();
       bar_named(kBarEpi);
-      // Y X^T
+      // (-Y) X^T; the top-right block is copied out alongside
       issue([&] { mma_hilo(acc0, a_s0 - kHalf, a_s0, a_xt, a_xt + kHalf, false, true, 16, kIdescBmn); });
+      if (img && i == 0) {
+        bulk_store(img + kImgRegion, a_s0, kHalf);
+        bulk_store(img + kImgHalf + kImgRegion, a_s0 + kHalf, kHalf);
+        bulk_commit();
+      }
       wait_mma();
       tmem_row64(acc0 + lane_off, v);
-      // top-left block: P^{-1} + Y X^T; once every row of P^{-1} is read the
-      // sweep warps may overwrite it with the next frame's
+      // top-left block: P^{-1} - (-Y) X^T, written over this row of the P^{-1} tile
+#pragma unroll
+      for (int e = 0; e < 64; ++e) v[e] = -v[e];
       tile_row_add(pi_t, i, v, true);
-      if (f + gridDim.x < nframes) handoff_arrive(kBarPiFree);
-      if (img) img_row_store(img, 0, i, v, 1.f);
+      tile_row_store(pi_t, i, v, 1.f);
       if (Wf) w_row_store(Wf, 0, i, v, 1.f);
+      // bottom-left block: -Y^T, into the X^T tile (the last product is done)
+      tmem_row64(acc1 + lane_off, v);
+      tile_row_store(xt, i, v, -1.f);
+      if (Wf) w_row_store(Wf, 0, 64 + i, v, -1.f);
+      fence_proxy_async_smem();
+      bar_named(kBarEpi);
+      if (img && i == 0) {
+        bulk_store(img, a_pi, kHalf);
+        bulk_store(img + kImgHalf, a_pi + kHalf, kHalf);
+        bulk_store(img + 64 * 128, a_xt, kHalf);
+        bulk_store(img + kImgHalf + 64 * 128, a_xt + kHalf, kHalf);
+        bulk_commit();
+        bulk_wait_read<0>();  // the P^{-1}, X^T and -Y tiles may be reused
+      }
+      bar_named(kBarEpi);
+      // the sweep warps may now write the next frame's P^{-1} tile
+      if (f + gridDim.x < nframes) handoff_arrive(kBarPiFree);
       tc_fence_before();
     }
   }
+  if (tid == 64) bulk_wait_all();  // the image's bulk copies have landed
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
