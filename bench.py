@@ -35,8 +35,12 @@ ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # sha256 prefix of the kernel source the counters were taken on; reported as
 # None as soon as that source changes.
 NCU_TRAFFIC = {
-    "frame_factor": {"bytes": 101.3e6 + 104.8e6, "source": "frame_wise_delta_b200/csrc/invert_tc.cu",
-                     "sha256_16": "71f8ec1c98c2a934", "workload": "h3"},
+    "frame_grams": {"bytes": 1264.5e6 + 290.1e6, "source": "frame_wise_delta_b200/csrc/gram_tc.cu",
+                    "sha256_16": "6cd0f03a3878d8ed", "workload": "h3"},
+    "frame_factor": {"bytes": 100.4e6 + 99.7e6, "source": "frame_wise_delta_b200/csrc/invert_tc.cu",
+                     "sha256_16": "d9c6ae7b69b1e55e", "workload": "h3"},
+    "chunk_readout": {"bytes": 700.7e6 + 581.2e6, "source": "frame_wise_delta_b200/csrc/readout_tc.cu",
+                      "sha256_16": "245d5ff033f12626", "workload": "h3"},
 }
 
 
