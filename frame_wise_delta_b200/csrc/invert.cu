@@ -65,36 +65,6 @@ __global__ void __launch_bounds__(kSweepThreads) invert_sweep_kernel(const float
   }
 }
 
-// d = 64: one warp per frame (SweepW64).
-__global__ void __launch_bounds__(32) invert_warp64_kernel(const float *__restrict__ A, float *__restrict__ W,
-                                                           int32_t *__restrict__ info, long long frame_base) {
-  __shared__ __align__(16) float buf[2 * 128];
-  const long long f = blockIdx.x;
-  const int lane = threadIdx.x, rg = lane >> 3, cg = lane & 7;
-  const float *Af = A + f * 64LL * 64;
-  SweepW64 X;
-#pragma unroll
-  for (int a = 0; a < 16; ++a)
-#pragma unroll
-    for (int b = 0; 2 * b <= a; ++b) {
-      const int i = rg + 4 * a, j = cg + 8 * b;
-      X.at(a, b) = Af[i * 64 + j] + (i == j ? 1.f : 0.f);
-    }
-  const bool ok = X.run(buf, rg, cg);
-  if (!ok && lane == 0) report_frame_failure(info, frame_base + f);
-  if (W) {
-    float *Wf = W + f * 64LL * 64;
-#pragma unroll
-    for (int a = 0; a < 16; ++a)
-#pragma unroll
-      for (int b = 0; 2 * b <= a; ++b) {
-        const int i = rg + 4 * a, j = cg + 8 * b;
-        Wf[i * 64 + j] = -X.at(a, b);
-        if (a > 2 * b + 1) Wf[j * 64 + i] = -X.at(a, b);  // below the diagonal block
-      }
-  }
-}
-
 }  // namespace
 
 cudaError_t launch_invert_simt(const float *A, float *W, uint8_t *Wimg, int32_t *info,
@@ -104,7 +74,7 @@ cudaError_t launch_invert_simt(const float *A, float *W, uint8_t *Wimg, int32_t 
   switch (D) {
     case 16: invert_sweep_kernel<16><<<(unsigned)nframes, kSweepThreads, 0, st>>>(A, W, nullptr, info, frame_base); break;
     case 32: invert_sweep_kernel<32><<<(unsigned)nframes, kSweepThreads, 0, st>>>(A, W, nullptr, info, frame_base); break;
-    case 64: invert_warp64_kernel<<<(unsigned)nframes, 32, 0, st>>>(A, W, info, frame_base); break;
+    case 64: invert_sweep_kernel<64><<<(unsigned)nframes, kSweepThreads, 0, st>>>(A, W, nullptr, info, frame_base); break;
     case 128: invert_sweep_kernel<128><<<(unsigned)nframes, kSweepThreads, 0, st>>>(A, W, Wimg, info, frame_base); break;
     default: return cudaErrorInvalidValue;
   }

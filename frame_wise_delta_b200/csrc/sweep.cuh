@@ -190,107 +190,4 @@ struct Sweep {
   }
 };
 
-// The same sweep on a 64 x 64 matrix by ONE warp. Lane (rg = lane / 8,
-// cg = lane % 8) owns (rg + 4a, cg + 8b) for 2b <= a (block rows a < 16,
-// block columns b < 8): the lower block-triangle with whole 8 x 8 diagonal
-// blocks, 72 values per lane, held as fp32x2 pairs over b plus a single where
-// a row's count (a / 2 + 1) is odd. The pivot exchange goes through shared
-// memory with __syncwarp instead of a block barrier. Pivot k = 8 kb + kr has
-// its column on lanes cg == kr and its row on lanes rg == kr % 4 (block row
-// 2 kb + kr / 4).
-struct SweepW64 {
-  float2 XP[16][4];
-  float XS[16];
-
-  __device__ __forceinline__ float &at(int a, int b) {
-    const int n = a / 2 + 1;
-    return ((n & 1) && b == n - 1) ? XS[a] : ((b & 1) ? XP[a][b >> 1].y : XP[a][b >> 1].x);
-  }
-
-  // buf: 2 x 128 floats of shared memory private to this warp. c_x = G[x][k]
-  // is kept twice, in row order (slot (x % 4) * 16 + x / 4) for the lanes'
-  // rows and in column order (slot 64 + (x % 8) * 8 + x / 8) for their
-  // columns. Returns false if any pivot was non-positive or non-finite.
-  __device__ __forceinline__ bool run(float *buf, int rg, int cg) {
-    bool bad = false;
-#pragma unroll
-    for (int kb = 0; kb < 8; ++kb) {
-#pragma unroll 1
-      for (int kr = 0; kr < 8; ++kr) {
-        float *cr = buf + (kr & 1) * 128, *cc = cr + 64;
-        // publish column k (rows 8 kb .. 63) and row k (columns 0 .. 8 kb - 1)
-        if (cg == kr) {
-#pragma unroll
-          for (int a = 2 * kb; a < 16; ++a) {
-            const int x = rg + 4 * a;
-            const float v = at(a, kb);
-            cr[(x & 3) * 16 + (x >> 2)] = v;
-            cc[(x & 7) * 8 + (x >> 3)] = v;
-          }
-        }
-        if (rg == (kr & 3)) {
-#pragma unroll
-          for (int b = 0; b < kb; ++b) {
-            const int x = cg + 8 * b;
-            const float v = kr < 4 ? at(2 * kb, b) : at(2 * kb + 1, b);
-            cr[(x & 3) * 16 + (x >> 2)] = v;
-            cc[(x & 7) * 8 + (x >> 3)] = v;
-          }
-        }
-        __syncwarp();
-        const int k = 8 * kb + kr;
-        const float piv = cr[(k & 3) * 16 + (k >> 2)];
-        bad |= !(piv > 0.f) || !isfinite(piv);
-        const float rp = __frcp_rn(piv);
-        float ci[16];
-#pragma unroll
-        for (int a = 0; a < 16; a += 4) {
-          const float4 w = *reinterpret_cast<const float4 *>(&cr[rg * 16 + a]);
-          ci[a] = w.x;
-          ci[a + 1] = w.y;
-          ci[a + 2] = w.z;
-          ci[a + 3] = w.w;
-        }
-        float2 cj2[4];  // c_j / piv for this lane's columns, as pairs
-        {
-          const float2 rp2 = make_float2(rp, rp);
-          const float4 w0 = *reinterpret_cast<const float4 *>(&cc[cg * 8]);
-          const float4 w1 = *reinterpret_cast<const float4 *>(&cc[cg * 8 + 4]);
-          cj2[0] = __fmul2_rn(make_float2(w0.x, w0.y), rp2);
-          cj2[1] = __fmul2_rn(make_float2(w0.z, w0.w), rp2);
-          cj2[2] = __fmul2_rn(make_float2(w1.x, w1.y), rp2);
-          cj2[3] = __fmul2_rn(make_float2(w1.z, w1.w), rp2);
-        }
-#define VDN_CJW(b) (((b) & 1) ? cj2[(b) >> 1].y : cj2[(b) >> 1].x)
-#pragma unroll
-        for (int a = 0; a < 16; ++a) {
-          const int n = a / 2 + 1;
-          const float2 na = make_float2(-ci[a], -ci[a]);
-#pragma unroll
-          for (int q = 0; q < n / 2; ++q) XP[a][q] = __ffma2_rn(na, cj2[q], XP[a][q]);
-          if (n & 1) XS[a] = fmaf(-ci[a], VDN_CJW(n - 1), XS[a]);
-        }
-        // column k: G[x][k] / piv; row k: the same by symmetry, and the pivot -> -1/piv
-        if (cg == kr) {
-#pragma unroll
-          for (int a = 2 * kb; a < 16; ++a) at(a, kb) = ci[a] * rp;
-        }
-        if (rg == (kr & 3)) {
-          if (kr < 4) {
-#pragma unroll
-            for (int b = 0; b < kb; ++b) at(2 * kb, b) = VDN_CJW(b);
-            at(2 * kb, kb) = (cg == kr) ? -rp : VDN_CJW(kb);
-          } else {
-#pragma unroll
-            for (int b = 0; b < kb; ++b) at(2 * kb + 1, b) = VDN_CJW(b);
-            at(2 * kb + 1, kb) = (cg == kr) ? -rp : VDN_CJW(kb);
-          }
-        }
-#undef VDN_CJW
-      }
-    }
-    return !bad;
-  }
-};
-
 }  // namespace vdn
