@@ -290,8 +290,9 @@ def main():
     fwd_dev = make_forward()
     # our kernels per step: text (gram, invert, injection chain) + gram +
     # invert + compose (M and J chains) + scan + readout, per head group
-    launches_per_step = (6 + 2 * max(G, 1)) if tensor_path else 7
-    n_ev = 7 + 3 * G if G else 7
+    # tensor path: text (3) + Grams per group (they also sweep P) + inverse, compose, scan, readout
+    launches_per_step = (7 + max(G, 1)) if tensor_path else 7
+    n_ev = 8 + G if G else 7
 
     def step(ev=None):
         if G:
@@ -364,19 +365,13 @@ def main():
 
 
 def pipelined_stage_ms(e, G):
-    """Per-stage device time of one vdn_forward_pipelined step from its 7 + 3 G
-    events, each stage timed on its own stream and summed over head groups;
-    the text state and the inverses run on the auxiliary stream beside the
-    Grams, so these overlap and add up to more than the step."""
-    t = 3 + 3 * G
-    out = {"text_state": event_ms(e[1], e[2]), "frame_grams": 0.0, "frame_factor": 0.0,
-           "chunk_compose": event_ms(e[t], e[t + 1]), "scan_bidir": event_ms(e[t + 1], e[t + 2]),
-           "chunk_readout": event_ms(e[t + 2], e[t + 3])}
-    for g in range(G):
-        b = 3 + 3 * g
-        out["frame_grams"] += event_ms(e[0] if g == 0 else e[b - 3], e[b])
-        out["frame_factor"] += event_ms(e[b + 1], e[b + 2])
-    return out
+    """Per-stage device time of one vdn_forward_pipelined step from its 8 + G
+    events, each stage timed on its own stream. The text state runs on the
+    auxiliary stream beside the Grams."""
+    t = 3 + G
+    return {"text_state": event_ms(e[1], e[2]), "frame_grams": event_ms(e[0], e[3 + G - 1]),
+            "frame_factor": event_ms(e[t], e[t + 1]), "chunk_compose": event_ms(e[t + 1], e[t + 2]),
+            "scan_bidir": event_ms(e[t + 2], e[t + 3]), "chunk_readout": event_ms(e[t + 3], e[t + 4])}
 
 
 def e2e_measure(args, host, d, make_forward, stream, barrier, world, frames_all, dt, og=None):

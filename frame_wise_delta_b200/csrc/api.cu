@@ -121,20 +121,25 @@ size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
 
 // ----------------------------------------------------------- stage calls
+// Pimg (tensor path): also write each frame's P^{-1} tile for the block inverse
 vdn_status run_grams(const Geo &g, const void *K, const void *V, const float *beta, float *A,
-                     float *Bm, long long nframes, int U, int32_t *info, cudaStream_t st) {
+                     float *Bm, long long nframes, int U, int32_t *info, cudaStream_t st,
+                     uint8_t *Pimg = nullptr, long long frame_base = 0) {
   if (nframes <= 0) return VDN_OK;
   const size_t bytes = (size_t)nframes * g.D * g.D * sizeof(float);
   if (U == 0) {
     VDN_CUDA(cudaMemsetAsync(A, 0, bytes, st), "memset A");
     VDN_CUDA(cudaMemsetAsync(Bm, 0, bytes, st), "memset Bm");
+    if (Pimg) VDN_CUDA(launch_psweep(A, Pimg, info, nframes, st, frame_base), "P sweep");
     return VDN_OK;
   }
   if (gram_tc_supported(g.in_dtype, g.D, U)) {
-    VDN_CUDA(launch_gram_tc(K, V, beta, g.tokb != 0, A, Bm, nframes, U, info, st), "gram_tc");
+    VDN_CUDA(launch_gram_tc(K, V, beta, g.tokb != 0, A, Bm, nframes, U, info, st, Pimg, frame_base),
+             "gram_tc");
   } else {
     VDN_CUDA(launch_gram_simt(K, V, g.in_dtype, beta, g.tokb != 0, A, Bm, nframes, U, g.D, st),
              "gram_simt");
+    if (Pimg) VDN_CUDA(launch_psweep(A, Pimg, info, nframes, st, frame_base), "P sweep");
   }
   return VDN_OK;
 }
@@ -395,7 +400,7 @@ vdn_status vdn_frame_invert(const vdn_shape *s, const float *A, float *W, int32_
 
 namespace {
 struct FwdLayout {
-  size_t text, st, a, b, wimg, mf, jf, mb, jb, mimg, f, g, total;
+  size_t text, st, a, b, wimg, pimg, mf, jf, mb, jb, mimg, f, g, total;
 };
 FwdLayout fwd_layout(const Geo &g) {
   FwdLayout L{};
@@ -412,6 +417,7 @@ FwdLayout fwd_layout(const Geo &g) {
   L.a = take(g.BH * g.T * dd);
   L.b = take(g.BH * g.T * dd);
   L.wimg = take(tc ? (size_t)g.BH * g.T * kImgBytes : 0);
+  L.pimg = take(tc ? (size_t)g.BH * g.T * kPTileBytes : 0);
   L.mf = take(g.BH * g.C * dd);
   L.jf = take(g.BH * g.C * dd);
   L.mb = take(g.BH * g.C * dd);
@@ -486,11 +492,12 @@ vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K, const v
   VDN_CUDA(cudaMemsetAsync(info, 0, sizeof(int32_t), st), "memset info");
   VDN_TRY(run_text_state(g, Kx, Vx, beta_x, S_T, w + L.text, info, st));
   VDN_TRY(mark(1));
-  if (frames) VDN_TRY(run_grams(g, K, V, beta, A, Bm, g.BH * g.T, g.U, info, st));
+  uint8_t *Pimg = tc ? (uint8_t *)(w + L.pimg) : nullptr;
+  if (frames) VDN_TRY(run_grams(g, K, V, beta, A, Bm, g.BH * g.T, g.U, info, st, Pimg));
   VDN_TRY(mark(2));
   if (frames) {
     if (tc) {
-      VDN_CUDA(launch_invert_tc(A, nullptr, Wimg, info, g.BH * g.T, st), "invert");
+      VDN_CUDA(launch_invert_tc(A, nullptr, Wimg, info, g.BH * g.T, st, 0, Pimg), "invert");
     } else {
       // M and J overwrite A and Bm in place (each element is read and
       // written by the same thread).
@@ -534,7 +541,7 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
     return fail(VDN_ERR_UNSUPPORTED, "the pipelined pass needs bf16 inputs and output and d = 128");
   if (groups < 1 || groups > 64) return fail(VDN_ERR_INVALID, "groups = %d not in [1, 64]", groups);
   if (!events) return fail(VDN_ERR_INVALID, "events is NULL");
-  for (int i = 0; i < 7 + 3 * groups; ++i)
+  for (int i = 0; i < 8 + groups; ++i)
     if (!events[i]) return fail(VDN_ERR_INVALID, "events[%d] is NULL", i);
   const bool frames = g.BH * g.T > 0;
   VDN_TRY(need(Q, "Q", frames && g.U > 0));
@@ -565,6 +572,7 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
   float *S_T = (float *)(w + L.st);
   float *A = (float *)(w + L.a), *Bm = (float *)(w + L.b);
   uint8_t *Wimg = (uint8_t *)(w + L.wimg), *Mimg = (uint8_t *)(w + L.mimg);
+  uint8_t *Pimg = (uint8_t *)(w + L.pimg);
   float *Jf = (float *)(w + L.jf), *Jb = (float *)(w + L.jb);
   float *Fo = F ? F : (float *)(w + L.f);
   float *Go = G ? G : (float *)(w + L.g);
@@ -580,42 +588,37 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
   VDN_CUDA(cudaEventRecord(ev(1), ax), "event record");
   VDN_TRY(run_text_state(g, Kx, Vx, beta_x, S_T, w + L.text, info, ax));
   VDN_CUDA(cudaEventRecord(ev(2), ax), "event record");
-  // the Grams of every group on the main stream; each group's inverse on the
-  // auxiliary stream once its Grams are done, beside the next group's Grams
+  // the Grams of every group on the main stream (their kernel also writes the
+  // P^{-1} tiles of the block inverse)
   for (int gi = 0; gi < groups; ++gi) {
-    const int base = 3 + 3 * gi;
     const bool run = gi < G_ && frames;
     const long long b0 = run ? lo(gi) : 0, nbh = run ? lo(gi + 1) - b0 : 0;
     if (run)
-      VDN_TRY(run_grams(g, tok(K, b0), tok(V, b0), beta + b0 * T * (g.tokb ? U : 1), A + b0 * T * DD, Bm + b0 * T * DD, nbh * T,
-                        (int)U, info, st));
-    VDN_CUDA(cudaEventRecord(ev(base + 0), st), "event record");
-    VDN_CUDA(cudaStreamWaitEvent(ax, ev(base + 0), 0), "stream wait");
-    VDN_CUDA(cudaEventRecord(ev(base + 1), ax), "event record");
-    if (run)
-      VDN_CUDA(launch_invert_tc(A + b0 * T * DD, nullptr, Wimg + b0 * T * kImgBytes, info, nbh * T, ax,
-                                b0 * T),
-               "invert");
-    VDN_CUDA(cudaEventRecord(ev(base + 2), ax), "event record");
+      VDN_TRY(run_grams(g, tok(K, b0), tok(V, b0), beta + b0 * T * (g.tokb ? U : 1), A + b0 * T * DD,
+                        Bm + b0 * T * DD, nbh * T, (int)U, info, st, Pimg + b0 * T * kPTileBytes, b0 * T));
+    VDN_CUDA(cudaEventRecord(ev(3 + gi), st), "event record");
   }
-  // composition, scans and readout over all pairs once the auxiliary stream
-  // (text state and every inverse) is done: these are latency-bound chains
-  // whose time grows if they are split
-  const int tail = 3 + 3 * groups;
-  VDN_CUDA(cudaStreamWaitEvent(st, ev(tail - 1), 0), "stream wait");
+  // the rest of the inverse, the composition, the scans and the readout over
+  // all pairs once the auxiliary stream (text state and every P sweep) is
+  // done: these are latency-bound chains whose time grows if they are split
+  const int tail = 3 + groups;
+  VDN_CUDA(cudaStreamWaitEvent(st, ev(2), 0), "stream wait");
   VDN_CUDA(cudaEventRecord(ev(tail), st), "event record");
+  if (frames)
+    VDN_CUDA(launch_invert_tc(A, nullptr, Wimg, info, g.BH * g.T, st, 0, Pimg), "invert");
+  VDN_CUDA(cudaEventRecord(ev(tail + 1), st), "event record");
   if (frames)
     VDN_CUDA(launch_compose_tc(Wimg, Bm, alpha, nullptr, Jf, nullptr, Jb, Mimg, g.BH, g.T, g.chunk, g.anchors,
                                2, info, st),
              "compose");
-  VDN_CUDA(cudaEventRecord(ev(tail + 1), st), "event record");
+  VDN_CUDA(cudaEventRecord(ev(tail + 2), st), "event record");
   if (frames)
     VDN_CUDA(launch_scan_tc(Mimg, Jf, Jb, S_T, Fo, Go, g.BH, g.C, info, st), "scan");
   else if (g.BH > 0)
     VDN_CUDA(launch_scan_simt(nullptr, nullptr, nullptr, nullptr, S_T, Fo, Go, g.BH, g.C, g.D, 3, st), "scan");
-  VDN_CUDA(cudaEventRecord(ev(tail + 2), st), "event record");
-  if (frames) VDN_TRY(run_readout(g, Q, Fo, Go, O, info, st, gate));
   VDN_CUDA(cudaEventRecord(ev(tail + 3), st), "event record");
+  if (frames) VDN_TRY(run_readout(g, Q, Fo, Go, O, info, st, gate));
+  VDN_CUDA(cudaEventRecord(ev(tail + 4), st), "event record");
   return VDN_OK;
 }
 

@@ -21,13 +21,19 @@
 //   warp 0     : TMA producer (4 loads of 8 KB per 64-token stage)
 //   warp 1     : TMEM allocator and single-thread MMA issuer
 //   warps 2..5 : epilogue: TMEM -> registers -> fp32 stores
-//   warps 6..9 : (per-token gates) the scaled K tile of each stage
+//   warps 6..9 : (per-token gates) the scaled K tile of each stage, or
+//                (PSW) two pairs of sweep warps: each takes every other frame's
+//                leading 64 x 64 block of I + A_t, which the epilogue stages in
+//                shared memory, and writes its inverse P^{-1} as the hi/lo tile
+//                the block inverse reads (so the CUDA-core sweeps run beside the
+//                HBM-bound stream instead of after it)
 // TMEM holds two 256-column accumulators so a frame's epilogue overlaps the
 // next frame's MMAs. Every wait is bounded (see common.cuh).
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
 #include "internal.h"
+#include "sweep.cuh"
 
 namespace vdn {
 namespace {
@@ -37,14 +43,20 @@ constexpr int kUT = 64;                          // tokens per pipeline stage
 constexpr int kStagesMax = 4;
 constexpr int kBlockBytes = kUT * 128;           // one 64-channel block
 constexpr uint32_t kTmemCols = 512;
-constexpr int kBarBytes = 8 * (3 * kStagesMax + 2 + 2 + 1);
+constexpr int kBarBytes = 8 * (3 * kStagesMax + 2 + 2 + 1 + 4);
+// PSW: per sweep pair an fp32 staging of P (64 rows of 65 floats: no bank
+// conflicts for the sweep's loads), a hi/lo tile for the bulk store, and the
+// pair's exchange vector
+constexpr int kPStage = 64 * 65 * 4;
+constexpr int kPTile = 16384;
+constexpr int kPSmem = 2 * (kPStage + kPTile + 2 * 64 * 4);
 // per stage: the K and V blocks of channels 0..63 and 64..127 (+ the scaled
 // K blocks: hi part of both, then lo part of both)
 template <bool TOKB> constexpr int kStagesT = TOKB ? 3 : 4;
 template <bool TOKB> constexpr int kStageBytesT = (TOKB ? 8 : 4) * kBlockBytes;
 template <bool TOKB> constexpr int kThreadsT = TOKB ? 320 : 192;
-template <bool TOKB>
-constexpr size_t kSmemBytesT = 1024 + (size_t)kStagesT<TOKB> * kStageBytesT<TOKB> + kBarBytes + 16;
+template <bool TOKB, bool PSW>
+constexpr size_t kSmemBytesT = 1024 + (size_t)kStagesT<TOKB> * kStageBytesT<TOKB> + (PSW ? kPSmem : 0) + kBarBytes + 16;
 
 struct GramArgs {
   float *A;
@@ -54,6 +66,8 @@ struct GramArgs {
   long long nframes;
   int ntiles;
   int U;
+  uint8_t *Pimg;          // PSW: [nframes] P^{-1} tiles
+  long long frame_base;   // PSW: frame index of frame 0 for *info
 };
 
 __device__ __forceinline__ void fail(volatile int *abort, int32_t *info) {
@@ -61,18 +75,23 @@ __device__ __forceinline__ void fail(volatile int *abort, int32_t *info) {
   if (info) atomicExch(info, VDN_INFO_TIMEOUT);
 }
 
-template <bool TOKB>
-__global__ void __launch_bounds__(kThreadsT<TOKB>, 1)
+template <bool TOKB, bool PSW>
+__global__ void __launch_bounds__((TOKB || PSW) ? 320 : 192, 1)
     gram_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    GramArgs p) {
+  static_assert(!(TOKB && PSW), "one use of warps 6..9");
   constexpr int kStageBytes = kStageBytesT<TOKB>;
   constexpr int kStages = kStagesT<TOKB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
   uint8_t *stages = smem;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kStages * kStageBytes + kBarBytes);
+  uint8_t *pmem = smem + kStages * kStageBytes;  // PSW area
+  float *pstage = reinterpret_cast<float *>(pmem);                        // [2][64][65]
+  uint8_t *ptile = pmem + 2 * kPStage;                                    // [2][16 KB]
+  float *pcbuf = reinterpret_cast<float *>(pmem + 2 * kPStage + 2 * kPTile);  // [2][2][64]
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes + (PSW ? kPSmem : 0));
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(bars) + kBarBytes);
   volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -82,6 +101,8 @@ __global__ void __launch_bounds__(kThreadsT<TOKB>, 1)
   const uint32_t tempty0 = tfull0 + 16;
   const uint32_t drain = tempty0 + 16;
   const uint32_t scaled0 = drain + 8;  // per stage: the scaled K tile is written
+  const uint32_t pready0 = scaled0 + 8 * kStagesMax;  // PSW, per pair: P staged (128 arrivals)
+  const uint32_t pfree0 = pready0 + 16;               // PSW, per pair: staging read (64 arrivals)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -95,6 +116,11 @@ __global__ void __launch_bounds__(kThreadsT<TOKB>, 1)
     mbar_init(drain, 1);
     if (TOKB)
       for (int s = 0; s < kStages; ++s) mbar_init(scaled0 + 8 * s, 128);
+    if (PSW)
+      for (int q = 0; q < 2; ++q) {
+        mbar_init(pready0 + 8 * q, 128);
+        mbar_init(pfree0 + 8 * q, 64);
+      }
     *abort = 0;
     fence_barrier_init();
   }
@@ -234,6 +260,42 @@ __global__ void __launch_bounds__(kThreadsT<TOKB>, 1)
         }
       }
     }
+  } else if (PSW && warp >= 6) {
+    // a sweep pair (warps 6-7 or 8-9): every other frame of this CTA
+    const int pq = (warp - 6) >> 1;
+    const int st = threadIdx.x - 192 - 64 * pq;  // 0..63
+    const int rg = st / kSweepGrid, cg = st % kSweepGrid;
+    const int nb = 3 + pq;  // the pair's named barrier
+    const float *ps = pstage + pq * (64 * 65);
+    uint8_t *pt = ptile + pq * kPTile;
+    float(*cb)[64] = reinterpret_cast<float(*)[64]>(pcbuf + pq * 128);
+    bool okw = true;
+    int it = 0;
+    for (long long f = blockIdx.x; f < p.nframes; f += gridDim.x, ++it) {
+      if ((it & 1) != pq) continue;
+      if (okw && !mbar_wait(pready0 + 8 * pq, (uint32_t)(it >> 1) & 1, abort)) {
+        fail(abort, p.info);
+        okw = false;
+      }
+      Sweep<64> X;
+#pragma unroll
+      for (int a = 0; a < Sweep<64>::R; ++a)
+#pragma unroll
+        for (int b = 0; b <= a; ++b) X.at(a, b) = ps[(rg + kSweepGrid * a) * 65 + cg + kSweepGrid * b];
+      mbar_arrive(pfree0 + 8 * pq);  // the staging may take the pair's next frame
+      const bool ok = X.run(cb, rg, cg, [nb] { asm volatile("bar.sync %0, 64;" ::"r"(nb) : "memory"); });
+      if (st == 0) bulk_wait_read<0>();  // the previous P^{-1} tile has left
+      asm volatile("bar.sync %0, 64;" ::"r"(nb) : "memory");
+      store_swept_tile(X, pt, rg, cg);
+      fence_proxy_async_smem();
+      asm volatile("bar.sync %0, 64;" ::"r"(nb) : "memory");
+      if (st == 0) {
+        bulk_store(p.Pimg + f * (long long)kPTile, smem_u32(pt), kPTile);
+        bulk_commit();
+        if (!ok) report_frame_failure(p.info, p.frame_base + f);
+      }
+    }
+    if (st == 0) bulk_wait_all();
   } else {
     // epilogue warps 2..5 -> TMEM sub-partitions 2, 3, 0, 1
     const int sub = warp & 3;
@@ -242,6 +304,12 @@ __global__ void __launch_bounds__(kThreadsT<TOKB>, 1)
     for (long long f = blockIdx.x; f < p.nframes; f += gridDim.x, ++it) {
       const int buf = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
+      const int pq = it & 1;  // PSW: the sweep pair of this frame
+      float *ps = pstage + pq * (64 * 65);
+      if (PSW && row < 64 && use > 0) {
+        // the pair has read its staging of two frames ago
+        if (!mbar_wait(pfree0 + 8 * pq, (use - 1) & 1, abort)) fail(abort, p.info);
+      }
       // every lane waits (acquire); the warp then agrees on the outcome so
       // that it enters the aligned TMEM loads together or not at all
       const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull0 + 8 * buf, use & 1, abort));
@@ -263,9 +331,15 @@ __global__ void __launch_bounds__(kThreadsT<TOKB>, 1)
         float *dst = (cc < 4 ? Af + (cc * 32) * kD : Bf + ((cc - 4) * 32) * kD) + row;
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) dst[jj * kD] = bt * v[jj];
+        if (PSW && cc < 2 && row < 64) {
+          // P = I + A[0..63][0..63] for the sweep pair (A symmetric: row `row`)
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) ps[row * 65 + cc * 32 + jj] = bt * v[jj] + (row == cc * 32 + jj ? 1.f : 0.f);
+        }
       }
       tc_fence_before();
       mbar_arrive(tempty0 + 8 * buf);
+      if (PSW) mbar_arrive(pready0 + 8 * pq);
     }
   }
 
@@ -296,25 +370,34 @@ bool make_rows_map(CUtensorMap *m, const void *base, long long frames, int rows,
   return r == CUDA_SUCCESS;
 }
 
-template <bool TOKB>
+template <bool TOKB, bool PSW>
 cudaError_t launch_gram_t(const CUtensorMap &tmK, const CUtensorMap &tmV, const GramArgs &a, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(gram_tc_kernel<TOKB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBytesT<TOKB>);
+  constexpr size_t smem = kSmemBytesT<TOKB, PSW>;
+  cudaError_t e = cudaFuncSetAttribute(gram_tc_kernel<TOKB, PSW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
   if (e != cudaSuccess) return e;
   const int sms = device_sm_count();
   const long long grid = a.nframes < sms ? a.nframes : sms;
-  gram_tc_kernel<TOKB><<<(unsigned)grid, kThreadsT<TOKB>, kSmemBytesT<TOKB>, st>>>(tmK, tmV, a);
+  gram_tc_kernel<TOKB, PSW><<<(unsigned)grid, (TOKB || PSW) ? 320 : 192, smem, st>>>(tmK, tmV, a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gram_tc(const void *K, const void *V, const float *beta, bool per_token, float *A,
-                           float *Bm, long long nframes, int U, int32_t *info, cudaStream_t st) {
+                           float *Bm, long long nframes, int U, int32_t *info, cudaStream_t st, uint8_t *Pimg,
+                           long long frame_base) {
   if (nframes <= 0) return cudaSuccess;
   CUtensorMap tmK, tmV;
   if (!make_rows_map(&tmK, K, nframes, U, kUT) || !make_rows_map(&tmV, V, nframes, U, kUT))
     return cudaErrorInvalidValue;
-  GramArgs a{A, Bm, beta, info, nframes, (U + kUT - 1) / kUT, U};
-  return per_token ? launch_gram_t<true>(tmK, tmV, a, st) : launch_gram_t<false>(tmK, tmV, a, st);
+  GramArgs a{A, Bm, beta, info, nframes, (U + kUT - 1) / kUT, U, Pimg, frame_base};
+  if (per_token) {
+    // the per-token stages use warps 6..9 and most of shared memory: the
+    // P^{-1} tiles then come from their own kernel
+    cudaError_t e = launch_gram_t<true, false>(tmK, tmV, a, st);
+    if (e != cudaSuccess || !Pimg) return e;
+    return launch_psweep(A, Pimg, info, nframes, st, frame_base);
+  }
+  return Pimg ? launch_gram_t<false, true>(tmK, tmV, a, st) : launch_gram_t<false, false>(tmK, tmV, a, st);
 }
 
 }  // namespace vdn

@@ -35,8 +35,11 @@ cudaError_t launch_readout_simt(const void *Q, int in_dtype, const float *F, con
 
 // Tensor-core kernels (tcgen05 + TMA), bf16 inputs, d = 128.
 bool gram_tc_supported(int in_dtype, int D, int U);
+// Pimg: null, or where to write each frame's P^{-1} tile (the leading 64 x 64
+// block of I + A inverted, as launch_psweep does), swept beside the stream
 cudaError_t launch_gram_tc(const void *K, const void *V, const float *beta, bool per_token, float *A,
-                           float *Bm, long long nframes, int U, int32_t *info, cudaStream_t st);
+                           float *Bm, long long nframes, int U, int32_t *info, cudaStream_t st,
+                           uint8_t *Pimg = nullptr, long long frame_base = 0);
 bool readout_tc_supported(int in_dtype, int out_dtype, int D, int U);
 cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, void *O, long long BH,
                               int T, int U, int chunk, int anchors, int32_t *info, cudaStream_t st,
@@ -47,8 +50,13 @@ cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, voi
 // frame_base: index of the first frame, for the failure index in *info.
 // (I + A)^{-1} of fp32 128 x 128 frames by the tensor-core block inverse, as
 // fp32 row-major W and/or hi/lo MMA images (either may be null)
+// Pimg: null, or the P^{-1} tiles of launch_psweep (then the kernel skips its P sweeps)
 cudaError_t launch_invert_tc(const float *A, float *W, uint8_t *Wimg, int32_t *info, long long nframes,
-                             cudaStream_t st, long long frame_base = 0);
+                             cudaStream_t st, long long frame_base = 0, const uint8_t *Pimg = nullptr);
+// P^{-1} (leading 64 x 64 block of I + A) of every frame as a 16 KB hi/lo tile
+constexpr long long kPTileBytes = 16384;
+cudaError_t launch_psweep(const float *A, uint8_t *Pimg, int32_t *info, long long nframes, cudaStream_t st,
+                          long long frame_base = 0);
 cudaError_t launch_invert_simt(const float *A, float *W, uint8_t *Wimg, int32_t *info,
                                long long nframes, int D, cudaStream_t st, long long frame_base = 0);
 // Chunk maps from W images (tensor cores, d = 128): per (direction, b*h,

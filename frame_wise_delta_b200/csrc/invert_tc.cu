@@ -142,27 +142,42 @@ __device__ __forceinline__ void fail(volatile int *abort, int32_t *info) {
   if (info) atomicExch(info, VDN_INFO_TIMEOUT);
 }
 
-// -G^{-1} of a 64 x 64 block from the sweep -> hi/lo tile of G^{-1} (both triangles)
-__device__ __forceinline__ void store_swept(Sweep<64> &X, uint8_t *tile, int rg, int cg) {
+// P^{-1} of every frame as a hi/lo tile in global memory (16 KB per frame,
+// the layout of the kernel below's P^{-1} slot), by the same sweep: lets the
+// block inverse skip its own P sweeps.
+__global__ void __launch_bounds__(kSweepThreads) psweep_kernel(const float *__restrict__ A, uint8_t *__restrict__ Pimg,
+                                                               int32_t *__restrict__ info, long long frame_base) {
+  __shared__ __align__(1024) uint8_t tile[kTile];
+  __shared__ __align__(16) float cbuf[2][64];
+  const long long f = blockIdx.x;
+  const int tid = threadIdx.x, rg = tid / kSweepGrid, cg = tid % kSweepGrid;
+  const float *Af = A + f * 128LL * 128;
+  Sweep<64> X;
 #pragma unroll
   for (int a = 0; a < Sweep<64>::R; ++a)
 #pragma unroll
     for (int b = 0; b <= a; ++b) {
-      const int i = rg + kSweepGrid * a, j = cg + kSweepGrid * b;
-      __nv_bfloat16 h, l;
-      split_bf16(-X.at(a, b), h, l);
-      *reinterpret_cast<__nv_bfloat16 *>(tile + tile_off(i, j)) = h;
-      *reinterpret_cast<__nv_bfloat16 *>(tile + kHalf + tile_off(i, j)) = l;
-      if (a != b) {
-        *reinterpret_cast<__nv_bfloat16 *>(tile + tile_off(j, i)) = h;
-        *reinterpret_cast<__nv_bfloat16 *>(tile + kHalf + tile_off(j, i)) = l;
-      }
+      const int r = rg + kSweepGrid * a, c = cg + kSweepGrid * b;
+      X.at(a, b) = __ldg(Af + r * 128 + c) + (r == c ? 1.f : 0.f);
     }
+  const bool ok = X.run(cbuf, rg, cg, [] { __syncthreads(); });
+  store_swept_tile(X, tile, rg, cg);
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (tid == 0) {
+    bulk_store(Pimg + f * (long long)kTile, smem_u32(tile), kTile);
+    bulk_commit();
+    bulk_wait_all();
+    if (!ok) report_frame_failure(info, frame_base + f);
+  }
 }
 
+// PRE_P: the P^{-1} tiles come from psweep_kernel (Pimg) instead of the sweep warps.
+template <bool PRE_P>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     invert_tc_kernel(const float *__restrict__ A, float *__restrict__ W, uint8_t *__restrict__ Wimg,
-                     int32_t *__restrict__ info, long long nframes, long long frame_base) {
+                     int32_t *__restrict__ info, long long nframes, long long frame_base,
+                     const uint8_t *__restrict__ Pimg) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *pi_t = sm + kSlotPi, *s0 = sm + kSlotS0, *xt = sm + kSlotXT;
@@ -170,10 +185,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kSlotMisc + 512);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kSlotMisc + 520);
   volatile int *abort = reinterpret_cast<volatile int *>(sm + kSlotMisc + 524);
+  const uint32_t pbar = smem_u32(sm + kSlotMisc + 528);  // (PRE_P) the P^{-1} tile has landed
   const int tid = threadIdx.x, warp = tid >> 5;
   const uint32_t mbar = smem_u32(bar);
   if (tid == 0) {
     mbar_init(mbar, 1);
+    mbar_init(pbar, 1);
     *abort = 0;
     fence_barrier_init();
   }
@@ -197,19 +214,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     for (long long f = blockIdx.x; f < nframes; f += gridDim.x) {
       const float *Af = A + f * 128LL * 128;
       Sweep<64> X;
+      bool ok = true;
+      if constexpr (!PRE_P) {
 #pragma unroll
-      for (int a = 0; a < Sweep<64>::R; ++a)
+        for (int a = 0; a < Sweep<64>::R; ++a)
 #pragma unroll
-        for (int b = 0; b <= a; ++b) {
-          const int r = rg + kSweepGrid * a, c = cg + kSweepGrid * b;
-          X.at(a, b) = __ldg(Af + r * 128 + c) + (r == c ? 1.f : 0.f);
-        }
-      bool ok = X.run(cbuf, rg, cg, [] { bar_named(kBarSweep); });
-      if (!first) handoff_wait(kBarPiFree);  // the previous frame's last product has read P^{-1}
-      first = false;
-      store_swept(X, pi_t, rg, cg);
-      fence_proxy_async_smem();
-      handoff_arrive(kBarPiReady);
+          for (int b = 0; b <= a; ++b) {
+            const int r = rg + kSweepGrid * a, c = cg + kSweepGrid * b;
+            X.at(a, b) = __ldg(Af + r * 128 + c) + (r == c ? 1.f : 0.f);
+          }
+        ok = X.run(cbuf, rg, cg, [] { bar_named(kBarSweep); });
+        if (!first) handoff_wait(kBarPiFree);  // the previous frame's last product has read P^{-1}
+        first = false;
+        store_swept_tile(X, pi_t, rg, cg);
+        fence_proxy_async_smem();
+        handoff_arrive(kBarPiReady);
+      }
       handoff_wait(kBarTReady);
       // S = R - Q^T X and S^{-1} by the sweep; S^{-1} replaces the staging
       // (every thread has read its part before the sweep's first barrier)
@@ -222,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                        stage[r * 64 + (((c >> 2) ^ (r & 15)) << 2) + (c & 3)];
         }
       ok = X.run(cbuf, rg, cg, [] { bar_named(kBarSweep); }) && ok;
-      store_swept(X, s0, rg, cg);
+      store_swept_tile(X, s0, rg, cg);
       fence_proxy_async_smem();
       handoff_arrive(kBarSiReady);
       if (!ok && tid == 0) report_frame_failure(info, frame_base + f);
@@ -244,10 +264,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         tc_commit(mbar);
       }
     };
+    uint32_t puse = 0;
     for (long long f = blockIdx.x; f < nframes; f += gridDim.x) {
       const float *Af = A + f * 128LL * 128;
       uint8_t *img = Wimg ? Wimg + f * (long long)kImgBytes : nullptr;
       float *Wf = W ? W + f * 128LL * 128 : nullptr;
+      if (PRE_P && i == 0) {
+        // the P^{-1} slot is free (the last frame's output copies have read it)
+        mbar_arrive_expect_tx(pbar, kTile);
+        bulk_load(a_pi, Pimg + f * (long long)kTile, kTile, pbar);
+      }
       // Q^T = G[64 + r][0 .. 63] as a hi/lo tile, read row-contiguously
 #pragma unroll 4
       for (int it = 0; it < 16; ++it) {
@@ -261,7 +287,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         *reinterpret_cast<uint2 *>(s0 + kHalf + o) = l;
       }
       fence_proxy_async_smem();
-      handoff_wait(kBarPiReady);
+      if constexpr (PRE_P) {
+        if (!mbar_wait(pbar, puse & 1, abort)) fail(abort, info);
+        ++puse;
+        bar_named(kBarEpi);  // every epilogue thread's Q^T rows are written
+      } else {
+        handoff_wait(kBarPiReady);
+      }
       // X^T = Q^T P^{-1}
       issue([&] { mma_hilo(acc0, a_s0 - kHalf, a_s0, a_pi, a_pi + kHalf, false, false, 16, kIdesc); });
       float v[64];
@@ -342,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       }
       bar_named(kBarEpi);
       // the sweep warps may now write the next frame's P^{-1} tile
-      if (f + gridDim.x < nframes) handoff_arrive(kBarPiFree);
+      if (!PRE_P && f + gridDim.x < nframes) handoff_arrive(kBarPiFree);
       tc_fence_before();
     }
   }
@@ -357,14 +389,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 }  // namespace
 
 cudaError_t launch_invert_tc(const float *A, float *W, uint8_t *Wimg, int32_t *info, long long nframes,
-                             cudaStream_t st, long long frame_base) {
+                             cudaStream_t st, long long frame_base, const uint8_t *Pimg) {
   if (nframes <= 0) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(invert_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBytes);
+  auto kern = Pimg ? invert_tc_kernel<true> : invert_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   const long long cap = (long long)kCtasPerSm * device_sm_count();
   const long long grid = nframes < cap ? nframes : cap;
-  invert_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(A, W, Wimg, info, nframes, frame_base);
+  kern<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(A, W, Wimg, info, nframes, frame_base, Pimg);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_psweep(const float *A, uint8_t *Pimg, int32_t *info, long long nframes, cudaStream_t st,
+                          long long frame_base) {
+  if (nframes <= 0) return cudaSuccess;
+  psweep_kernel<<<(unsigned)nframes, kSweepThreads, 0, st>>>(A, Pimg, info, frame_base);
   return cudaGetLastError();
 }
 

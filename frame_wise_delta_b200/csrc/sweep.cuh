@@ -190,4 +190,26 @@ struct Sweep {
   }
 };
 
+// -G^{-1} of a 64 x 64 block from the sweep, stored as the hi/lo tile of
+// G^{-1} (both triangles; 64 rows of 128 bytes per part, K-major with the
+// 128-byte swizzle, hi part then lo part 8 KB later) that the tensor cores read.
+__device__ __forceinline__ void store_swept_tile(Sweep<64> &X, uint8_t *tile, int rg, int cg) {
+  constexpr int kPart = 64 * 128;
+#pragma unroll
+  for (int a = 0; a < Sweep<64>::R; ++a)
+#pragma unroll
+    for (int b = 0; b <= a; ++b) {
+      const int i = rg + kSweepGrid * a, j = cg + kSweepGrid * b;
+      __nv_bfloat16 h, l;
+      split_bf16(-X.at(a, b), h, l);
+      const uint32_t oij = kmajor_sw128_offset(i, j, 64), oji = kmajor_sw128_offset(j, i, 64);
+      *reinterpret_cast<__nv_bfloat16 *>(tile + oij) = h;
+      *reinterpret_cast<__nv_bfloat16 *>(tile + kPart + oij) = l;
+      if (a != b) {
+        *reinterpret_cast<__nv_bfloat16 *>(tile + oji) = h;
+        *reinterpret_cast<__nv_bfloat16 *>(tile + kPart + oji) = l;
+      }
+    }
+}
+
 }  // namespace vdn

@@ -231,9 +231,9 @@ def vdn_forward(s, Q, K, V, beta, alpha, Kx, Vx, beta_x, O, F, G, workspace, inf
 
 
 def pipeline_events(groups: int):
-    """The 7 + 3 * groups timing events vdn_forward_pipelined records (created
+    """The 8 + groups timing events vdn_forward_pipelined records (created
     here by torch and recorded once so that their CUDA handles exist)."""
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(7 + 3 * groups)]
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(8 + groups)]
     for e in evs:
         e.record()
     return evs
@@ -243,8 +243,8 @@ def vdn_forward_pipelined(s, Q, K, V, beta, alpha, Kx, Vx, beta_x, O, F, G, work
                           events, stream=None, og=None):
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     handles = [e.cuda_event for e in events]
-    if len(handles) < 7 + 3 * groups or not all(handles):
-        raise VdnError(VDN_ERR_INVALID, "need 7 + 3 * groups recorded events")
+    if len(handles) < 8 + groups or not all(handles):
+        raise VdnError(VDN_ERR_INVALID, "need 8 + groups recorded events")
     arr = (ctypes.c_void_p * len(handles))(*handles)
     _check(lib().vdn_forward_pipelined(_shp(s), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(alpha), _ptr(Kx),
                                        _ptr(Vx), _ptr(beta_x), _ptr(O), _ptr(F), _ptr(G), _ptr(workspace),

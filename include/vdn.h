@@ -276,20 +276,19 @@ vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K,
                        vdn_stream_t stream);
 
 /*
- * The fused pass of vdn_forward (bf16 inputs and output, d = 128 only) on two
- * streams: the B*H pairs are split into `groups` contiguous head groups, and
- * while `stream` computes one group's Grams, `aux` inverts the previous
- * group's frames (the inverse runs on the CUDA cores, the Grams on the tensor
- * cores and HBM); the text state also runs on `aux`. Composition, scans and
- * readout then run once over all pairs on `stream`. Same inputs, outputs,
- * workspace and *info as vdn_forward (a failing frame is reported by its index
- * over all B*H*T frames). The library records and waits on the caller's events
- * and creates or allocates nothing.
- * events: 7 + 3 * groups cudaEvent_t, none NULL: [0] start (stream);
- *   [1] / [2] before / after the text state (aux); per group g at 3 + 3g:
- *   +0 after its Grams (stream), +1 / +2 before / after its inverse (aux);
- *   at 3 + 3 * groups: +0 after `stream` waited for `aux`, +1 / +2 / +3 after
- *   the composition, scans and readout (stream).
+ * The fused pass of vdn_forward (bf16 inputs and output, d = 128 only) with
+ * the text state on a second stream, `aux`, beside the frame Grams on
+ * `stream`; the Grams may be split into `groups` launches over contiguous
+ * head groups. The block inverse, the composition, the scans and the readout
+ * then run over all pairs on `stream`. Same inputs, outputs, workspace and
+ * *info as vdn_forward, bit for bit (a failing frame is reported by its
+ * index over all B*H*T frames). The library records and waits on the
+ * caller's events and creates or allocates nothing.
+ * events: 8 + groups cudaEvent_t, none NULL: [0] start (stream); [1] / [2]
+ *   before / after the text state (aux); [3 + g] after the Grams of group g
+ *   (stream); at 3 + groups: +0 after `stream` waited for `aux`, +1 / +2 /
+ *   +3 / +4 after the block inverse, the composition, the scans and the
+ *   readout.
  *   On return `stream` has waited for all work on `aux`.
  */
 vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *K,

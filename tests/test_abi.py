@@ -121,7 +121,7 @@ def test_binding_refuses_host_tensors(L):
 def test_pipelined_validation(L):
     s = _shape()  # float32, d = 16: not the tensor path
     need = vdn.vdn_forward_workspace_bytes(s)
-    ev = (ctypes.c_void_p * 13)(*([16] * 13))
+    ev = (ctypes.c_void_p * 10)(*([16] * 10))
     evp = ctypes.cast(ev, ctypes.c_void_p)
     args = [_p(s)] + [16] * 11 + [256, need, 16]  # Q..O, F, G, workspace, bytes, info
     assert L.vdn_forward_pipelined(*args, 2, None, evp, None, None) == vdn.VDN_ERR_UNSUPPORTED
@@ -132,7 +132,7 @@ def test_pipelined_validation(L):
     assert "groups" in vdn.vdn_last_error()
     assert L.vdn_forward_pipelined(*args, 2, None, None, None, None) == vdn.VDN_ERR_INVALID
     assert "events" in vdn.vdn_last_error()
-    ev[9] = None  # 7 + 3 * 2 = 13 events, one missing
+    ev[9] = None  # 8 + 2 = 10 events, one missing
     assert L.vdn_forward_pipelined(*args, 2, None, evp, None, None) == vdn.VDN_ERR_INVALID
     assert "events[9]" in vdn.vdn_last_error()
 
