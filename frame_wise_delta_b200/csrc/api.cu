@@ -124,7 +124,7 @@ size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 // Pimg (tensor path): also write each frame's P^{-1} tile for the block inverse
 vdn_status run_grams(const Geo &g, const void *K, const void *V, const float *beta, float *A,
                      float *Bm, long long nframes, int U, int32_t *info, cudaStream_t st,
-                     uint8_t *Pimg = nullptr, long long frame_base = 0) {
+                     uint8_t *Pimg = nullptr, long long frame_base = 0, int spare_sms = 0) {
   if (nframes <= 0) return VDN_OK;
   const size_t bytes = (size_t)nframes * g.D * g.D * sizeof(float);
   if (U == 0) {
@@ -134,7 +134,7 @@ vdn_status run_grams(const Geo &g, const void *K, const void *V, const float *be
     return VDN_OK;
   }
   if (gram_tc_supported(g.in_dtype, g.D, U)) {
-    VDN_CUDA(launch_gram_tc(K, V, beta, g.tokb != 0, A, Bm, nframes, U, info, st, Pimg, frame_base),
+    VDN_CUDA(launch_gram_tc(K, V, beta, g.tokb != 0, A, Bm, nframes, U, info, st, Pimg, frame_base, spare_sms),
              "gram_tc");
   } else {
     VDN_CUDA(launch_gram_simt(K, V, g.in_dtype, beta, g.tokb != 0, A, Bm, nframes, U, g.D, st),
@@ -589,13 +589,15 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
   VDN_TRY(run_text_state(g, Kx, Vx, beta_x, S_T, w + L.text, info, ax));
   VDN_CUDA(cudaEventRecord(ev(2), ax), "event record");
   // the Grams of every group on the main stream (their kernel also writes the
-  // P^{-1} tiles of the block inverse)
+  // P^{-1} tiles of the block inverse). Their persistent grid leaves some SMs
+  // to the text state: its kernels need TMEM, which a Gram CTA takes whole.
+  const int spare = g.n_text > 0 ? (int)(g.BH < device_sm_count() / 6 ? g.BH : device_sm_count() / 6) : 0;
   for (int gi = 0; gi < groups; ++gi) {
     const bool run = gi < G_ && frames;
     const long long b0 = run ? lo(gi) : 0, nbh = run ? lo(gi + 1) - b0 : 0;
     if (run)
       VDN_TRY(run_grams(g, tok(K, b0), tok(V, b0), beta + b0 * T * (g.tokb ? U : 1), A + b0 * T * DD,
-                        Bm + b0 * T * DD, nbh * T, (int)U, info, st, Pimg + b0 * T * kPTileBytes, b0 * T));
+                        Bm + b0 * T * DD, nbh * T, (int)U, info, st, Pimg + b0 * T * kPTileBytes, b0 * T, spare));
     VDN_CUDA(cudaEventRecord(ev(3 + gi), st), "event record");
   }
   // the rest of the inverse, the composition, the scans and the readout over

@@ -26,7 +26,8 @@
 //                leading 64 x 64 block of I + A_t, which the epilogue stages in
 //                shared memory, and writes its inverse P^{-1} as the hi/lo tile
 //                the block inverse reads (so the CUDA-core sweeps run beside the
-//                HBM-bound stream instead of after it)
+//                HBM-bound stream instead of after it); A_t is then written
+//                from row 64 on only, the rows the block inverse reads
 // TMEM holds two 256-column accumulators so a frame's epilogue overlaps the
 // next frame's MMAs. Every wait is bounded (see common.cuh).
 #include <cudaTypedefs.h>
@@ -329,8 +330,12 @@ __global__ void __launch_bounds__((TOKB || PSW) ? 320 : 192, 1)
         // column so that a warp stores 32 consecutive floats); n >= 128 ->
         // B[n-128][row].
         float *dst = (cc < 4 ? Af + (cc * 32) * kD : Bf + ((cc - 4) * 32) * kD) + row;
+        // PSW: rows 0..63 of A (P and Q^T's transpose) are not read after
+        // this kernel (P is swept here, the block inverse reads rows 64..127)
+        if (!(PSW && cc < 2)) {
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) dst[jj * kD] = bt * v[jj];
+          for (int jj = 0; jj < 32; ++jj) dst[jj * kD] = bt * v[jj];
+        }
         if (PSW && cc < 2 && row < 64) {
           // P = I + A[0..63][0..63] for the sweep pair (A symmetric: row `row`)
 #pragma unroll
@@ -371,12 +376,14 @@ bool make_rows_map(CUtensorMap *m, const void *base, long long frames, int rows,
 }
 
 template <bool TOKB, bool PSW>
-cudaError_t launch_gram_t(const CUtensorMap &tmK, const CUtensorMap &tmV, const GramArgs &a, cudaStream_t st) {
+cudaError_t launch_gram_t(const CUtensorMap &tmK, const CUtensorMap &tmV, const GramArgs &a, cudaStream_t st,
+                          int spare_sms) {
   constexpr size_t smem = kSmemBytesT<TOKB, PSW>;
   cudaError_t e = cudaFuncSetAttribute(gram_tc_kernel<TOKB, PSW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  const int sms = device_sm_count();
+  int sms = device_sm_count() - spare_sms;
+  if (sms < 1) sms = 1;
   const long long grid = a.nframes < sms ? a.nframes : sms;
   gram_tc_kernel<TOKB, PSW><<<(unsigned)grid, (TOKB || PSW) ? 320 : 192, smem, st>>>(tmK, tmV, a);
   return cudaGetLastError();
@@ -384,7 +391,7 @@ cudaError_t launch_gram_t(const CUtensorMap &tmK, const CUtensorMap &tmV, const 
 
 cudaError_t launch_gram_tc(const void *K, const void *V, const float *beta, bool per_token, float *A,
                            float *Bm, long long nframes, int U, int32_t *info, cudaStream_t st, uint8_t *Pimg,
-                           long long frame_base) {
+                           long long frame_base, int spare_sms) {
   if (nframes <= 0) return cudaSuccess;
   CUtensorMap tmK, tmV;
   if (!make_rows_map(&tmK, K, nframes, U, kUT) || !make_rows_map(&tmV, V, nframes, U, kUT))
@@ -393,11 +400,12 @@ cudaError_t launch_gram_tc(const void *K, const void *V, const float *beta, bool
   if (per_token) {
     // the per-token stages use warps 6..9 and most of shared memory: the
     // P^{-1} tiles then come from their own kernel
-    cudaError_t e = launch_gram_t<true, false>(tmK, tmV, a, st);
+    cudaError_t e = launch_gram_t<true, false>(tmK, tmV, a, st, spare_sms);
     if (e != cudaSuccess || !Pimg) return e;
     return launch_psweep(A, Pimg, info, nframes, st, frame_base);
   }
-  return Pimg ? launch_gram_t<false, true>(tmK, tmV, a, st) : launch_gram_t<false, false>(tmK, tmV, a, st);
+  return Pimg ? launch_gram_t<false, true>(tmK, tmV, a, st, spare_sms)
+              : launch_gram_t<false, false>(tmK, tmV, a, st, spare_sms);
 }
 
 }  // namespace vdn

@@ -36,10 +36,12 @@ cudaError_t launch_readout_simt(const void *Q, int in_dtype, const float *F, con
 // Tensor-core kernels (tcgen05 + TMA), bf16 inputs, d = 128.
 bool gram_tc_supported(int in_dtype, int D, int U);
 // Pimg: null, or where to write each frame's P^{-1} tile (the leading 64 x 64
-// block of I + A inverted, as launch_psweep does), swept beside the stream
+// block of I + A inverted, as launch_psweep does), swept beside the stream;
+// then only rows 64..127 of A are written (all the block inverse reads).
+// spare_sms: SMs the persistent grid leaves free for a concurrent stream.
 cudaError_t launch_gram_tc(const void *K, const void *V, const float *beta, bool per_token, float *A,
                            float *Bm, long long nframes, int U, int32_t *info, cudaStream_t st,
-                           uint8_t *Pimg = nullptr, long long frame_base = 0);
+                           uint8_t *Pimg = nullptr, long long frame_base = 0, int spare_sms = 0);
 bool readout_tc_supported(int in_dtype, int out_dtype, int D, int U);
 cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, void *O, long long BH,
                               int T, int U, int chunk, int anchors, int32_t *info, cudaStream_t st,
