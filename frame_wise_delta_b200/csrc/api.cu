@@ -591,7 +591,7 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
   // the Grams of every group on the main stream (their kernel also writes the
   // P^{-1} tiles of the block inverse). Their persistent grid leaves some SMs
   // to the text state: its kernels need TMEM, which a Gram CTA takes whole.
-  const int spare = g.n_text > 0 ? (int)(g.BH < device_sm_count() / 6 ? g.BH : device_sm_count() / 6) : 0;
+  const int spare = g.n_text > 0 ? (int)(g.BH < device_sm_count() / 12 ? g.BH : device_sm_count() / 12) : 0;
   for (int gi = 0; gi < groups; ++gi) {
     const bool run = gi < G_ && frames;
     const long long b0 = run ? lo(gi) : 0, nbh = run ? lo(gi + 1) - b0 : 0;
