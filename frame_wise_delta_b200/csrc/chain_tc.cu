@@ -16,8 +16,9 @@
 //  M_t = Diag(alpha_t) W_t and J_t = B_t W_t, so the per-frame (M_t, J_t) are
 //  never materialised. The M and J rows are independent groups of N = 128.
 //
-//  scan, one CTA per (b*h, direction): X <- X Mc_c + Jc_c over the chunks,
-//  from X = S_T / 2, writing every boundary state (N = 128).
+//  scan, one CTA per (b*h, direction, half of the state rows): X <- X Mc_c +
+//  Jc_c over the chunks, from X = S_T / 2, writing every boundary state; the
+//  rows of X are independent, so each CTA carries 64 of them (N = 64).
 //
 // One product: D[m][n] = sum_k Op[k][m] E[n][k], i.e. D = (E Op)^T in TMEM
 // (lane m = state column, TMEM column n = state row). Op arrives as a
@@ -100,7 +101,7 @@ __device__ __forceinline__ void write_img32(uint8_t *img, int rr, int x0, const 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) chain_tc_kernel(ChainArgs p) {
   // N: state rows per product; the E image has N/64 regions of kImgRegion bytes
-  constexpr int N = MODE == kCompose ? 256 : 128;
+  constexpr int N = MODE == kCompose ? 256 : 64;
   constexpr uint32_t kEHalf = N * kD * 2;  // bytes of one bf16 part of E
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -125,11 +126,12 @@ __global__ void __launch_bounds__(kThreads, 1) chain_tc_kernel(ChainArgs p) {
 
   // ---- the chain this CTA walks
   long long bh;
-  int dir, c_cmp = 0, nsteps = 0;
+  int dir, c_cmp = 0, nsteps = 0, hz = 0;
   int frames[16];
   if (MODE == kScan) {
     bh = blockIdx.x;
     dir = blockIdx.y;
+    hz = blockIdx.z;  // state rows 64 hz .. 64 hz + 63
     nsteps = p.C;
   } else {
     dir = blockIdx.x;
@@ -167,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_tc_kernel(ChainArgs p) {
 
   if (warp == 8) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, true, true);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, MODE == kCompose ? 128 : 64, true, true);
       const uint32_t e_hi = smem_u32(eimg), e_lo = e_hi + kEHalf;
       auto load = [&](int s) {
         const int b = s % kBufs;
@@ -231,12 +233,12 @@ __global__ void __launch_bounds__(kThreads, 1) chain_tc_kernel(ChainArgs p) {
   } else {
     // ---- epilogue: thread owns state column m (TMEM lane m) for column half h
     const int m = (warp & 3) * 32 + lane;
-    const int h = warp >> 2;                     // scan: rows 64h..64h+63; compose: group (0 M, 1 J)
+    const int h = warp >> 2;                     // scan: rows 64hz+32h..+31; compose: group (0 M, 1 J)
     const int grp = MODE == kCompose ? h : 0;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    constexpr int kRows = MODE == kCompose ? 128 : 64;  // state rows handled per thread
-    const int row0 = MODE == kCompose ? 0 : 64 * h;     // first state row of this thread
-    const int tcol0 = MODE == kCompose ? 128 * h : 64 * h;  // first TMEM column / E image row index
+    constexpr int kRows = MODE == kCompose ? 128 : 32;  // state rows handled per thread
+    const int row0 = MODE == kCompose ? 0 : 64 * hz + 32 * h;  // first state row of this thread
+    const int tcol0 = MODE == kCompose ? 128 * h : 32 * h;     // first TMEM column / E image column
 
     // ---- E_0 (and, for the scan, the first boundary state)
     if (MODE == kScan) {
@@ -253,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_tc_kernel(ChainArgs p) {
           v[e] = x0[32 * j + e];
           o[(row0 + 32 * j + e) * kD] = v[e];
         }
-        if (nsteps > 0) write_img32(eimg, m, row0 + 32 * j, v, kImgRegion, kEHalf);
+        if (nsteps > 0) write_img32(eimg, m, tcol0 + 32 * j, v, kImgRegion, kEHalf);
       }
     } else {
       const long long cidx = bh * p.C + c_cmp;
@@ -327,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1) chain_tc_kernel(ChainArgs p) {
           for (int e = 0; e < 32; ++e) v[e] += addv[32 * j + e];
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[(n0 + e) * kD] = v[e];
-          if (!last) write_img32(eimg, m, n0, v, kImgRegion, kEHalf);
+          if (!last) write_img32(eimg, m, tcol0 + 32 * j, v, kImgRegion, kEHalf);
         } else if (!last) {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
@@ -410,7 +412,7 @@ cudaError_t launch_scan_tc(const uint8_t *Mimg, const float *Jf, const float *Jb
   a.G = G;
   a.info = info;
   a.C = C;
-  return launch_mode<kScan>(dim3((unsigned)BH, 2, 1), a, st);
+  return launch_mode<kScan>(dim3((unsigned)BH, 2, 2), a, st);
 }
 
 }  // namespace vdn
