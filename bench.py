@@ -35,10 +35,10 @@ ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # sha256 prefix of the kernel source the counters were taken on; reported as
 # None as soon as that source changes.
 NCU_TRAFFIC = {
-    "frame_grams": {"bytes": 1264.5e6 + 290.1e6, "source": "frame_wise_delta_b200/csrc/gram_tc.cu",
-                    "sha256_16": "6cd0f03a3878d8ed", "workload": "h3"},
-    "frame_factor": {"bytes": 100.4e6 + 99.7e6, "source": "frame_wise_delta_b200/csrc/invert_tc.cu",
-                     "sha256_16": "d9c6ae7b69b1e55e", "workload": "h3"},
+    "frame_grams": {"bytes": 1292.5e6 + 253.9e6, "source": "frame_wise_delta_b200/csrc/gram_tc.cu",
+                    "sha256_16": "00240b7db02fd61b", "workload": "h3"},
+    "frame_factor": {"bytes": 110.4e6 + 101.8e6, "source": "frame_wise_delta_b200/csrc/invert_tc.cu",
+                     "sha256_16": "3547c44be31a9b49", "workload": "h3"},
     "chunk_readout": {"bytes": 700.7e6 + 581.2e6, "source": "frame_wise_delta_b200/csrc/readout_tc.cu",
                       "sha256_16": "245d5ff033f12626", "workload": "h3"},
 }
@@ -428,6 +428,8 @@ def alg_bytes(w, gated=False):
 def roofline(w, stage_ms, hbm_gbs, peak_src, bf16_tflops=1607.7):
     """Roofline of the dominant stage. Per-unit algorithmic figures:
     frame_grams: per frame reads K, V (2 U d bf16) and writes A, B (2 d^2 fp32);
+      on the tensor path only rows 64.. of A (d^2/2 fp32) plus the 16 KB P^{-1}
+      tile its sweep warps produce;
     chunk_readout: per frame reads Q, writes O (2 U d bf16) plus two states per chunk;
     frame_factor: on the tensor path the CUDA cores sweep two 64 x 64 blocks per
       non-anchor frame (d^3 / 4 flop; the block products run on the tensor
@@ -445,7 +447,9 @@ def roofline(w, stage_ms, hbm_gbs, peak_src, bf16_tflops=1607.7):
         fr = [t for t in range(5 * c, min(5 * c + 5, T)) if not (w.anchors and t in (0, T - 1))]
         steps += len(fr) if tensor_path else max(0, len(range(5 * c, min(5 * c + 5, T))) - 1)
     units = {
-        "frame_grams": ("hbm", frames * (2 * U * d * e + 2 * d * d * 4 + (U * 4 if w.beta_per_token else 0))),
+        "frame_grams": ("hbm", frames * (2 * U * d * e + (d * d * 4 // 2 + d * d * 4 + 16384 if tensor_path
+                                                          else 2 * d * d * 4)
+                                         + (U * 4 if w.beta_per_token else 0))),
         "chunk_readout": ("hbm", frames * 2 * U * d * e + BH * C * 2 * d * d * 4),
         "frame_factor": ("alu", live * (d ** 3 // 4 if tensor_path else 4 * d ** 3)),
         "chunk_compose": ("tensor" if tensor_path else "alu", BH * 2 * steps * 4 * d ** 3),
