@@ -206,7 +206,7 @@ vdn_status run_text_state(const Geo &g, const void *Kx, const void *Vx, const fl
     uint8_t *Wimg = (uint8_t *)(ws + L.wimg);
     VDN_CUDA(launch_invert_tc(Ax, nullptr, Wimg, info, g.BH, st), "text invert");
     VDN_CUDA(launch_compose_tc(Wimg, Bx, Ax, nullptr, S_T, nullptr, nullptr, nullptr, g.BH, 1, 1, 0,
-                               /*ndirs=*/1, info, st),
+                               /*ndirs=*/1, /*j_transposed=*/false, info, st),
              "text injection");
   } else {
     VDN_CUDA(launch_factor_simt(Ax, Bx, nullptr, nullptr, S_T, info, g.BH, 1, 0, g.D, st),
@@ -510,7 +510,7 @@ vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K, const v
     if (tc) {
       // the fp32 Mc are not needed here: the scan reads their images
       VDN_CUDA(launch_compose_tc(Wimg, Bm, alpha, nullptr, Jf, nullptr, Jb, Mimg, g.BH, g.T, g.chunk,
-                                 g.anchors, 2, info, st),
+                                 g.anchors, 2, true, info, st),
                "compose");
     } else {
       VDN_CUDA(launch_compose_simt(A, Bm, Mf, Jf, Mb, Jb, g.BH, g.T, g.chunk, g.D, st), "compose");
@@ -611,7 +611,7 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
   VDN_CUDA(cudaEventRecord(ev(tail + 1), st), "event record");
   if (frames)
     VDN_CUDA(launch_compose_tc(Wimg, Bm, alpha, nullptr, Jf, nullptr, Jb, Mimg, g.BH, g.T, g.chunk, g.anchors,
-                               2, info, st),
+                               2, true, info, st),
              "compose");
   VDN_CUDA(cudaEventRecord(ev(tail + 2), st), "event record");
   if (frames)

@@ -62,13 +62,16 @@ cudaError_t launch_psweep(const float *A, uint8_t *Pimg, int32_t *info, long lon
 cudaError_t launch_invert_simt(const float *A, float *W, uint8_t *Wimg, int32_t *info,
                                long long nframes, int D, cudaStream_t st, long long frame_base = 0);
 // Chunk maps from W images (tensor cores, d = 128): per (direction, b*h,
-// chunk) the M-chain (Mf/Mb, and their images if Mimg) and the J-chain
-// (Jf/Jb); any output pointer may be NULL. ndirs = 1 runs the forward
-// direction only.
+// chunk) the M-chain (Mf/Mb fp32, and if Mimg its transposed image: the
+// K-major A operand of the scan) and the J-chain (Jf/Jb, row-major, or
+// transposed with j_transposed, as the scan reads it); any output pointer may
+// be NULL. ndirs = 1 runs the forward direction only.
 cudaError_t launch_compose_tc(const uint8_t *Wimg, const float *Bm, const float *alpha, float *Mf,
                               float *Jf, float *Mb, float *Jb, uint8_t *Mimg, long long BH, int T,
-                              int chunk, int anchors, int ndirs, int32_t *info, cudaStream_t st);
-// Both scans from Mc images and fp32 Jc (tensor cores, d = 128).
+                              int chunk, int anchors, int ndirs, bool j_transposed, int32_t *info,
+                              cudaStream_t st);
+// Both scans from the compose's Mc images and transposed fp32 Jc (tensor
+// cores, d = 128).
 cudaError_t launch_scan_tc(const uint8_t *Mimg, const float *Jf, const float *Jb, const float *S_T,
                            float *F, float *G, long long BH, int C, int32_t *info, cudaStream_t st);
 
