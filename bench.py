@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--impl", choices=["vdn", "reference"], default="vdn")
     ap.add_argument("--workload", default="h3")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (small profiling cases)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the tokens per frame (profiling the chain stages at full head count)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -228,9 +230,11 @@ def main():
     from frame_wise_delta_b200 import synth
 
     w = synth.WORKLOADS[args.workload]
+    import dataclasses
     if args.heads:
-        import dataclasses
         w = dataclasses.replace(w, H=args.heads, name=f"{w.name}_h{args.heads}")
+    if args.tokens:
+        w = dataclasses.replace(w, U=args.tokens, name=f"{w.name}_u{args.tokens}")
     if args.impl == "reference":
         return run_reference(args, w)
 

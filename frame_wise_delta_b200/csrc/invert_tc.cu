@@ -39,7 +39,7 @@ constexpr int kSlotPi = 0;              // P^{-1} image
 constexpr int kSlotS0 = kTile;          // Q^T image -> fp32 Q^T X staging -> S^{-1} image -> Y image
 constexpr int kSlotXT = 2 * kTile;      // X^T image
 constexpr int kSlotMisc = 3 * kTile;    // sweep exchange buffer, barrier, TMEM address, abort flag
-constexpr size_t kSmemBytes = 1024 + kSlotMisc + 2 * 64 * 4 + 64;
+constexpr size_t kSmemBytes = 1024 + kSlotMisc + 2 * 2 * 64 * 4 + 64;
 constexpr uint32_t kTmemCols = 128;     // two 64-column accumulators
 constexpr uint32_t kIdesc = idesc_bf16_f32(128, 64, false, false);    // A, B K-major
 constexpr uint32_t kIdescAmn = idesc_bf16_f32(128, 64, true, false);  // A MN-major
@@ -181,11 +181,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *pi_t = sm + kSlotPi, *s0 = sm + kSlotS0, *xt = sm + kSlotXT;
-  float(*cbuf)[64] = reinterpret_cast<float(*)[64]>(sm + kSlotMisc);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kSlotMisc + 512);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kSlotMisc + 520);
-  volatile int *abort = reinterpret_cast<volatile int *>(sm + kSlotMisc + 524);
-  const uint32_t pbar = smem_u32(sm + kSlotMisc + 528);  // (PRE_P) the P^{-1} tile has landed
+  float(*cbuf)[64] = reinterpret_cast<float(*)[64]>(sm + kSlotMisc);         // single-pivot sweeps
+  float(*cbuf2)[2][64] = reinterpret_cast<float(*)[2][64]>(sm + kSlotMisc);  // pivot-pair sweeps
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kSlotMisc + 1024);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kSlotMisc + 1032);
+  volatile int *abort = reinterpret_cast<volatile int *>(sm + kSlotMisc + 1036);
+  const uint32_t pbar = smem_u32(sm + kSlotMisc + 1040);  // (PRE_P) the P^{-1} tile has landed
   const int tid = threadIdx.x, warp = tid >> 5;
   const uint32_t mbar = smem_u32(bar);
   if (tid == 0) {
@@ -241,7 +242,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           X.at(a, b) = __ldg(Af + (64 + r) * 128 + 64 + c) + (r == c ? 1.f : 0.f) -
                        stage[r * 64 + (((c >> 2) ^ (r & 15)) << 2) + (c & 3)];
         }
-      ok = X.run(cbuf, rg, cg, [] { bar_named(kBarSweep); }) && ok;
+      if constexpr (PRE_P)
+        ok = X.run2(cbuf2, rg, cg, [] { bar_named(kBarSweep); }) && ok;
+      else
+        ok = X.run(cbuf, rg, cg, [] { bar_named(kBarSweep); }) && ok;
       store_swept_tile(X, s0, rg, cg);
       fence_proxy_async_smem();
       handoff_arrive(kBarSiReady);
@@ -274,8 +278,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         mbar_arrive_expect_tx(pbar, kTile);
         bulk_load(a_pi, Pimg + f * (long long)kTile, kTile, pbar);
       }
-      // Q^T = G[64 + r][0 .. 63] as a hi/lo tile, read row-contiguously
-#pragma unroll 4
+      // Q^T = G[64 + r][0 .. 63] as a hi/lo tile, read row-contiguously (all
+      // loads in flight at once)
+#pragma unroll
       for (int it = 0; it < 16; ++it) {
         const int r = it * 4 + (i >> 4), c4 = i & 15;
         const float4 x = __ldg(reinterpret_cast<const float4 *>(Af + (64 + r) * 128 + 4 * c4));
@@ -313,6 +318,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
       tc_fence_before();
       handoff_arrive(kBarTReady);
+      // while the S sweep runs: the next frame's rows 64..127 of A (Q^T and
+      // R) into L2, so its Q^T tile and S assembly read them from there
+      if (i == 0 && f + gridDim.x < nframes) {
+        bulk_prefetch_l2(Af + gridDim.x * 128LL * 128 + 64 * 128, 64 * 128 * 4);
+        if (PRE_P) bulk_prefetch_l2(Pimg + (f + gridDim.x) * (long long)kTile, kTile);
+      }
       handoff_wait(kBarSiReady);
       issue([&] {
         // Y = X S^{-1}: A = X, the X^T tile read MN-major as the second 64-row
