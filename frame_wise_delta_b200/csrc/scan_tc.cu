@@ -242,14 +242,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       mbar_arrive(jfree0 + 8 * b);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) o[(row0 + e) * kD] = v[e];
+      // the next operand first (the next product waits for it), then the
+      // boundary state, whose stores drain under that product
       if (!last) {
         write_img32(eimg, m, tcol0, v, kEHalf);
         tc_fence_before();
         fence_proxy_async_smem();
         mbar_arrive(ready);
       }
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[(row0 + e) * kD] = v[e];
     }
   }
 
