@@ -37,8 +37,8 @@ ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 NCU_TRAFFIC = {
     "frame_grams": {"bytes": 1292.5e6 + 253.9e6, "source": "frame_wise_delta_b200/csrc/gram_tc.cu",
                     "sha256_16": "00240b7db02fd61b", "workload": "h3"},
-    "frame_factor": {"bytes": 110.4e6 + 101.8e6, "source": "frame_wise_delta_b200/csrc/invert_tc.cu",
-                     "sha256_16": "3547c44be31a9b49", "workload": "h3"},
+    "frame_factor": {"bytes": 126.7e6 + 102.4e6, "source": "frame_wise_delta_b200/csrc/invert_tc.cu",
+                     "sha256_16": "85a8941c4be055cf", "workload": "h3"},
     "chunk_readout": {"bytes": 700.7e6 + 581.2e6, "source": "frame_wise_delta_b200/csrc/readout_tc.cu",
                       "sha256_16": "245d5ff033f12626", "workload": "h3"},
 }
