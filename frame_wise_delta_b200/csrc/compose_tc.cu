@@ -24,11 +24,12 @@
 // chain overlap the last products of the current one.
 //
 // Roles (320 threads):
-//   warps 0..3  M-group epilogue, warps 4..7 J-group epilogue: each thread owns
-//               one state row (TMEM lane), reads its accumulator row with
-//               tcgen05.ld and writes the next operand row with tcgen05.st.
-//               The groups have their own accumulators and barriers, so one
-//               group's epilogue overlaps the other group's MMAs;
+//   warps 0..7  epilogue: warp w owns one state row per thread (TMEM lanes
+//               32(w % 4) ..) and the column half w / 4 of both groups; it
+//               reads accumulator rows with tcgen05.ld and writes the next
+//               operand rows with tcgen05.st. The groups have their own
+//               accumulators and barriers, so one group's operand update (on
+//               all eight warps) overlaps the other group's MMAs;
 //   warp 8      allocates TMEM; one lane issues the MMAs;
 //   warp 9      one lane issues the loads: W images into two buffers (bulk
 //               copies), B_t by TMA in two column halves with the 128-byte
@@ -139,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(wfree + 8 * i, 1);
       mbar_init(bfull + 8 * i, 1);
       mbar_init(bfree + 8 * i, 128);
-      mbar_init(ready + 8 * i, 128);
+      mbar_init(ready + 8 * i, 256);
       mbar_init(done + 8 * i, 1);
       mbar_init(afull + 8 * i, 1);
       mbar_init(afree + 8 * i, 256);
@@ -256,50 +257,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int g = warp >> 2;              // 0: M rows, 1: J rows
+    // Every epilogue warp serves both groups: warp w owns TMEM lanes
+    // 32(w % 4) .. + 31 (state rows n) and the column half ch = w / 4 of each
+    // accumulator and operand, so a group's operand update runs on all eight
+    // warps while the other group's product runs.
+    const int ch = warp >> 2;              // columns 64 ch .. 64 ch + 63
     const int n = (warp & 3) * 32 + lane;  // state row (TMEM lane)
     const uint32_t lanes = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tD = tmem + lanes + kColD + 128 * g;
-    const uint32_t tEh = tmem + lanes + kColE + 128 * g, tEl = tEh + 64;
     const uint8_t *bbuf = smem + kOffB;
+    auto tD = [&](int g) { return tmem + lanes + kColD + 128 * g + 64 * ch; };
+    auto tEh = [&](int g) { return tmem + lanes + kColE + 128 * g + 32 * ch; };
     auto alpha_slot = [&](long long i) {
-      return reinterpret_cast<const float *>(smem + kOffAl + (i & 1) * kAlphaBytes);
+      return reinterpret_cast<const float *>(smem + kOffAl + (i & 1) * kAlphaBytes) + 64 * ch;
     };
-    // alpha (and B for the J group) of step i are in shared memory
-    auto wait_inputs = [&](long long i) {
-      bool w = mbar_wait(afull + 8 * (i & 1), (uint32_t)((i >> 1) & 1), abort);
-      if (g == 1) w = w && mbar_wait(bfull, (uint32_t)(i & 1), abort) && mbar_wait(bfull + 8, (uint32_t)(i & 1), abort);
-      return __all_sync(0xffffffffu, w);
+    auto wait_alpha = [&](long long i) {
+      return __all_sync(0xffffffffu, mbar_wait(afull + 8 * (i & 1), (uint32_t)((i >> 1) & 1), abort));
     };
-    // Operand of step i from v = columns 32j.. of row n; B_t is released by
-    // halves as soon as this thread has read it
-    auto put_operand = [&](int j, const float (&v)[32]) {
+    auto wait_b = [&](long long i) {  // this warp's column half of B_t
+      return __all_sync(0xffffffffu, mbar_wait(bfull + 8 * ch, (uint32_t)(i & 1), abort));
+    };
+    // Operand chunk j (of this half) of group g, row n
+    auto put_operand = [&](int g, int j, const float (&v)[32]) {
       uint32_t hi[16], lo[16];
       pack_row32(v, hi, lo);
-      tmem_st16(tEh + 16 * j, hi);
-      tmem_st16(tEl + 16 * j, lo);
-      if (g == 1 && (j & 1)) mbar_arrive(bfree + 8 * (j >> 1));
+      tmem_st16(tEh(g) + 16 * j, hi);
+      tmem_st16(tEh(g) + 64 + 16 * j, lo);
     };
-    auto publish = [&]() {
+    auto publish = [&](int g) {
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(ready + 8 * g);
     };
-
-    // Columns 32j .. 32j + 31 of row n of the chain's result. Transposed
+    // Columns 64 ch + 32 j .. + 31 of row n of a chain's result. Transposed
     // outputs (the image of Mc, Jc with jt) put the 32 threads of a warp on
     // consecutive addresses for each column m, so those stores coalesce.
-    const bool jtr = p.jt && g == 1;
-    auto write_out = [&](int j, const float (&v)[32], float *oF, uint8_t *oI) {
+    auto write_out = [&](int g, int j, const float (&v)[32], float *oF, uint8_t *oI) {
+      const int m0 = 64 * ch + 32 * j;
       if (oF) {
-        if (jtr) {
+        if (p.jt && g == 1) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) oF[(32 * j + e) * kD] = v[e];
+          for (int e = 0; e < 32; ++e) oF[(m0 + e) * kD] = v[e];
         } else {
 #pragma unroll
           for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<float4 *>(oF + 32 * j + 4 * c) =
-                make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            *reinterpret_cast<float4 *>(oF + m0 + 4 * c) = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
         }
       }
       if (oI) {
@@ -307,101 +308,130 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 32; ++e) {
           __nv_bfloat16 h, l;
           split_bf16(v[e], h, l);
-          const uint32_t off = mn_off(32 * j + e, n);  // row m, column n
+          const uint32_t off = mn_off(m0 + e, n);  // row m, column n
           *reinterpret_cast<__nv_bfloat16 *>(oI + off) = h;
           *reinterpret_cast<__nv_bfloat16 *>(oI + kImgHalf + off) = l;
         }
       }
     };
 
+    // First-step operands of a chain starting at step i: E_M = Diag(alpha),
+    // E_J = B (each published as soon as it is written)
+    auto first_m = [&](long long i) {
+      if (!wait_alpha(i)) return false;
+      const float a_n = reinterpret_cast<const float *>(smem + kOffAl + (i & 1) * kAlphaBytes)[n];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float v[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = (64 * ch + 32 * j + e == n) ? a_n : 0.f;
+        put_operand(0, j, v);
+      }
+      mbar_arrive(afree + 8 * (i & 1));
+      publish(0);
+      return true;
+    };
+    auto first_j = [&](long long i) {
+      if (!wait_b(i)) return false;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float v[32];
+        load_b_row32(bbuf, 2 * ch + j, n, v);
+        put_operand(1, j, v);
+      }
+      mbar_arrive(bfree + 8 * ch);
+      publish(1);
+      return true;
+    };
+
     long long gs = 0;
     bool ok = true;
     for (long long q = blockIdx.x; ok && q < p.nchains; q += gridDim.x) {
-      const Chain ch = decode(p, q);
-      const long long cidx = ch.bh * p.C + ch.c;
-      float *outF = g == 0 ? (ch.dir == 0 ? p.Mf : p.Mb) : (ch.dir == 0 ? p.Jf : p.Jb);
-      if (outF) outF += cidx * DD + (jtr ? (long long)n : (long long)n * kD);
-      uint8_t *outI = (g == 0 && p.Mimg) ? p.Mimg + ((ch.bh * 2 + ch.dir) * p.C + ch.c) * (long long)kImgBytes
-                                         : nullptr;
-      if (ch.nsteps == 0) {
+      const Chain ch_ = decode(p, q);
+      const long long cidx = ch_.bh * p.C + ch_.c;
+      float *outM = ch_.dir == 0 ? p.Mf : p.Mb, *outJ = ch_.dir == 0 ? p.Jf : p.Jb;
+      if (outM) outM += cidx * DD + (long long)n * kD;
+      if (outJ) outJ += cidx * DD + (p.jt ? (long long)n : (long long)n * kD);
+      uint8_t *outI = p.Mimg ? p.Mimg + ((ch_.bh * 2 + ch_.dir) * p.C + ch_.c) * (long long)kImgBytes : nullptr;
+      if (ch_.nsteps == 0) {
         // every frame of the chunk is an anchor: the identity map
 #pragma unroll 1
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 2; ++j) {
           float v[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = (g == 0 && 32 * j + e == n) ? 1.f : 0.f;
-          write_out(j, v, outF, outI);
+          for (int e = 0; e < 32; ++e) v[e] = (64 * ch + 32 * j + e == n) ? 1.f : 0.f;
+          write_out(0, j, v, outM, outI);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0.f;
+          write_out(1, j, v, outJ, nullptr);
         }
         continue;
       }
-      // ---- operand of the chain's first step: E_M = Diag(alpha), E_J = B
-      if (!wait_inputs(gs)) {
+      // ---- operands of the chain's first step
+      if (!first_m(gs) || !first_j(gs)) {
         ok = false;
         break;
       }
-      {
-        const float a_n = alpha_slot(gs)[n];
-        mbar_arrive(afree + 8 * (gs & 1));
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float v[32];
-          if (g == 0) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = (32 * j + e == n) ? a_n : 0.f;
-          } else {
-            load_b_row32(bbuf, j, n, v);
+      for (int s = 0; s < ch_.nsteps; ++s, ++gs) {
+        const bool last = s + 1 == ch_.nsteps;
+        if (!last && !wait_alpha(gs + 1)) {
+          ok = false;
+          break;
+        }
+        for (int g = 0; g < 2; ++g) {
+          if (g == 1 && !last && !wait_b(gs + 1)) {
+            ok = false;
+            break;
           }
-          put_operand(j, v);
-        }
-        publish();
-      }
-      for (int s = 0; s < ch.nsteps; ++s, ++gs) {
-        const bool last = s + 1 == ch.nsteps;
-        if (!last && !wait_inputs(gs + 1)) {
-          ok = false;
-          break;
-        }
-        if (!__all_sync(0xffffffffu, mbar_wait(done + 8 * g, (uint32_t)(gs & 1), abort))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (!last) {
-          // E = D Diag(alpha) (+ B) for the next step
-          const float *al = alpha_slot(gs + 1);
+          if (!__all_sync(0xffffffffu, mbar_wait(done + 8 * g, (uint32_t)(gs & 1), abort))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (!last) {
+            // E = D Diag(alpha) (+ B) for the next step
+            const float *al = alpha_slot(gs + 1);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float v[32], b[32];
-            tmem_ld32(tD + 32 * j, v);
-            if (g == 1) load_b_row32(bbuf, j, n, b);
+            for (int j = 0; j < 2; ++j) {
+              float v[32], b[32];
+              tmem_ld32(tD(g) + 32 * j, v);
+              if (g == 1) load_b_row32(bbuf, 2 * ch + j, n, b);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const float4 a4 = *reinterpret_cast<const float4 *>(al + 32 * j + 4 * c);
-              const float2 b01 = g == 1 ? make_float2(b[4 * c], b[4 * c + 1]) : make_float2(0.f, 0.f);
-              const float2 b23 = g == 1 ? make_float2(b[4 * c + 2], b[4 * c + 3]) : make_float2(0.f, 0.f);
-              const float2 r01 = __ffma2_rn(make_float2(v[4 * c], v[4 * c + 1]), make_float2(a4.x, a4.y), b01);
-              const float2 r23 =
-                  __ffma2_rn(make_float2(v[4 * c + 2], v[4 * c + 3]), make_float2(a4.z, a4.w), b23);
-              v[4 * c] = r01.x;
-              v[4 * c + 1] = r01.y;
-              v[4 * c + 2] = r23.x;
-              v[4 * c + 3] = r23.y;
+              for (int c = 0; c < 8; ++c) {
+                const float4 a4 = *reinterpret_cast<const float4 *>(al + 32 * j + 4 * c);
+                const float2 b01 = g == 1 ? make_float2(b[4 * c], b[4 * c + 1]) : make_float2(0.f, 0.f);
+                const float2 b23 = g == 1 ? make_float2(b[4 * c + 2], b[4 * c + 3]) : make_float2(0.f, 0.f);
+                const float2 r01 = __ffma2_rn(make_float2(v[4 * c], v[4 * c + 1]), make_float2(a4.x, a4.y), b01);
+                const float2 r23 =
+                    __ffma2_rn(make_float2(v[4 * c + 2], v[4 * c + 3]), make_float2(a4.z, a4.w), b23);
+                v[4 * c] = r01.x;
+                v[4 * c + 1] = r01.y;
+                v[4 * c + 2] = r23.x;
+                v[4 * c + 3] = r23.y;
+              }
+              put_operand(g, j, v);
             }
-            put_operand(j, v);
-          }
-          mbar_arrive(afree + 8 * ((gs + 1) & 1));
-          publish();
-        } else {
-          // the chain's result: Mc (fp32 rows and/or its image) or Jc
+            if (g == 1) {
+              mbar_arrive(bfree + 8 * ch);
+              mbar_arrive(afree + 8 * ((gs + 1) & 1));
+            }
+            publish(g);
+          } else {
+            // the chain's result: Mc (fp32 rows and/or its image) or Jc
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float v[32];
-            tmem_ld32(tD + 32 * j, v);
-            write_out(j, v, outF, outI);
+            for (int j = 0; j < 2; ++j) {
+              float v[32];
+              tmem_ld32(tD(g) + 32 * j, v);
+              if (g == 0)
+                write_out(0, j, v, outM, outI);
+              else
+                write_out(1, j, v, outJ, nullptr);
+            }
+            // the accumulator is read; the next chain's first operand follows
+            tc_fence_before();
           }
-          // the accumulator is read; the next chain's first operand follows
-          tc_fence_before();
         }
+        if (!ok) break;
       }
     }
     if (!ok) fail(abort, p.info);

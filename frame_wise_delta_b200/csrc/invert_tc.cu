@@ -231,16 +231,23 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         fence_proxy_async_smem();
         handoff_arrive(kBarPiReady);
       }
-      handoff_wait(kBarTReady);
       // S = R - Q^T X and S^{-1} by the sweep; S^{-1} replaces the staging
-      // (every thread has read its part before the sweep's first barrier)
+      // (every thread has read its part before the sweep's first barrier).
+      // R + I is read while the epilogue warps still compute Q^T X.
 #pragma unroll
       for (int a = 0; a < Sweep<64>::R; ++a)
 #pragma unroll
         for (int b = 0; b <= a; ++b) {
           const int r = rg + kSweepGrid * a, c = cg + kSweepGrid * b;
-          X.at(a, b) = __ldg(Af + (64 + r) * 128 + 64 + c) + (r == c ? 1.f : 0.f) -
-                       stage[r * 64 + (((c >> 2) ^ (r & 15)) << 2) + (c & 3)];
+          X.at(a, b) = __ldg(Af + (64 + r) * 128 + 64 + c) + (r == c ? 1.f : 0.f);
+        }
+      handoff_wait(kBarTReady);
+#pragma unroll
+      for (int a = 0; a < Sweep<64>::R; ++a)
+#pragma unroll
+        for (int b = 0; b <= a; ++b) {
+          const int r = rg + kSweepGrid * a, c = cg + kSweepGrid * b;
+          X.at(a, b) -= stage[r * 64 + (((c >> 2) ^ (r & 15)) << 2) + (c & 3)];
         }
       if constexpr (PRE_P)
         ok = X.run2(cbuf2, rg, cg, [] { bar_named(kBarSweep); }) && ok;
