@@ -14,6 +14,7 @@ from .vda import (  # noqa: F401
     readout_state,
     rel_frobenius,
     scan_states,
+    stream_segment,
     text_state,
     transition,
     vda_head,

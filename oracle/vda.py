@@ -228,6 +228,44 @@ def vda_head(inp: dict, chunk: int = 5, anchors: int = 0) -> dict:
     return out
 
 
+def stream_segment(Q, K, V, beta, alpha, S_prev, S_in, chunk: int = 5, anchor_first: bool = False):
+    """One segment of a live stream read through the forward memory only.
+
+    Reading of the page's livestream framing ("Future directions": continuous
+    generation with streaming systems): the frames after the segment do not
+    exist yet, so only the forward scan runs, carried from segment to segment;
+    each chunk c reads the forward state before the chunk ahead of it,
+    R_c = F_{max(c-1,0)} of the whole stream, with no backward term.
+    The segment starts on a chunk boundary; S_prev and S_in are the stream's
+    forward states before chunks c0 - 1 and c0 (for the first segment both are
+    the text state, counted once by the single scan); anchor_first makes the
+    segment's first frame an anchor (the stream's frame 0).
+
+    Q, K, V: [T, U, d]; beta: [T] (or [T, U]); alpha: [T, d_k].
+    Returns O [T, U, d_v] and F [C+1, d_v, d_k] with F[0] = S_in and F[j] the
+    state after the segment's chunks 0..j-1 (frame by frame, no chunk maps).
+    """
+    Q = _f64(Q)
+    T = K.shape[0]
+    C = num_chunks(T, chunk)
+    S = _f64(S_in).copy()
+    F = np.empty((C + 1,) + S.shape)
+    F[0] = S
+    for t in range(T):
+        if not (anchor_first and t == 0):
+            S = frame_update(S, alpha[t], *frame_stats(K[t], V[t], beta[t]))
+        if (t + 1) % chunk == 0 or t == T - 1:
+            F[num_chunks(t + 1, chunk)] = S
+    O = np.zeros((T,) + Q.shape[1:2] + (S.shape[0],))
+    for t in range(T):
+        if anchor_first and t == 0:
+            continue
+        c = t // chunk
+        R = _f64(S_prev) if c == 0 else F[c - 1]
+        O[t] = Q[t] @ R.T
+    return O, F
+
+
 def rel_frobenius(x, ref) -> float:
     """||x - ref||_F / ||ref||_F (0 when both are zero)."""
     x = _f64(x)
