@@ -35,12 +35,12 @@ ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # sha256 prefix of the kernel source the counters were taken on; reported as
 # None as soon as that source changes.
 NCU_TRAFFIC = {
-    "frame_grams": {"bytes": 1292.5e6 + 253.9e6, "source": "frame_wise_delta_b200/csrc/gram_tc.cu",
+    "frame_grams": {"bytes": 1291.9e6 + 253.8e6, "source": "frame_wise_delta_b200/csrc/gram_tc.cu",
                     "sha256_16": "00240b7db02fd61b", "workload": "h3"},
-    "frame_factor": {"bytes": 126.7e6 + 102.4e6, "source": "frame_wise_delta_b200/csrc/invert_tc.cu",
-                     "sha256_16": "85a8941c4be055cf", "workload": "h3"},
-    "chunk_readout": {"bytes": 700.7e6 + 581.2e6, "source": "frame_wise_delta_b200/csrc/readout_tc.cu",
-                      "sha256_16": "245d5ff033f12626", "workload": "h3"},
+    "frame_factor": {"bytes": 126.3e6 + 102.9e6, "source": "frame_wise_delta_b200/csrc/invert_tc.cu",
+                     "sha256_16": "d4085e639e7135a8", "workload": "h3"},
+    "chunk_readout": {"bytes": 700.7e6 + 581.7e6, "source": "frame_wise_delta_b200/csrc/readout_tc.cu",
+                      "sha256_16": "c1b3db4af3bc6542", "workload": "h3"},
 }
 
 
@@ -61,6 +61,9 @@ def parse():
                     help="time the pass with the readout epilogue (RMSNorm + sigmoid gate, synthetic gates)")
     ap.add_argument("--groups", type=int, default=1,
                     help="head groups of vdn_forward_pipelined (tensor path); 0 = plain vdn_forward")
+    ap.add_argument("--stream", type=int, default=0,
+                    help="time the causal streaming call instead: the clip as a live stream in segments of "
+                         "this many frames (a multiple of the chunk; >= T for one segment)")
     return ap.parse_args()
 
 
@@ -282,6 +285,9 @@ def main():
     f32 = dict(dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
+    if args.stream:
+        return stream_bench(args, w, s, d, dev, stream, barrier, rank, world, local)
+
     stages = ["text_state", "frame_grams", "frame_factor", "chunk_compose", "scan_bidir", "chunk_readout"]
     tensor_path = w.dtype == "bf16" and D == 128
     G = min(args.groups, B * H) if tensor_path else 0
@@ -414,6 +420,85 @@ def e2e_measure(args, host, d, make_forward, stream, barrier, world, frames_all,
     assert int(fwd.info.item()) == 0
     return {"value": frames_all / (te / e2e_steps / 1e3), "unit": "frames/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+
+
+def stream_bench(args, w, s, d, dev, stream, barrier, rank, world, local):
+    """The clip as a live stream through vdn_stream_segment: each step computes
+    the text state, then runs the segments in order, carrying the two forward
+    states between them (the states' copies are torch copies, not counted as
+    our launches). Each segment's inputs sit in their own buffers, as a
+    stream delivers them."""
+    import torch
+
+    from frame_wise_delta_b200 import dist as vdist
+    from frame_wise_delta_b200 import vdn
+
+    seg = min(args.stream, w.T)
+    if seg < w.T and seg % w.chunk:
+        raise SystemExit(f"--stream {seg}: segments must hold whole chunks of {w.chunk} frames")
+    cuts = [(t0, min(seg, w.T - t0)) for t0 in range(0, w.T, seg)]
+    shapes = {T: vdn.make_shape(w.B, w.H, T, w.U, w.d, w.n_text, w.chunk, w.anchors, w.dtype,
+                                beta_per_token=w.beta_per_token) for _, T in cuts}
+    ws = vdn.workspace(max(vdn.vdn_stream_workspace_bytes(x) for x in shapes.values()), dev)
+    tws = vdn.workspace(vdn.vdn_text_state_workspace_bytes(s), dev)
+    info = torch.zeros(1, dtype=torch.int32, device=dev)
+    parts = [{k: d[k][:, :, t0:t0 + T].contiguous() for k in ("Q", "K", "V", "beta", "alpha")} for t0, T in cuts]
+    outs = [(torch.empty((w.B, w.H, T, w.U, w.d), dtype=d["Q"].dtype, device=dev),
+             torch.empty((w.B, w.H, shapes[T].C + 1, w.d, w.d), dtype=torch.float32, device=dev)) for _, T in cuts]
+    S_T, S_prev, S_in = (torch.empty((w.B, w.H, w.d, w.d), dtype=torch.float32, device=dev) for _ in range(3))
+
+    def step():
+        vdn.vdn_text_state(s, d["Kx"], d["Vx"], d["beta_x"], S_T, tws, info)
+        sp, si = S_T, S_T
+        for (t0, T), x, (O, F) in zip(cuts, parts, outs):
+            vdn.vdn_stream_segment(shapes[T], x["Q"], x["K"], x["V"], x["beta"], x["alpha"], t0, sp, si, O, F, ws,
+                                   info)
+            C = shapes[T].C
+            S_prev.copy_(F[:, :, C - 1])
+            S_in.copy_(F[:, :, C])
+            sp, si = S_prev, S_in
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert int(info.item()) == 0, f"device status {int(info.item())}"
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    assert int(info.item()) == 0, f"device status {int(info.item())}"
+    ms_per_step = vdist.max_over_ranks(e0.elapsed_time(e1)) / args.steps
+    value = vdist.throughput(w.B * w.T, world, ms_per_step / 1e3)
+    tensor_path = w.dtype == "bf16" and w.d == 128
+    if rank == 0:
+        hbm_gbs, _, peak_src = load_peaks()
+        frac = alg_bytes(w) * world / (ms_per_step / 1e3) / (hbm_gbs * 1e9)
+        cfg = workload_config(w)
+        cfg["workload"] += f", causal stream in segments of {seg} frames"
+        print(json.dumps({
+            "metric": "stream frames/s", "value": value, "unit": "frames/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "state_dtype": "f32", "data": "synthetic", "config": cfg, "segments": len(cuts),
+            "roofline": {"kernel": "whole stream step", "bound": "hbm", "achieved": frac * hbm_gbs,
+                         "peak": hbm_gbs, "unit": "GB/s", "frac": frac, "traffic": None,
+                         "peak_source": f"{peak_src} HBM copy bandwidth"},
+            "gpu_launches": ((3 if tensor_path else 2) + 5 * len(cuts)) * args.steps,
+            "clocks": clk.summary()}), flush=True)
+    if world > 1:
+        dist_destroy()
+
+
+def dist_destroy():
+    import torch.distributed as dist
+    dist.barrier()
+    dist.destroy_process_group()
 
 
 def alg_bytes(w, gated=False):

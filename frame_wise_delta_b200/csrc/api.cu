@@ -81,7 +81,7 @@ vdn_status check_shape(const vdn_shape *s, Geo *g) {
   g->D = s->dk;
   g->chunk = s->chunk;
   g->C = (s->T + s->chunk - 1) / s->chunk;
-  g->anchors = s->anchors;
+  g->anchors = s->anchors ? 3 : 0;  // kernel mask: first and last frame
   g->n_text = s->n_text;
   g->in_dtype = s->in_dtype;
   g->out_dtype = s->out_dtype;
@@ -145,15 +145,17 @@ vdn_status run_grams(const Geo &g, const void *K, const void *V, const float *be
 }
 
 // og: the readout epilogue (step (5)), or nullptr
+// F0: the forward state chunk 0 reads instead of F[0] (streaming), or nullptr
 vdn_status run_readout(const Geo &g, const void *Q, const float *F, const float *G, void *O,
-                       int32_t *info, cudaStream_t st, const OutGate *og = nullptr) {
+                       int32_t *info, cudaStream_t st, const OutGate *og = nullptr,
+                       const float *F0 = nullptr) {
   if (g.BH * g.T * g.U == 0) return VDN_OK;
   if (readout_tc_supported(g.in_dtype, g.out_dtype, g.D, g.U)) {
-    VDN_CUDA(launch_readout_tc(Q, F, G, O, g.BH, g.T, g.U, g.chunk, g.anchors, info, st, og),
+    VDN_CUDA(launch_readout_tc(Q, F, G, O, g.BH, g.T, g.U, g.chunk, g.anchors, info, st, og, F0),
              "readout_tc");
   } else {
     VDN_CUDA(launch_readout_simt(Q, g.in_dtype, F, G, O, g.out_dtype, g.BH, g.T, g.U, g.chunk,
-                                 g.anchors, g.D, st, og),
+                                 g.anchors, g.D, st, og, F0),
              "readout_simt");
   }
   return VDN_OK;
@@ -525,6 +527,69 @@ vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K, const v
   VDN_TRY(mark(5));
   if (frames) VDN_TRY(run_readout(g, Q, Fo, Go, O, info, st, gate));
   VDN_TRY(mark(6));
+  return VDN_OK;
+}
+
+size_t vdn_stream_workspace_bytes(const vdn_shape *s) { return vdn_forward_workspace_bytes(s); }
+
+vdn_status vdn_stream_segment(const vdn_shape *s, const void *Q, const void *K, const void *V,
+                              const float *beta, const float *alpha, long long frame0, const float *S_prev,
+                              const float *S_in, void *O, float *F, void *workspace, size_t workspace_bytes,
+                              int32_t *info, vdn_stream_t stream) {
+  g_err[0] = 0;
+  Geo g;
+  VDN_TRY(check_shape(s, &g));
+  if (frame0 < 0 || frame0 % g.chunk != 0)
+    return fail(VDN_ERR_INVALID, "frame0 = %lld is not a non-negative multiple of chunk = %d", frame0, g.chunk);
+  // only the stream's first frame can be an anchor; there is no last one
+  g.anchors = (s->anchors && frame0 == 0) ? 1 : 0;
+  const bool frames = g.BH * g.T > 0;
+  VDN_TRY(need(Q, "Q", frames && g.U > 0));
+  VDN_TRY(need(K, "K", frames && g.U > 0));
+  VDN_TRY(need(V, "V", frames && g.U > 0));
+  VDN_TRY(need(beta, "beta", frames && g.U > 0));
+  VDN_TRY(need(alpha, "alpha", frames));
+  VDN_TRY(need(S_prev, "S_prev", g.BH > 0));
+  VDN_TRY(need(S_in, "S_in", g.BH > 0));
+  VDN_TRY(need(O, "O", frames && g.U > 0));
+  VDN_TRY(need(F, "F", g.BH > 0));
+  VDN_TRY(need(info, "info", true));
+  const FwdLayout L = fwd_layout(g);
+  VDN_TRY(need(workspace, "workspace", g.BH > 0));
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(VDN_ERR_INVALID, "workspace is not 256-byte aligned");
+  if (workspace_bytes < L.total)
+    return fail(VDN_ERR_INVALID, "workspace of %zu bytes < %zu required", workspace_bytes, L.total);
+  if (g.BH == 0) return VDN_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  char *w = (char *)workspace;
+  float *A = (float *)(w + L.a), *Bm = (float *)(w + L.b);
+  uint8_t *Wimg = (uint8_t *)(w + L.wimg), *Mimg = (uint8_t *)(w + L.mimg);
+  float *Mf = (float *)(w + L.mf), *Jf = (float *)(w + L.jf);
+  float *Mb = (float *)(w + L.mb), *Jb = (float *)(w + L.jb);
+  const bool tc = tensor_path(g);
+  VDN_CUDA(cudaMemsetAsync(info, 0, sizeof(int32_t), st), "memset info");
+  if (frames) {
+    uint8_t *Pimg = tc ? (uint8_t *)(w + L.pimg) : nullptr;
+    VDN_TRY(run_grams(g, K, V, beta, A, Bm, g.BH * g.T, g.U, info, st, Pimg));
+    if (tc) {
+      VDN_CUDA(launch_invert_tc(A, nullptr, Wimg, info, g.BH * g.T, st, 0, Pimg), "invert");
+      VDN_CUDA(launch_compose_tc(Wimg, Bm, alpha, nullptr, Jf, nullptr, nullptr, Mimg, g.BH, g.T, g.chunk,
+                                 g.anchors, 1, true, info, st),
+               "compose");
+      VDN_CUDA(launch_scan_tc(Mimg, Jf, nullptr, S_in, F, nullptr, g.BH, g.C, info, st, /*dir_mask=*/1,
+                              /*init_scale=*/1.f),
+               "scan");
+    } else {
+      VDN_CUDA(launch_factor_simt(A, Bm, alpha, A, Bm, info, g.BH * g.T, g.T, g.anchors, g.D, st), "factor");
+      VDN_CUDA(launch_compose_simt(A, Bm, Mf, Jf, Mb, Jb, g.BH, g.T, g.chunk, g.D, st), "compose");
+      VDN_CUDA(launch_scan_simt(Mf, Jf, nullptr, nullptr, S_in, F, nullptr, g.BH, g.C, g.D, 1, st, 1.f), "scan");
+    }
+    VDN_TRY(run_readout(g, Q, F, nullptr, O, info, st, nullptr, S_prev));
+  } else {
+    VDN_CUDA(launch_scan_simt(nullptr, nullptr, nullptr, nullptr, S_in, F, nullptr, g.BH, 0, g.D, 1, st, 1.f),
+             "scan");
+  }
   return VDN_OK;
 }
 

@@ -71,8 +71,9 @@ struct ComposeArgs {
   int jt;  // J outputs transposed (Jc[n][m] at m * d + n)
 };
 
-// A chain and the frames it takes: anchors only sit at t = 0 and t = T - 1,
-// so the non-anchor frames of a chunk are the contiguous range [lo, hi].
+// A chain and the frames it takes: anchors only sit at t = 0 (anchors bit 0)
+// and t = T - 1 (bit 1), so the non-anchor frames of a chunk are the
+// contiguous range [lo, hi].
 struct Chain {
   long long bh;
   int dir, c, lo, hi, nsteps;
@@ -86,8 +87,8 @@ __device__ __forceinline__ Chain decode(const ComposeArgs &p, long long q) {
   ch.bh = r % p.BH;
   ch.c = (int)(r / p.BH);
   const int t0 = ch.c * p.chunk, t1 = min(t0 + p.chunk, p.T);
-  ch.lo = (p.anchors && t0 == 0) ? 1 : t0;
-  ch.hi = (p.anchors && t1 == p.T) ? p.T - 2 : t1 - 1;
+  ch.lo = ((p.anchors & 1) && t0 == 0) ? 1 : t0;
+  ch.hi = ((p.anchors & 2) && t1 == p.T) ? p.T - 2 : t1 - 1;
   ch.nsteps = max(ch.hi - ch.lo + 1, 0);
   return ch;
 }

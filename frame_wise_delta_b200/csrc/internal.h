@@ -9,6 +9,8 @@
 namespace vdn {
 
 // Generic CUDA-core kernels: any d in {16, 32, 64, 128}, float32 or bf16 inputs.
+// `anchors` is a mask throughout: bit 0 makes the first frame of each (b, h)
+// an anchor, bit 1 the last one (identity transitions, zero reads).
 // beta: one gate per frame ([nframes]) or, with per_token, per token ([nframes, U])
 cudaError_t launch_gram_simt(const void *K, const void *V, int in_dtype, const float *beta, bool per_token,
                              float *A, float *Bm, long long nframes, int U, int D, cudaStream_t st);
@@ -18,9 +20,11 @@ cudaError_t launch_factor_simt(const float *A, const float *Bm, const float *alp
 cudaError_t launch_compose_simt(const float *M, const float *J, float *Mf, float *Jf, float *Mb,
                                 float *Jb, long long BH, int T, int chunk, int D, cudaStream_t st);
 // dir_mask: bit 0 forward (writes F), bit 1 backward (writes G).
+// Both scans start from init_scale * S_T (1/2: the two scans share the text
+// state; 1: a forward-only scan from a carried state).
 cudaError_t launch_scan_simt(const float *Mf, const float *Jf, const float *Mb, const float *Jb,
                              const float *S_T, float *F, float *G, long long BH, int C, int D,
-                             int dir_mask, cudaStream_t st);
+                             int dir_mask, cudaStream_t st, float init_scale = 0.5f);
 // Readout epilogue of step (5): y = o / sqrt(mean o^2 + eps) * w[h] * sigmoid(gate),
 // per token over its d channels; gate == nullptr leaves o as it is.
 struct OutGate {
@@ -29,9 +33,12 @@ struct OutGate {
   float eps;
   int H;
 };
+// R_c = F[max(c - 1, 0)] + G[min(c + 2, C)]; G may be null (forward reads
+// only) and F0 ([BH, d, d], may be null) replaces F[0] for chunk 0.
 cudaError_t launch_readout_simt(const void *Q, int in_dtype, const float *F, const float *G, void *O,
                                 int out_dtype, long long BH, int T, int U, int chunk, int anchors,
-                                int D, cudaStream_t st, const OutGate *og = nullptr);
+                                int D, cudaStream_t st, const OutGate *og = nullptr,
+                                const float *F0 = nullptr);
 
 // Tensor-core kernels (tcgen05 + TMA), bf16 inputs, d = 128.
 bool gram_tc_supported(int in_dtype, int D, int U);
@@ -45,7 +52,7 @@ cudaError_t launch_gram_tc(const void *K, const void *V, const float *beta, bool
 bool readout_tc_supported(int in_dtype, int out_dtype, int D, int U);
 cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, void *O, long long BH,
                               int T, int U, int chunk, int anchors, int32_t *info, cudaStream_t st,
-                              const OutGate *og = nullptr);
+                              const OutGate *og = nullptr, const float *F0 = nullptr);
 
 // W = (I + A)^{-1} per frame (CUDA cores); W fp32 and/or Wimg (hi/lo MMA
 // images of kImgBytes per frame, d = 128 only), each optional.
@@ -70,10 +77,12 @@ cudaError_t launch_compose_tc(const uint8_t *Wimg, const float *Bm, const float 
                               float *Jf, float *Mb, float *Jb, uint8_t *Mimg, long long BH, int T,
                               int chunk, int anchors, int ndirs, bool j_transposed, int32_t *info,
                               cudaStream_t st);
-// Both scans from the compose's Mc images and transposed fp32 Jc (tensor
-// cores, d = 128).
+// Both scans (dir_mask bit 0 forward, bit 1 backward) from the compose's Mc
+// images and transposed fp32 Jc (tensor cores, d = 128), started from
+// init_scale * S_T.
 cudaError_t launch_scan_tc(const uint8_t *Mimg, const float *Jf, const float *Jb, const float *S_T,
-                           float *F, float *G, long long BH, int C, int32_t *info, cudaStream_t st);
+                           float *F, float *G, long long BH, int C, int32_t *info, cudaStream_t st,
+                           int dir_mask = 3, float init_scale = 0.5f);
 
 // Message returned by vdn_last_error() on this thread.
 void set_last_error(const char *msg);

@@ -51,7 +51,8 @@ constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 2 * kRBytes
 
 struct ReadoutArgs {
   const float *F;
-  const float *G;
+  const float *G;   // optional (forward reads only when null)
+  const float *F0;  // optional: per-b*h forward state chunk 0 reads instead of F[0]
   __nv_bfloat16 *O;
   int32_t *info;
   long long nframes;
@@ -69,7 +70,7 @@ __device__ __forceinline__ void fail(volatile int *abort, int32_t *info) {
 
 __device__ __forceinline__ bool is_anchor(const ReadoutArgs &p, long long f) {
   const int t = (int)(f % p.T);
-  return p.anchors && (t == 0 || t == p.T - 1);
+  return ((p.anchors & 1) && t == 0) || ((p.anchors & 2) && t == p.T - 1);
 }
 
 __device__ __forceinline__ long long chunk_key(const ReadoutArgs &p, long long f) {
@@ -258,13 +259,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         cur = key;
         const long long bh = f / p.T;
         const int c = (int)((f % p.T) / p.chunk);
-        const float *Fs = p.F + (bh * (p.C + 1) + max(c - 1, 0)) * (long long)(kD * kD);
-        const float *Gs = p.G + (bh * (p.C + 1) + min(c + 2, p.C)) * (long long)(kD * kD);
+        const float *Fs = (c == 0 && p.F0) ? p.F0 + bh * (long long)(kD * kD)
+                                           : p.F + (bh * (p.C + 1) + max(c - 1, 0)) * (long long)(kD * kD);
+        const float *Gs = p.G ? p.G + (bh * (p.C + 1) + min(c + 2, p.C)) * (long long)(kD * kD) : nullptr;
         for (int e8 = et; e8 < kD * kD / 8; e8 += 256) {
           const int i = e8 >> 4, k0 = (e8 & 15) * 8;
           const float4 *f4 = reinterpret_cast<const float4 *>(Fs + i * kD + k0);
-          const float4 *g4 = reinterpret_cast<const float4 *>(Gs + i * kD + k0);
-          const float4 a0 = f4[0], a1 = f4[1], b0 = g4[0], b1 = g4[1];
+          const float4 a0 = f4[0], a1 = f4[1];
+          float4 b0 = make_float4(0.f, 0.f, 0.f, 0.f), b1 = b0;
+          if (Gs) {
+            const float4 *g4 = reinterpret_cast<const float4 *>(Gs + i * kD + k0);
+            b0 = g4[0];
+            b1 = g4[1];
+          }
           const float r[8] = {a0.x + b0.x, a0.y + b0.y, a0.z + b0.z, a0.w + b0.w,
                               a1.x + b1.x, a1.y + b1.y, a1.z + b1.z, a1.w + b1.w};
           uint4 h, l;
@@ -407,7 +414,7 @@ bool readout_tc_supported(int in_dtype, int out_dtype, int D, int U) {
 
 cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, void *O, long long BH,
                               int T, int U, int chunk, int anchors, int32_t *info, cudaStream_t st,
-                              const OutGate *og) {
+                              const OutGate *og, const float *F0) {
   const long long nframes = BH * T;
   if (nframes <= 0) return cudaSuccess;
   CUtensorMap tmQ, tmO, tmG;
@@ -420,7 +427,7 @@ cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, voi
   if (e != cudaSuccess) return e;
   const int sms = device_sm_count();
   const long long grid = nframes < sms ? nframes : sms;
-  ReadoutArgs a{F, G, (__nv_bfloat16 *)O, info, nframes, T, U, chunk, anchors,
+  ReadoutArgs a{F, G, F0, (__nv_bfloat16 *)O, info, nframes, T, U, chunk, anchors,
                 (T + chunk - 1) / chunk, (U + kNT - 1) / kNT,
                 gated ? og->w : nullptr, gated ? og->eps : 0.f, gated ? og->H : 1};
   readout_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(tmQ, tmO, tmG, a);

@@ -54,6 +54,7 @@ struct ScanArgs {
   float *F, *G;              // [BH, C+1, d, d]
   int32_t *info;
   int C;
+  float init_scale;          // the state starts as init_scale * S_T
 };
 
 __device__ __forceinline__ void fail(volatile int *abort, int32_t *info) {
@@ -206,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float *o = (dir == 0 ? p.F + (bh * (p.C + 1)) * DD : p.G + (bh * (p.C + 1) + p.C) * DD) + m;
       float v[kRows];  // every load first: one memory latency, not one per row
 #pragma unroll
-      for (int e = 0; e < kRows; ++e) v[e] = 0.5f * st[(row0 + e) * kD];
+      for (int e = 0; e < kRows; ++e) v[e] = p.init_scale * st[(row0 + e) * kD];
 #pragma unroll
       for (int e = 0; e < kRows; ++e) o[(row0 + e) * kD] = v[e];
       if (nsteps > 0) {
@@ -282,12 +283,13 @@ bool make_jt_map(CUtensorMap *m, const float *J, long long maps) {
 }  // namespace
 
 cudaError_t launch_scan_tc(const uint8_t *Mimg, const float *Jf, const float *Jb, const float *S_T,
-                           float *F, float *G, long long BH, int C, int32_t *info, cudaStream_t st) {
+                           float *F, float *G, long long BH, int C, int32_t *info, cudaStream_t st,
+                           int dir_mask, float init_scale) {
   if (BH <= 0) return cudaSuccess;
   // with no chunks the maps are never read: describe S_T instead of empty Jc
   CUtensorMap tmJf, tmJb;
   const long long maps = C > 0 ? BH * C : BH;
-  if (!make_jt_map(&tmJf, C > 0 ? Jf : S_T, maps) || !make_jt_map(&tmJb, C > 0 ? Jb : S_T, maps))
+  if (!make_jt_map(&tmJf, C > 0 ? Jf : S_T, maps) || !make_jt_map(&tmJb, C > 0 ? (Jb ? Jb : Jf) : S_T, maps))
     return cudaErrorInvalidValue;
   ScanArgs a{};
   a.Mimg = Mimg;
@@ -296,9 +298,11 @@ cudaError_t launch_scan_tc(const uint8_t *Mimg, const float *Jf, const float *Jb
   a.G = G;
   a.info = info;
   a.C = C;
+  a.init_scale = init_scale;
   cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  scan_tc_kernel<<<dim3((unsigned)BH, 2, 2), kThreads, kSmemBytes, st>>>(tmJf, tmJb, a);
+  // forward only: grid.y = 1 (direction 0); backward only is not needed
+  scan_tc_kernel<<<dim3((unsigned)BH, dir_mask == 1 ? 1 : 2, 2), kThreads, kSmemBytes, st>>>(tmJf, tmJb, a);
   return cudaGetLastError();
 }
 

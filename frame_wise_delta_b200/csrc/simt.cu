@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(kThreads, 1) factor_simt_kernel(
   const int rg = threadIdx.x / 16, cg = threadIdx.x % 16;
   const long long base = f * (long long)D * D;
 
-  if (anchors && (t == 0 || t == T - 1)) {  // identity transition
+  if (((anchors & 1) && t == 0) || ((anchors & 2) && t == T - 1)) {  // identity transition
 #pragma unroll
     for (int a = 0; a < RA; ++a)
 #pragma unroll
@@ -284,7 +284,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads) scan_simt_kernel(
     const float *__restrict__ Mf, const float *__restrict__ Jf, const float *__restrict__ Mb,
     const float *__restrict__ Jb, const float *__restrict__ S_T, float *__restrict__ F,
-    float *__restrict__ G, int C, int dir_mask) {
+    float *__restrict__ G, int C, int dir_mask, float init_scale) {
   constexpr int RB = D / 16;
   constexpr int RR = 16;  // state rows per block
   extern __shared__ __align__(16) float sm[];
@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(kThreads) scan_simt_kernel(
 #pragma unroll
   for (int b = 0; b < RB; ++b) {
     const int j = cg + 16 * b;
-    s[b] = 0.5f * S_T[bh * DD + (r0 + r) * D + j];
+    s[b] = init_scale * S_T[bh * DD + (r0 + r) * D + j];
     Ss[r * D + j] = s[b];
     out[(bh * (C + 1) + (dir == 0 ? 0 : C)) * DD + (r0 + r) * D + j] = s[b];
   }
@@ -340,7 +340,8 @@ __global__ void __launch_bounds__(kThreads) scan_simt_kernel(
 template <int D, typename Tin, typename Tout>
 __global__ void __launch_bounds__(kThreads) readout_simt_kernel(
     const Tin *__restrict__ Q, const float *__restrict__ F, const float *__restrict__ G,
-    Tout *__restrict__ O, int T, int U, int chunk, int anchors, int C, OutGate og) {
+    Tout *__restrict__ O, int T, int U, int chunk, int anchors, int C, OutGate og,
+    const float *__restrict__ F0) {
   constexpr int TU = 64;
   constexpr int RB = D / 16;
   constexpr int LD = D + 1;
@@ -355,7 +356,7 @@ __global__ void __launch_bounds__(kThreads) readout_simt_kernel(
   const long long DD = (long long)D * D;
   Tout *Of = O + f * (long long)U * D;
 
-  if (anchors && (t == 0 || t == T - 1)) {
+  if (((anchors & 1) && t == 0) || ((anchors & 2) && t == T - 1)) {
     for (int e = threadIdx.x; e < TU * D; e += kThreads) {
       const int u = u0 + e / D;
       if (u < U) store_val(&Of[(long long)u * D + e % D], 0.f);
@@ -363,11 +364,11 @@ __global__ void __launch_bounds__(kThreads) readout_simt_kernel(
     return;
   }
   const int c = t / chunk;
-  const float *Fs = F + (bh * (C + 1) + max(c - 1, 0)) * DD;
-  const float *Gs = G + (bh * (C + 1) + min(c + 2, C)) * DD;
+  const float *Fs = (c == 0 && F0) ? F0 + bh * DD : F + (bh * (C + 1) + max(c - 1, 0)) * DD;
+  const float *Gs = G ? G + (bh * (C + 1) + min(c + 2, C)) * DD : nullptr;
   for (int e = threadIdx.x; e < D * D; e += kThreads) {
     const int i = e / D, k = e % D;
-    Rt[k * LD + i] = Fs[e] + Gs[e];
+    Rt[k * LD + i] = Fs[e] + (Gs ? Gs[e] : 0.f);
   }
   const Tin *Qf = Q + f * (long long)U * D;
   for (int e = threadIdx.x; e < TU * D; e += kThreads) {
@@ -453,19 +454,19 @@ cudaError_t compose_d(const float *M, const float *J, float *Mf, float *Jf, floa
 template <int D>
 cudaError_t scan_d(const float *Mf, const float *Jf, const float *Mb, const float *Jb,
                    const float *S_T, float *F, float *G, long long BH, int C, int dir_mask,
-                   cudaStream_t st) {
+                   float init_scale, cudaStream_t st) {
   const size_t smem = (size_t)(D * D + 16 * D) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(scan_simt_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)BH, 2, D / 16);
-  scan_simt_kernel<D><<<grid, kThreads, smem, st>>>(Mf, Jf, Mb, Jb, S_T, F, G, C, dir_mask);
+  scan_simt_kernel<D><<<grid, kThreads, smem, st>>>(Mf, Jf, Mb, Jb, S_T, F, G, C, dir_mask, init_scale);
   return cudaGetLastError();
 }
 
 template <int D, typename Tin, typename Tout>
 cudaError_t readout_dt(const void *Q, const float *F, const float *G, void *O, long long BH, int T,
-                       int U, int chunk, int anchors, cudaStream_t st, const OutGate &og) {
+                       int U, int chunk, int anchors, cudaStream_t st, const OutGate &og, const float *F0) {
   const int C = (T + chunk - 1) / chunk;
   const size_t smem = (size_t)(D * (D + 1) + 64 * D) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(readout_simt_kernel<D, Tin, Tout>,
@@ -473,22 +474,22 @@ cudaError_t readout_dt(const void *Q, const float *F, const float *G, void *O, l
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)(BH * T), (unsigned)((U + 63) / 64));
   readout_simt_kernel<D, Tin, Tout><<<grid, kThreads, smem, st>>>(
-      (const Tin *)Q, F, G, (Tout *)O, T, U, chunk, anchors, C, og);
+      (const Tin *)Q, F, G, (Tout *)O, T, U, chunk, anchors, C, og, F0);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t readout_d(const void *Q, int in_dtype, const float *F, const float *G, void *O,
                       int out_dtype, long long BH, int T, int U, int chunk, int anchors,
-                      cudaStream_t st, const OutGate &og) {
+                      cudaStream_t st, const OutGate &og, const float *F0) {
   if (in_dtype == VDN_BF16) {
     if (out_dtype == VDN_BF16)
-      return readout_dt<D, __nv_bfloat16, __nv_bfloat16>(Q, F, G, O, BH, T, U, chunk, anchors, st, og);
-    return readout_dt<D, __nv_bfloat16, float>(Q, F, G, O, BH, T, U, chunk, anchors, st, og);
+      return readout_dt<D, __nv_bfloat16, __nv_bfloat16>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0);
+    return readout_dt<D, __nv_bfloat16, float>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0);
   }
   if (out_dtype == VDN_BF16)
-    return readout_dt<D, float, __nv_bfloat16>(Q, F, G, O, BH, T, U, chunk, anchors, st, og);
-  return readout_dt<D, float, float>(Q, F, G, O, BH, T, U, chunk, anchors, st, og);
+    return readout_dt<D, float, __nv_bfloat16>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0);
+  return readout_dt<D, float, float>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0);
 }
 
 }  // namespace
@@ -530,18 +531,18 @@ cudaError_t launch_compose_simt(const float *M, const float *J, float *Mf, float
 
 cudaError_t launch_scan_simt(const float *Mf, const float *Jf, const float *Mb, const float *Jb,
                              const float *S_T, float *F, float *G, long long BH, int C, int D,
-                             int dir_mask, cudaStream_t st) {
+                             int dir_mask, cudaStream_t st, float init_scale) {
   if (BH <= 0) return cudaSuccess;
-  VDN_DISPATCH_D(D, scan_d<DD_>(Mf, Jf, Mb, Jb, S_T, F, G, BH, C, dir_mask, st))
+  VDN_DISPATCH_D(D, scan_d<DD_>(Mf, Jf, Mb, Jb, S_T, F, G, BH, C, dir_mask, init_scale, st))
 }
 
 cudaError_t launch_readout_simt(const void *Q, int in_dtype, const float *F, const float *G, void *O,
                                 int out_dtype, long long BH, int T, int U, int chunk, int anchors,
-                                int D, cudaStream_t st, const OutGate *og) {
+                                int D, cudaStream_t st, const OutGate *og, const float *F0) {
   if (BH <= 0 || T <= 0 || U <= 0) return cudaSuccess;
   const OutGate none{nullptr, nullptr, 0.f, 1};
   const OutGate &g = og ? *og : none;
-  VDN_DISPATCH_D(D, readout_d<DD_>(Q, in_dtype, F, G, O, out_dtype, BH, T, U, chunk, anchors, st, g))
+  VDN_DISPATCH_D(D, readout_d<DD_>(Q, in_dtype, F, G, O, out_dtype, BH, T, U, chunk, anchors, st, g, F0))
 }
 
 }  // namespace vdn

@@ -86,6 +86,7 @@ _SIGS = {
     "vdn_text_state_noalloc": [_P, _P, _P, _P, _P, _P, _P],
     "vdn_forward_pipelined": [_P] * 13 + [ctypes.c_size_t, _P, ctypes.c_int32, _P, _P, _P, _P],
     "vdn_chunk_readout_gated": [_P] * 8,
+    "vdn_stream_segment": [_P] * 6 + [ctypes.c_longlong] + [_P] * 5 + [ctypes.c_size_t, _P, _P],
 }
 
 
@@ -101,7 +102,8 @@ def lib() -> ctypes.CDLL:
             fn = getattr(L, name)
             fn.argtypes = args
             fn.restype = ctypes.c_int
-        for name in ("vdn_text_state_workspace_bytes", "vdn_forward_workspace_bytes"):
+        for name in ("vdn_text_state_workspace_bytes", "vdn_forward_workspace_bytes",
+                     "vdn_stream_workspace_bytes"):
             fn = getattr(L, name)
             fn.argtypes = [_P]
             fn.restype = ctypes.c_size_t
@@ -257,6 +259,18 @@ def vdn_chunk_readout_gated(s, Q, F, G, og, O, info=None, stream=None):
                                          _stream(stream)))
 
 
+def vdn_stream_workspace_bytes(s) -> int:
+    return int(lib().vdn_stream_workspace_bytes(_shp(s)))
+
+
+def vdn_stream_segment(s, Q, K, V, beta, alpha, frame0, S_prev, S_in, O, F, workspace, info, stream=None):
+    """One segment of a live stream through the forward memory only (see vdn.h)."""
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().vdn_stream_segment(_shp(s), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(alpha), int(frame0),
+                                    _ptr(S_prev), _ptr(S_in), _ptr(O), _ptr(F), _ptr(workspace), nbytes,
+                                    _ptr(info), _stream(stream)))
+
+
 def vdn_status_string(status: int) -> str:
     return lib().vdn_status_string(status).decode()
 
@@ -273,6 +287,32 @@ def vdn_version() -> int:
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:
     """A 256-byte-aligned uint8 device buffer of at least nbytes bytes."""
     return torch.empty(max(1, nbytes), dtype=torch.uint8, device=device)
+
+
+class Stream:
+    """A live stream read through the forward memory: call with each segment's
+    frames (whole chunks except the last); the carried states (the forward
+    states before the last two chunks) start as the text state S^T."""
+
+    def __init__(self, s: vdn_shape, S_T: torch.Tensor, device="cuda"):
+        self.s = s
+        self.ws = workspace(vdn_stream_workspace_bytes(s), device)
+        self.info = torch.zeros(1, dtype=torch.int32, device=device)
+        self.O = torch.empty((s.B, s.H, s.T, s.U, s.dv), dtype=TORCH_DTYPE[s.out_dtype], device=device)
+        self.F = torch.empty((s.B, s.H, s.C + 1, s.dv, s.dk), dtype=torch.float32, device=device)
+        self.S_prev = S_T.clone()
+        self.S_in = S_T.clone()
+        self.frame0 = 0
+
+    def __call__(self, Q, K, V, beta, alpha, stream=None):
+        vdn_stream_segment(self.s, Q, K, V, beta, alpha, self.frame0, self.S_prev, self.S_in, self.O, self.F,
+                           self.ws, self.info, stream)
+        C = self.s.C
+        if C > 0:
+            self.S_prev.copy_(self.F[:, :, C - 1])
+            self.S_in.copy_(self.F[:, :, C])
+        self.frame0 += self.s.T
+        return self.O
 
 
 class Forward:

@@ -301,6 +301,44 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
                                  const void *const *events, const vdn_out_gate *og,
                                  vdn_stream_t stream);
 
+/*
+ * Causal streaming variant: one segment of a live stream, read through the
+ * forward memory only. Paper: "Video DeltaNet: A Video-Native Hybrid
+ * Attention for Livestream Video Generation" (summary page) — the method
+ * targets livestream generation ("Future directions": continuous generation
+ * with streaming systems). In a stream the frames after the current segment
+ * do not exist yet, so the backward scan cannot run; this call keeps the
+ * forward scan, carried from segment to segment, and each chunk c of the
+ * stream reads R_c = F_{max(c-1,0)} (the forward state before the chunk
+ * ahead of it), with no backward term.
+ * The segment holds frames frame0 .. frame0 + T - 1 of the stream (shape.T =
+ * T; frame0 a multiple of shape.chunk; every segment but the stream's last
+ * holds whole chunks). shape.n_text is not used: the text state enters
+ * through the carried states. With shape.anchors the stream's first frame
+ * (frame0 = 0 only) is an anchor; a stream has no last-frame anchor.
+ * In : Q, K, V [B,H,T,U,d] (in_dtype); beta [B,H,T] (or [B,H,T,U] with
+ *      beta_per_token), alpha [B,H,T,dk] float32;
+ *      S_prev, S_in [B,H,dv,dk] float32: the stream's forward states before
+ *      chunks c0 - 1 and c0 (c0 = frame0 / chunk); for the first segment
+ *      both are the text state S^T (vdn_text_state), which a forward-only
+ *      stream counts once.
+ * Out: O [B,H,T,U,dv] (out_dtype); F [B,H,C+1,dv,dk] float32: F[0] = S_in
+ *      and F[c+1] the state after the segment's chunk c (C = ceil(T /
+ *      chunk)). The next segment continues from S_prev = F[C - 1] and
+ *      S_in = F[C]. *info as for vdn_frame_factor.
+ * workspace: at least vdn_stream_workspace_bytes(s) bytes, 256-byte aligned.
+ * Errors: VDN_ERR_INVALID for a frame0 that is negative or not a multiple of
+ * the chunk, and as for vdn_forward. Same kernels as vdn_forward (the
+ * tensor-core path for bf16 d = 128), run in one direction.
+ */
+size_t vdn_stream_workspace_bytes(const vdn_shape *s);
+vdn_status vdn_stream_segment(const vdn_shape *s, const void *Q, const void *K,
+                              const void *V, const float *beta, const float *alpha,
+                              long long frame0, const float *S_prev, const float *S_in,
+                              void *O, float *F, void *workspace,
+                              size_t workspace_bytes, int32_t *info,
+                              vdn_stream_t stream);
+
 /* Name of a status code (static string). */
 const char *vdn_status_string(vdn_status st);
 /* Message of the last failing call on this thread ("" if none). */
