@@ -4,6 +4,8 @@ Test infrastructure only: imported by the tests, the smoke check and the
 benchmark's CPU-baseline leg, never by the product path.
 """
 from .vda import (  # noqa: F401
+    bridge_factors,
+    bridged_readout,
     chunk_maps,
     chunk_readout,
     frame_stats,

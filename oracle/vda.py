@@ -168,6 +168,55 @@ def chunk_readout(Q, F, G, chunk: int = 5, anchors: int = 0):
     return O
 
 
+def bridge_factors(alpha, t: int, chunk: int = 5, anchors: int = 0):
+    """Decay bridge of "Method steps" step (5) for query frame t.
+
+    Reading: the forward state read by chunk c = t // chunk holds the frames
+    before its window (chunks c-1..c+1, clipped), i.e. frames < f0 with
+    f0 = chunk * max(c - 1, 0); the window's frames write through the softmax
+    branch, not the memory, but their decay still acts, so the state is
+    carried to frame t through Diag(alpha_r) for r = f0..t. The backward state
+    holds the frames after the window, > f1 = min(chunk * (c + 2), T) - 1, and
+    is carried down to t through r = f1..t. An anchor frame's transition is
+    the identity, so its alpha counts as 1.
+    alpha: [T, d_k]. Returns (pf, pb), each [d_k].
+    """
+    alpha = _f64(alpha)
+    T, d_k = alpha.shape
+    c = t // chunk
+    f0 = chunk * max(c - 1, 0)
+    f1 = min(chunk * (c + 2), T) - 1
+    pf = np.ones(d_k)
+    for r in range(f0, t + 1):
+        if not is_anchor(r, T, anchors):
+            pf = pf * alpha[r]
+    pb = np.ones(d_k)
+    for r in range(t, f1 + 1):
+        if not is_anchor(r, T, anchors):
+            pb = pb * alpha[r]
+    return pf, pb
+
+
+def bridged_readout(Q, F, G, alpha, chunk: int = 5, anchors: int = 0):
+    """Linear-branch readout with the decay bridge (step (5)):
+    o_{t,u} = R_t q_{t,u} with R_t = F_{max(c-1,0)} Diag(pf_t) + G_{min(c+2,C)} Diag(pb_t)
+    (bridge_factors); anchor rows read nothing. With every alpha = 1 this is
+    chunk_readout. Q: [T, U, d_k], alpha: [T, d_k] -> O: [T, U, d_v]."""
+    Q = _f64(Q)
+    T, U, _ = Q.shape
+    C = F.shape[0] - 1
+    d_v = F.shape[1]
+    O = np.zeros((T, U, d_v))
+    for t in range(T):
+        if is_anchor(t, T, anchors):
+            continue
+        c = t // chunk
+        pf, pb = bridge_factors(alpha, t, chunk, anchors)
+        R = _f64(F[max(c - 1, 0)]) * pf[None, :] + _f64(G[min(c + 2, C)]) * pb[None, :]
+        O[t] = Q[t] @ R.T
+    return O
+
+
 def gated_rmsnorm(O, weight, gate, eps: float = 1e-6):
     """Readout epilogue of "Method steps" step (5): RMSNorm of every token's
     readout over its d_v channels, then a sigmoid gate, channel by channel:
@@ -212,16 +261,20 @@ def chunk_maps(K, V, beta, alpha, chunk: int = 5, anchors: int = 0):
     return Mf, Jf, Mb, Jb
 
 
-def vda_head(inp: dict, chunk: int = 5, anchors: int = 0) -> dict:
+def vda_head(inp: dict, chunk: int = 5, anchors: int = 0, bridge: bool = False) -> dict:
     """The whole linear branch for one (batch, head) pair.
 
     inp holds Q, K, V [T, U, d], Kx, Vx [n_text, d], beta [T], alpha [T, d]
     and beta_x; with gate [T, U, d] and norm_w [d] also the gated RMSNorm
-    output Y. Returns S_T, F, G, O (and Y), all float64.
+    output Y. bridge: read through the decay bridge (bridged_readout).
+    Returns S_T, F, G, O (and Y), all float64.
     """
     S_T = text_state(inp["Kx"], inp["Vx"], inp.get("beta_x", 1.0))
     F, G = scan_states(inp["K"], inp["V"], inp["beta"], inp["alpha"], S_T, chunk, anchors)
-    O = chunk_readout(inp["Q"], F, G, chunk, anchors)
+    if bridge:
+        O = bridged_readout(inp["Q"], F, G, inp["alpha"], chunk, anchors)
+    else:
+        O = chunk_readout(inp["Q"], F, G, chunk, anchors)
     out = {"S_T": S_T, "F": F, "G": G, "O": O}
     if "gate" in inp:  # gated RMSNorm epilogue (step (5))
         out["Y"] = gated_rmsnorm(O, inp["norm_w"], inp["gate"], inp.get("eps", 1e-6))
