@@ -61,6 +61,8 @@ def parse():
                     help="time the pass with the readout epilogue (RMSNorm + sigmoid gate, synthetic gates)")
     ap.add_argument("--groups", type=int, default=1,
                     help="head groups of vdn_forward_pipelined (tensor path); 0 = plain vdn_forward")
+    ap.add_argument("--bridge", action="store_true",
+                    help="read through the decay bridge (the window's decay carried onto both states)")
     ap.add_argument("--stream", type=int, default=0,
                     help="time the causal streaming call instead: the clip as a live stream in segments of "
                          "this many frames (a multiple of the chunk; >= T for one segment)")
@@ -220,6 +222,8 @@ def workload_config(w, gated=False):
     gates = "per-token write gates" if w.beta_per_token else "per-frame write gates"
     if gated:
         gates += ", gated RMSNorm readout epilogue"
+    if getattr(w, "decay_bridge", False):
+        gates += ", decay-bridge readout"
     return {"workload": f"{w.name}: B={w.B} H={w.H} T={w.T} U={w.U} d_k=d_v={w.d} n_text={w.n_text} "
                         f"chunk={w.chunk} anchors={w.anchors} {w.dtype} inputs, fp32 state, {gates}",
             "global_batch": w.B, "frames": w.B * w.T, "tokens": w.B * w.T * w.U,
@@ -238,6 +242,8 @@ def main():
         w = dataclasses.replace(w, H=args.heads, name=f"{w.name}_h{args.heads}")
     if args.tokens:
         w = dataclasses.replace(w, U=args.tokens, name=f"{w.name}_u{args.tokens}")
+    if args.bridge:
+        w = dataclasses.replace(w, decay_bridge=True, name=f"{w.name}_bridge")
     if args.impl == "reference":
         return run_reference(args, w)
 

@@ -55,7 +55,7 @@ vdn_status cuda_fail(cudaError_t e, const char *where) {
 
 struct Geo {
   long long BH;
-  int H, T, U, D, C, chunk, anchors, n_text, in_dtype, out_dtype, tokb;
+  int H, T, U, D, C, chunk, anchors, n_text, in_dtype, out_dtype, tokb, bridge;
   size_t in_elem, out_elem;
 };
 
@@ -71,6 +71,7 @@ vdn_status check_shape(const vdn_shape *s, Geo *g) {
   if (s->anchors != 0 && s->anchors != 1) return fail(VDN_ERR_INVALID, "anchors must be 0 or 1");
   if (s->beta_per_token != 0 && s->beta_per_token != 1)
     return fail(VDN_ERR_INVALID, "beta_per_token must be 0 or 1");
+  if (s->decay_bridge != 0 && s->decay_bridge != 1) return fail(VDN_ERR_INVALID, "decay_bridge must be 0 or 1");
   if ((s->in_dtype != VDN_F32 && s->in_dtype != VDN_BF16) ||
       (s->out_dtype != VDN_F32 && s->out_dtype != VDN_BF16))
     return fail(VDN_ERR_INVALID, "dtype must be VDN_F32 or VDN_BF16");
@@ -86,6 +87,7 @@ vdn_status check_shape(const vdn_shape *s, Geo *g) {
   g->in_dtype = s->in_dtype;
   g->out_dtype = s->out_dtype;
   g->tokb = s->beta_per_token;
+  g->bridge = s->decay_bridge;
   g->in_elem = s->in_dtype == VDN_BF16 ? 2 : 4;
   g->out_elem = s->out_dtype == VDN_BF16 ? 2 : 4;
   if (g->BH * (long long)(g->T > 0 ? g->T : 1) > 0x7fffffffLL)
@@ -146,16 +148,19 @@ vdn_status run_grams(const Geo &g, const void *K, const void *V, const float *be
 
 // og: the readout epilogue (step (5)), or nullptr
 // F0: the forward state chunk 0 reads instead of F[0] (streaming), or nullptr
+// alpha: the decay gates when the readout goes through the decay bridge
+// (g.bridge), otherwise ignored.
 vdn_status run_readout(const Geo &g, const void *Q, const float *F, const float *G, void *O,
                        int32_t *info, cudaStream_t st, const OutGate *og = nullptr,
-                       const float *F0 = nullptr) {
+                       const float *F0 = nullptr, const float *alpha = nullptr) {
   if (g.BH * g.T * g.U == 0) return VDN_OK;
+  const float *bridge = g.bridge ? alpha : nullptr;
   if (readout_tc_supported(g.in_dtype, g.out_dtype, g.D, g.U)) {
-    VDN_CUDA(launch_readout_tc(Q, F, G, O, g.BH, g.T, g.U, g.chunk, g.anchors, info, st, og, F0),
+    VDN_CUDA(launch_readout_tc(Q, F, G, O, g.BH, g.T, g.U, g.chunk, g.anchors, info, st, og, F0, bridge),
              "readout_tc");
   } else {
     VDN_CUDA(launch_readout_simt(Q, g.in_dtype, F, G, O, g.out_dtype, g.BH, g.T, g.U, g.chunk,
-                                 g.anchors, g.D, st, og, F0),
+                                 g.anchors, g.D, st, og, F0, bridge),
              "readout_simt");
   }
   return VDN_OK;
@@ -334,6 +339,7 @@ vdn_status vdn_chunk_readout(const vdn_shape *s, const void *Q, const float *F, 
   VDN_TRY(need(F, "F", any));
   VDN_TRY(need(G, "G", any));
   VDN_TRY(need(O, "O", any));
+  if (g.bridge) return fail(VDN_ERR_INVALID, "decay_bridge needs alpha: use vdn_chunk_readout_bridged");
   return run_readout(g, Q, F, G, O, info, (cudaStream_t)stream);
 }
 
@@ -347,10 +353,30 @@ vdn_status vdn_chunk_readout_gated(const vdn_shape *s, const void *Q, const floa
   VDN_TRY(need(F, "F", any));
   VDN_TRY(need(G, "G", any));
   VDN_TRY(need(O, "O", any));
+  if (g.bridge) return fail(VDN_ERR_INVALID, "decay_bridge needs alpha: use vdn_chunk_readout_bridged");
   OutGate og_;
   const OutGate *use;
   VDN_TRY(check_gate(g, og, false, &og_, &use));
   return run_readout(g, Q, F, G, O, info, (cudaStream_t)stream, use);
+}
+
+vdn_status vdn_chunk_readout_bridged(const vdn_shape *s, const void *Q, const float *F, const float *G,
+                                     const float *alpha, const vdn_out_gate *og, void *O, int32_t *info,
+                                     vdn_stream_t stream) {
+  g_err[0] = 0;
+  Geo g;
+  VDN_TRY(check_shape(s, &g));
+  if (!g.bridge) return fail(VDN_ERR_INVALID, "vdn_chunk_readout_bridged needs shape.decay_bridge = 1");
+  const bool any = g.BH * g.T * g.U > 0;
+  VDN_TRY(need(Q, "Q", any));
+  VDN_TRY(need(F, "F", any));
+  VDN_TRY(need(G, "G", any));
+  VDN_TRY(need(alpha, "alpha", any));
+  VDN_TRY(need(O, "O", any));
+  OutGate og_;
+  const OutGate *use;
+  VDN_TRY(check_gate(g, og, true, &og_, &use));
+  return run_readout(g, Q, F, G, O, info, (cudaStream_t)stream, use, nullptr, alpha);
 }
 
 size_t vdn_text_state_workspace_bytes(const vdn_shape *s) {
@@ -525,7 +551,7 @@ vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K, const v
     VDN_CUDA(launch_scan_simt(Mf, Jf, Mb, Jb, S_T, Fo, Go, g.BH, g.C, g.D, 3, st), "scan");
   }
   VDN_TRY(mark(5));
-  if (frames) VDN_TRY(run_readout(g, Q, Fo, Go, O, info, st, gate));
+  if (frames) VDN_TRY(run_readout(g, Q, Fo, Go, O, info, st, gate, nullptr, alpha));
   VDN_TRY(mark(6));
   return VDN_OK;
 }
@@ -541,6 +567,8 @@ vdn_status vdn_stream_segment(const vdn_shape *s, const void *Q, const void *K, 
   VDN_TRY(check_shape(s, &g));
   if (frame0 < 0 || frame0 % g.chunk != 0)
     return fail(VDN_ERR_INVALID, "frame0 = %lld is not a non-negative multiple of chunk = %d", frame0, g.chunk);
+  if (g.bridge)
+    return fail(VDN_ERR_UNSUPPORTED, "decay_bridge: a segment's first chunk would need the previous segment's alpha");
   // only the stream's first frame can be an anchor; there is no last one
   g.anchors = (s->anchors && frame0 == 0) ? 1 : 0;
   const bool frames = g.BH * g.T > 0;
@@ -684,7 +712,7 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
   else if (g.BH > 0)
     VDN_CUDA(launch_scan_simt(nullptr, nullptr, nullptr, nullptr, S_T, Fo, Go, g.BH, g.C, g.D, 3, st), "scan");
   VDN_CUDA(cudaEventRecord(ev(tail + 3), st), "event record");
-  if (frames) VDN_TRY(run_readout(g, Q, Fo, Go, O, info, st, gate));
+  if (frames) VDN_TRY(run_readout(g, Q, Fo, Go, O, info, st, gate, nullptr, alpha));
   VDN_CUDA(cudaEventRecord(ev(tail + 4), st), "event record");
   return VDN_OK;
 }

@@ -35,10 +35,12 @@ struct OutGate {
 };
 // R_c = F[max(c - 1, 0)] + G[min(c + 2, C)]; G may be null (forward reads
 // only) and F0 ([BH, d, d], may be null) replaces F[0] for chunk 0.
+// bridge_alpha ([BH, T, d], may be null): read through the decay bridge,
+// R_t = F[max(c - 1, 0)] Diag(pf_t) + G[min(c + 2, C)] Diag(pb_t).
 cudaError_t launch_readout_simt(const void *Q, int in_dtype, const float *F, const float *G, void *O,
                                 int out_dtype, long long BH, int T, int U, int chunk, int anchors,
                                 int D, cudaStream_t st, const OutGate *og = nullptr,
-                                const float *F0 = nullptr);
+                                const float *F0 = nullptr, const float *bridge_alpha = nullptr);
 
 // Tensor-core kernels (tcgen05 + TMA), bf16 inputs, d = 128.
 bool gram_tc_supported(int in_dtype, int D, int U);
@@ -52,7 +54,8 @@ cudaError_t launch_gram_tc(const void *K, const void *V, const float *beta, bool
 bool readout_tc_supported(int in_dtype, int out_dtype, int D, int U);
 cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, void *O, long long BH,
                               int T, int U, int chunk, int anchors, int32_t *info, cudaStream_t st,
-                              const OutGate *og = nullptr, const float *F0 = nullptr);
+                              const OutGate *og = nullptr, const float *F0 = nullptr,
+                              const float *bridge_alpha = nullptr);
 
 // W = (I + A)^{-1} per frame (CUDA cores); W fp32 and/or Wimg (hi/lo MMA
 // images of kImgBytes per frame, d = 128 only), each optional.

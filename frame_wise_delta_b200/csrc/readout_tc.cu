@@ -17,6 +17,11 @@
 // over the token's TMEM row (mean square, then scale), with the tile's gate
 // logits brought by TMA into the staging tile that then receives y.
 //
+// Decay bridge (optional, step (5)): frame t reads
+//   R_t = F[max(c-1,0)] Diag(pf_t) + G[min(c+2,C)] Diag(pb_t),
+// pf_t and pb_t the products of the decay gates over the window's frames
+// f0..t and t..f1; R is then rebuilt for every frame.
+//
 // Persistent kernel, one CTA per SM, 10 warps; each CTA walks a contiguous
 // range of frames so consecutive frames usually share a chunk and R is
 // rebuilt only when the chunk changes.
@@ -53,6 +58,7 @@ struct ReadoutArgs {
   const float *F;
   const float *G;   // optional (forward reads only when null)
   const float *F0;  // optional: per-b*h forward state chunk 0 reads instead of F[0]
+  const float *bal; // optional: decay gates alpha [BH, T, 128]: read through the decay bridge
   __nv_bfloat16 *O;
   int32_t *info;
   long long nframes;
@@ -73,8 +79,9 @@ __device__ __forceinline__ bool is_anchor(const ReadoutArgs &p, long long f) {
   return ((p.anchors & 1) && t == 0) || ((p.anchors & 2) && t == p.T - 1);
 }
 
+// R changes with the chunk, or with every frame through the decay bridge
 __device__ __forceinline__ long long chunk_key(const ReadoutArgs &p, long long f) {
-  return (f / p.T) * p.C + (f % p.T) / p.chunk;
+  return p.bal ? f : (f / p.T) * p.C + (f % p.T) / p.chunk;
 }
 
 // tanh by the hardware approximation (PTX tanh.approx.f32, ~2^-11 relative)
@@ -262,6 +269,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float *Fs = (c == 0 && p.F0) ? p.F0 + bh * (long long)(kD * kD)
                                            : p.F + (bh * (p.C + 1) + max(c - 1, 0)) * (long long)(kD * kD);
         const float *Gs = p.G ? p.G + (bh * (p.C + 1) + min(c + 2, p.C)) * (long long)(kD * kD) : nullptr;
+        // decay bridge: this thread's 8 key channels k0.. (fixed over the
+        // loop below) scale F by prod alpha over the window's frames f0..t
+        // and G over t..f1; anchor frames count as 1
+        float pf[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f}, pb[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+        if (p.bal) {
+          const int t = (int)(f % p.T), k0 = (et & 15) * 8;
+          const int f0 = p.chunk * max(c - 1, 0), f1 = min(p.chunk * (c + 2), p.T) - 1;
+          const float *al = p.bal + bh * (long long)p.T * kD + k0;
+          for (int r = f0; r <= f1; ++r) {
+            if (((p.anchors & 1) && r == 0) || ((p.anchors & 2) && r == p.T - 1)) continue;
+            const float4 x0 = *reinterpret_cast<const float4 *>(al + (long long)r * kD);
+            const float4 x1 = *reinterpret_cast<const float4 *>(al + (long long)r * kD + 4);
+            const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              if (r <= t) pf[q] *= x[q];
+              if (r >= t) pb[q] *= x[q];
+            }
+          }
+        }
         for (int e8 = et; e8 < kD * kD / 8; e8 += 256) {
           const int i = e8 >> 4, k0 = (e8 & 15) * 8;
           const float4 *f4 = reinterpret_cast<const float4 *>(Fs + i * kD + k0);
@@ -272,8 +299,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             b0 = g4[0];
             b1 = g4[1];
           }
-          const float r[8] = {a0.x + b0.x, a0.y + b0.y, a0.z + b0.z, a0.w + b0.w,
-                              a1.x + b1.x, a1.y + b1.y, a1.z + b1.z, a1.w + b1.w};
+          float r[8];
+          if (p.bal) {
+            const float fa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float ga[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int q = 0; q < 8; ++q) r[q] = fmaf(fa[q], pf[q], ga[q] * pb[q]);
+          } else {
+            r[0] = a0.x + b0.x, r[1] = a0.y + b0.y, r[2] = a0.z + b0.z, r[3] = a0.w + b0.w;
+            r[4] = a1.x + b1.x, r[5] = a1.y + b1.y, r[6] = a1.z + b1.z, r[7] = a1.w + b1.w;
+          }
           uint4 h, l;
           split_bf16x2(r[0], r[1], h.x, l.x);
           split_bf16x2(r[2], r[3], h.y, l.y);
@@ -414,7 +449,7 @@ bool readout_tc_supported(int in_dtype, int out_dtype, int D, int U) {
 
 cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, void *O, long long BH,
                               int T, int U, int chunk, int anchors, int32_t *info, cudaStream_t st,
-                              const OutGate *og, const float *F0) {
+                              const OutGate *og, const float *F0, const float *bridge_alpha) {
   const long long nframes = BH * T;
   if (nframes <= 0) return cudaSuccess;
   CUtensorMap tmQ, tmO, tmG;
@@ -427,7 +462,7 @@ cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, voi
   if (e != cudaSuccess) return e;
   const int sms = device_sm_count();
   const long long grid = nframes < sms ? nframes : sms;
-  ReadoutArgs a{F, G, F0, (__nv_bfloat16 *)O, info, nframes, T, U, chunk, anchors,
+  ReadoutArgs a{F, G, F0, bridge_alpha, (__nv_bfloat16 *)O, info, nframes, T, U, chunk, anchors,
                 (T + chunk - 1) / chunk, (U + kNT - 1) / kNT,
                 gated ? og->w : nullptr, gated ? og->eps : 0.f, gated ? og->H : 1};
   readout_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(tmQ, tmO, tmG, a);

@@ -336,18 +336,23 @@ __global__ void __launch_bounds__(kThreads) scan_simt_kernel(
 
 // --------------------------------------------------------------- readout
 // One block per (frame, 64-token tile). R_c = F[max(c-1,0)] + G[min(c+2,C)]
-// is staged transposed (padded) in smem, the query tile as float32.
+// is staged transposed (padded) in smem, the query tile as float32. With the
+// decay bridge (bal = the decay gates alpha [BH, T, D]) frame t reads
+// R_t = F[max(c-1,0)] Diag(pf) + G[min(c+2,C)] Diag(pb), pf and pb the
+// products of alpha over the window's frames f0..t and t..f1 (anchor frames
+// count as 1), formed per channel in smem first.
 template <int D, typename Tin, typename Tout>
 __global__ void __launch_bounds__(kThreads) readout_simt_kernel(
     const Tin *__restrict__ Q, const float *__restrict__ F, const float *__restrict__ G,
     Tout *__restrict__ O, int T, int U, int chunk, int anchors, int C, OutGate og,
-    const float *__restrict__ F0) {
+    const float *__restrict__ F0, const float *__restrict__ bal) {
   constexpr int TU = 64;
   constexpr int RB = D / 16;
   constexpr int LD = D + 1;
   extern __shared__ __align__(16) float sm[];
   float *Rt = sm;            // [D][LD] : Rt[k][i] = R[i][k]
   float *Qs = sm + D * LD;   // [TU][D]
+  float *pfb = Qs + TU * D;  // [2][D] bridge factors pf, pb
   const long long f = blockIdx.x;
   const int u0 = blockIdx.y * TU;
   const long long bh = f / T;
@@ -366,9 +371,28 @@ __global__ void __launch_bounds__(kThreads) readout_simt_kernel(
   const int c = t / chunk;
   const float *Fs = (c == 0 && F0) ? F0 + bh * DD : F + (bh * (C + 1) + max(c - 1, 0)) * DD;
   const float *Gs = G ? G + (bh * (C + 1) + min(c + 2, C)) * DD : nullptr;
-  for (int e = threadIdx.x; e < D * D; e += kThreads) {
-    const int i = e / D, k = e % D;
-    Rt[k * LD + i] = Fs[e] + (Gs ? Gs[e] : 0.f);
+  if (bal) {
+    const int f0 = chunk * max(c - 1, 0), f1 = min(chunk * (c + 2), T) - 1;
+    for (int k = threadIdx.x; k < D; k += kThreads) {
+      const float *al = bal + bh * (long long)T * D + k;
+      float pf = 1.f, pb = 1.f;
+      for (int r = f0; r <= t; ++r)
+        if (!(((anchors & 1) && r == 0) || ((anchors & 2) && r == T - 1))) pf *= al[(long long)r * D];
+      for (int r = t; r <= f1; ++r)
+        if (!(((anchors & 1) && r == 0) || ((anchors & 2) && r == T - 1))) pb *= al[(long long)r * D];
+      pfb[k] = pf;
+      pfb[D + k] = pb;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < D * D; e += kThreads) {
+      const int i = e / D, k = e % D;
+      Rt[k * LD + i] = fmaf(Fs[e], pfb[k], Gs ? Gs[e] * pfb[D + k] : 0.f);
+    }
+  } else {
+    for (int e = threadIdx.x; e < D * D; e += kThreads) {
+      const int i = e / D, k = e % D;
+      Rt[k * LD + i] = Fs[e] + (Gs ? Gs[e] : 0.f);
+    }
   }
   const Tin *Qf = Q + f * (long long)U * D;
   for (int e = threadIdx.x; e < TU * D; e += kThreads) {
@@ -466,30 +490,31 @@ cudaError_t scan_d(const float *Mf, const float *Jf, const float *Mb, const floa
 
 template <int D, typename Tin, typename Tout>
 cudaError_t readout_dt(const void *Q, const float *F, const float *G, void *O, long long BH, int T,
-                       int U, int chunk, int anchors, cudaStream_t st, const OutGate &og, const float *F0) {
+                       int U, int chunk, int anchors, cudaStream_t st, const OutGate &og, const float *F0,
+                       const float *bal) {
   const int C = (T + chunk - 1) / chunk;
-  const size_t smem = (size_t)(D * (D + 1) + 64 * D) * sizeof(float);
+  const size_t smem = (size_t)(D * (D + 1) + 64 * D + 2 * D) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(readout_simt_kernel<D, Tin, Tout>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)(BH * T), (unsigned)((U + 63) / 64));
   readout_simt_kernel<D, Tin, Tout><<<grid, kThreads, smem, st>>>(
-      (const Tin *)Q, F, G, (Tout *)O, T, U, chunk, anchors, C, og, F0);
+      (const Tin *)Q, F, G, (Tout *)O, T, U, chunk, anchors, C, og, F0, bal);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t readout_d(const void *Q, int in_dtype, const float *F, const float *G, void *O,
                       int out_dtype, long long BH, int T, int U, int chunk, int anchors,
-                      cudaStream_t st, const OutGate &og, const float *F0) {
+                      cudaStream_t st, const OutGate &og, const float *F0, const float *bal) {
   if (in_dtype == VDN_BF16) {
     if (out_dtype == VDN_BF16)
-      return readout_dt<D, __nv_bfloat16, __nv_bfloat16>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0);
-    return readout_dt<D, __nv_bfloat16, float>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0);
+      return readout_dt<D, __nv_bfloat16, __nv_bfloat16>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0, bal);
+    return readout_dt<D, __nv_bfloat16, float>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0, bal);
   }
   if (out_dtype == VDN_BF16)
-    return readout_dt<D, float, __nv_bfloat16>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0);
-  return readout_dt<D, float, float>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0);
+    return readout_dt<D, float, __nv_bfloat16>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0, bal);
+  return readout_dt<D, float, float>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0, bal);
 }
 
 }  // namespace
@@ -538,11 +563,13 @@ cudaError_t launch_scan_simt(const float *Mf, const float *Jf, const float *Mb, 
 
 cudaError_t launch_readout_simt(const void *Q, int in_dtype, const float *F, const float *G, void *O,
                                 int out_dtype, long long BH, int T, int U, int chunk, int anchors,
-                                int D, cudaStream_t st, const OutGate *og, const float *F0) {
+                                int D, cudaStream_t st, const OutGate *og, const float *F0,
+                                const float *bridge_alpha) {
   if (BH <= 0 || T <= 0 || U <= 0) return cudaSuccess;
   const OutGate none{nullptr, nullptr, 0.f, 1};
   const OutGate &g = og ? *og : none;
-  VDN_DISPATCH_D(D, readout_d<DD_>(Q, in_dtype, F, G, O, out_dtype, BH, T, U, chunk, anchors, st, g, F0))
+  VDN_DISPATCH_D(D, readout_d<DD_>(Q, in_dtype, F, G, O, out_dtype, BH, T, U, chunk, anchors, st, g, F0,
+                                   bridge_alpha))
 }
 
 }  // namespace vdn

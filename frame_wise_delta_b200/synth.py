@@ -41,6 +41,8 @@ class Workload:
     near_dup: keys of a frame cluster around a few prototypes (cosine 0.99).
     beta_per_token: one write gate per token, beta [T, U] and beta_x
     [n_text] ~ U(beta_lo, 1); otherwise beta [T] per frame and beta_x = 1.
+    decay_bridge: the readout goes through the decay bridge (changes no
+    input; carried so that a workload names the whole computation).
     """
 
     name: str
@@ -58,6 +60,7 @@ class Workload:
     chunk: int = 5
     beta_lo: float = 0.1
     beta_per_token: bool = False
+    decay_bridge: bool = False
 
     @property
     def seed(self) -> int:

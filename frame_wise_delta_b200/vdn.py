@@ -34,7 +34,7 @@ class VdnError(RuntimeError):
 class vdn_shape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("B", "H", "T", "U", "dk", "dv", "n_text", "chunk", "anchors", "in_dtype", "out_dtype",
-                 "beta_per_token")]
+                 "beta_per_token", "decay_bridge")]
 
     @property
     def C(self) -> int:
@@ -42,16 +42,18 @@ class vdn_shape(ctypes.Structure):
 
 
 def make_shape(B, H, T, U, d, n_text, chunk=5, anchors=0, in_dtype="bf16", out_dtype=None,
-               beta_per_token=False) -> vdn_shape:
+               beta_per_token=False, decay_bridge=False) -> vdn_shape:
     in_dt = _DTYPES[in_dtype]
     out_dt = in_dt if out_dtype is None else _DTYPES[out_dtype]
-    return vdn_shape(B, H, T, U, d, d, n_text, chunk, anchors, in_dt, out_dt, int(bool(beta_per_token)))
+    return vdn_shape(B, H, T, U, d, d, n_text, chunk, anchors, in_dt, out_dt, int(bool(beta_per_token)),
+                     int(bool(decay_bridge)))
 
 
 def shape_for(w, B=None, H=None) -> vdn_shape:
     """Shape of a synth.Workload (optionally with other batch/head counts)."""
     return make_shape(w.B if B is None else B, w.H if H is None else H, w.T, w.U, w.d, w.n_text,
-                      w.chunk, w.anchors, w.dtype, beta_per_token=w.beta_per_token)
+                      w.chunk, w.anchors, w.dtype, beta_per_token=w.beta_per_token,
+                      decay_bridge=getattr(w, "decay_bridge", False))
 
 
 class vdn_out_gate(ctypes.Structure):
@@ -86,6 +88,7 @@ _SIGS = {
     "vdn_text_state_noalloc": [_P, _P, _P, _P, _P, _P, _P],
     "vdn_forward_pipelined": [_P] * 13 + [ctypes.c_size_t, _P, ctypes.c_int32, _P, _P, _P, _P],
     "vdn_chunk_readout_gated": [_P] * 8,
+    "vdn_chunk_readout_bridged": [_P] * 9,
     "vdn_stream_segment": [_P] * 6 + [ctypes.c_longlong] + [_P] * 5 + [ctypes.c_size_t, _P, _P],
 }
 
@@ -257,6 +260,12 @@ def vdn_forward_pipelined(s, Q, K, V, beta, alpha, Kx, Vx, beta_x, O, F, G, work
 def vdn_chunk_readout_gated(s, Q, F, G, og, O, info=None, stream=None):
     _check(lib().vdn_chunk_readout_gated(_shp(s), _ptr(Q), _ptr(F), _ptr(G), _og(og), _ptr(O), _ptr(info),
                                          _stream(stream)))
+
+
+def vdn_chunk_readout_bridged(s, Q, F, G, alpha, og, O, info=None, stream=None):
+    """The chunk readout through the decay bridge (shape.decay_bridge = 1); og may be None."""
+    _check(lib().vdn_chunk_readout_bridged(_shp(s), _ptr(Q), _ptr(F), _ptr(G), _ptr(alpha), _og(og), _ptr(O),
+                                           _ptr(info), _stream(stream)))
 
 
 def vdn_stream_workspace_bytes(s) -> int:

@@ -77,6 +77,18 @@ typedef struct {
                              beta_x [B,H]; 1: one per token ("Core method":
                              beta_{t,u}), beta [B,H,T,U] and beta_x
                              [B,H,n_text] */
+  int32_t decay_bridge;   /* 0: frame t of chunk c reads R_c = F[max(c-1,0)]
+                             + G[min(c+2,C)]; 1: the readout goes through the
+                             decay bridge ("Method steps" step (5)):
+                               R_t = F[max(c-1,0)] Diag(pf_t)
+                                   + G[min(c+2,C)] Diag(pb_t),
+                             pf_t = prod_{r=f0..t} alpha_r, pb_t =
+                             prod_{r=t..f1} alpha_r over the window's frames
+                             (f0 = chunk*max(c-1,0), f1 = min(chunk*(c+2),T)-1;
+                             an anchor frame's alpha counts as 1): the states
+                             outside the window carried to frame t through
+                             the decay of the window's frames, whose writes
+                             the softmax branch holds */
 } vdn_shape;
 
 /*
@@ -185,6 +197,9 @@ vdn_status vdn_scan_bidir(const vdn_shape *s, const float *Mf, const float *Jf,
 vdn_status vdn_chunk_readout(const vdn_shape *s, const void *Q, const float *F,
                              const float *G, void *O, int32_t *info,
                              vdn_stream_t stream);
+/* (vdn_chunk_readout and vdn_chunk_readout_gated take no alpha: with
+ * shape.decay_bridge = 1 they return VDN_ERR_INVALID; use
+ * vdn_chunk_readout_bridged.) */
 
 /*
  * Readout epilogue. Paper: "Method steps", step (5) ("after the readout,
@@ -208,6 +223,22 @@ typedef struct {
 vdn_status vdn_chunk_readout_gated(const vdn_shape *s, const void *Q, const float *F,
                                    const float *G, const vdn_out_gate *og, void *O,
                                    int32_t *info, vdn_stream_t stream);
+
+/*
+ * Chunk readout through the decay bridge (shape.decay_bridge = 1; see the
+ * field's comment for R_t). Paper: "Method steps" step (5) (the states at the
+ * window boundary continue through the decay bridge prod alpha_r before the
+ * readout) and "Core method" (the frame recurrence Sbar_t = S_{t-1}
+ * Diag(alpha_t)). In : Q, F, G as for vdn_chunk_readout; alpha [B,H,T,dk]
+ * float32 (the decay gates of the scans). og: NULL, or the readout epilogue
+ * as for vdn_chunk_readout_gated. Out: O [B,H,T,U,dv] (out_dtype), anchor
+ * rows 0. Errors as for vdn_chunk_readout_gated, plus VDN_ERR_INVALID when
+ * shape.decay_bridge is 0 or alpha is NULL/misaligned.
+ */
+vdn_status vdn_chunk_readout_bridged(const vdn_shape *s, const void *Q, const float *F,
+                                     const float *G, const float *alpha,
+                                     const vdn_out_gate *og, void *O, int32_t *info,
+                                     vdn_stream_t stream);
 
 /*
  * Text state. Paper: "Core method" (the text prompt is summarised into a text
@@ -265,6 +296,8 @@ vdn_status vdn_text_state_noalloc(const vdn_shape *s, const void *Kx,
  * shapes use the CUDA-core kernels of the stage calls above.
  * og: NULL for O as read out, or the readout epilogue of
  *      vdn_chunk_readout_gated (O then holds y).
+ * With shape.decay_bridge the readout goes through the decay bridge, as
+ * vdn_chunk_readout_bridged with this call's alpha.
  */
 size_t vdn_forward_workspace_bytes(const vdn_shape *s);
 vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K,
@@ -328,7 +361,9 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
  *      S_in = F[C]. *info as for vdn_frame_factor.
  * workspace: at least vdn_stream_workspace_bytes(s) bytes, 256-byte aligned.
  * Errors: VDN_ERR_INVALID for a frame0 that is negative or not a multiple of
- * the chunk, and as for vdn_forward. Same kernels as vdn_forward (the
+ * the chunk, and as for vdn_forward; VDN_ERR_UNSUPPORTED with
+ * shape.decay_bridge (the bridge of a segment's first chunk would need the
+ * previous segment's decay gates). Same kernels as vdn_forward (the
  * tensor-core path for bf16 d = 128), run in one direction.
  */
 size_t vdn_stream_workspace_bytes(const vdn_shape *s);
