@@ -52,7 +52,8 @@ constexpr int kAcc = 4;                       // TMEM accumulators (128 columns 
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBarBytes = 8 * (2 * kStages + 2 * kAcc + 2 + 2);
-constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + 2 * kRBytes + 2 * kOBytes + kBarBytes + 16;
+constexpr size_t kSmemBytes =
+    1024 + (size_t)kStages * kStageBytes + 2 * kRBytes + 2 * kOBytes + kBarBytes + 16 + 2 * kD * 4;
 
 struct ReadoutArgs {
   const float *F;
@@ -109,6 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *bars = reinterpret_cast<uint64_t *>(Obuf + 2 * kOBytes);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(bars) + kBarBytes);
   volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  float *bridge_fb = reinterpret_cast<float *>(tmem_slot + 4);  // [2][128]: pf, pb of the frame being read
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t full0 = smem_u32(bars);
@@ -269,54 +271,68 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float *Fs = (c == 0 && p.F0) ? p.F0 + bh * (long long)(kD * kD)
                                            : p.F + (bh * (p.C + 1) + max(c - 1, 0)) * (long long)(kD * kD);
         const float *Gs = p.G ? p.G + (bh * (p.C + 1) + min(c + 2, p.C)) * (long long)(kD * kD) : nullptr;
-        // decay bridge: this thread's 8 key channels k0.. (fixed over the
-        // loop below) scale F by prod alpha over the window's frames f0..t
-        // and G over t..f1; anchor frames count as 1
-        float pf[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f}, pb[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+        // decay bridge: thread et forms the factor of key channel et & 127,
+        // forward (pf, the window's frames f0..t) or backward (pb, t..f1),
+        // anchor frames counting as 1; the products go through shared memory
         if (p.bal) {
-          const int t = (int)(f % p.T), k0 = (et & 15) * 8;
-          const int f0 = p.chunk * max(c - 1, 0), f1 = min(p.chunk * (c + 2), p.T) - 1;
-          const float *al = p.bal + bh * (long long)p.T * kD + k0;
-          for (int r = f0; r <= f1; ++r) {
-            if (((p.anchors & 1) && r == 0) || ((p.anchors & 2) && r == p.T - 1)) continue;
-            const float4 x0 = *reinterpret_cast<const float4 *>(al + (long long)r * kD);
-            const float4 x1 = *reinterpret_cast<const float4 *>(al + (long long)r * kD + 4);
-            const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+          const int t = (int)(f % p.T), k = et & 127, dir = et >> 7;
+          const int lo = dir ? t : p.chunk * max(c - 1, 0);
+          const int hi = dir ? min(p.chunk * (c + 2), p.T) - 1 : t;
+          const float *al = p.bal + bh * (long long)p.T * kD + k;
+          float prod = 1.f;
+#pragma unroll 8
+          for (int r = lo; r <= hi; ++r) {
+            const float x = __ldg(al + (long long)r * kD);
+            if (!(((p.anchors & 1) && r == 0) || ((p.anchors & 2) && r == p.T - 1))) prod *= x;
+          }
+          bridge_fb[dir * kD + k] = prod;
+          asm volatile("bar.sync 3, 256;" ::: "memory");
+        }
+        // R (or R_t) as hi/lo bf16 operand images; each thread covers 8 key
+        // channels k0.. of 8 rows, the loads of four rows in flight at once
+        const int k0 = (et & 15) * 8;
+        float pf[8], pb[8];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              if (r <= t) pf[q] *= x[q];
-              if (r >= t) pb[q] *= x[q];
+        for (int q = 0; q < 8; ++q) {
+          pf[q] = p.bal ? bridge_fb[k0 + q] : 1.f;
+          pb[q] = p.bal ? bridge_fb[kD + k0 + q] : 1.f;
+        }
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          float4 fa[4][2], ga[4][2];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int i = (et + 256 * (4 * half + j)) >> 4;
+            const float4 *f4 = reinterpret_cast<const float4 *>(Fs + i * kD + k0);
+            fa[j][0] = __ldg(f4);
+            fa[j][1] = __ldg(f4 + 1);
+            if (Gs) {
+              const float4 *g4 = reinterpret_cast<const float4 *>(Gs + i * kD + k0);
+              ga[j][0] = __ldg(g4);
+              ga[j][1] = __ldg(g4 + 1);
+            } else {
+              ga[j][0] = ga[j][1] = make_float4(0.f, 0.f, 0.f, 0.f);
             }
           }
-        }
-        for (int e8 = et; e8 < kD * kD / 8; e8 += 256) {
-          const int i = e8 >> 4, k0 = (e8 & 15) * 8;
-          const float4 *f4 = reinterpret_cast<const float4 *>(Fs + i * kD + k0);
-          const float4 a0 = f4[0], a1 = f4[1];
-          float4 b0 = make_float4(0.f, 0.f, 0.f, 0.f), b1 = b0;
-          if (Gs) {
-            const float4 *g4 = reinterpret_cast<const float4 *>(Gs + i * kD + k0);
-            b0 = g4[0];
-            b1 = g4[1];
-          }
-          float r[8];
-          if (p.bal) {
-            const float fa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            const float ga[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-            for (int q = 0; q < 8; ++q) r[q] = fmaf(fa[q], pf[q], ga[q] * pb[q]);
-          } else {
-            r[0] = a0.x + b0.x, r[1] = a0.y + b0.y, r[2] = a0.z + b0.z, r[3] = a0.w + b0.w;
-            r[4] = a1.x + b1.x, r[5] = a1.y + b1.y, r[6] = a1.z + b1.z, r[7] = a1.w + b1.w;
+          for (int j = 0; j < 4; ++j) {
+            const int i = (et + 256 * (4 * half + j)) >> 4;
+            const float x[8] = {fa[j][0].x, fa[j][0].y, fa[j][0].z, fa[j][0].w,
+                                fa[j][1].x, fa[j][1].y, fa[j][1].z, fa[j][1].w};
+            const float y[8] = {ga[j][0].x, ga[j][0].y, ga[j][0].z, ga[j][0].w,
+                                ga[j][1].x, ga[j][1].y, ga[j][1].z, ga[j][1].w};
+            float r[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) r[q] = p.bal ? fmaf(x[q], pf[q], y[q] * pb[q]) : x[q] + y[q];
+            uint4 h, l;
+            split_bf16x2(r[0], r[1], h.x, l.x);
+            split_bf16x2(r[2], r[3], h.y, l.y);
+            split_bf16x2(r[4], r[5], h.z, l.z);
+            split_bf16x2(r[6], r[7], h.w, l.w);
+            const uint32_t off = kmajor_sw128_offset(i, k0, kD);
+            *reinterpret_cast<uint4 *>(Rhi + off) = h;
+            *reinterpret_cast<uint4 *>(Rlo + off) = l;
           }
-          uint4 h, l;
-          split_bf16x2(r[0], r[1], h.x, l.x);
-          split_bf16x2(r[2], r[3], h.y, l.y);
-          split_bf16x2(r[4], r[5], h.z, l.z);
-          split_bf16x2(r[6], r[7], h.w, l.w);
-          const uint32_t off = kmajor_sw128_offset(i, k0, kD);
-          *reinterpret_cast<uint4 *>(Rhi + off) = h;
-          *reinterpret_cast<uint4 *>(Rlo + off) = l;
         }
         fence_proxy_async_smem();
         asm volatile("bar.sync 3, 256;" ::: "memory");
