@@ -39,8 +39,8 @@ NCU_TRAFFIC = {
                     "sha256_16": "00240b7db02fd61b", "workload": "h3"},
     "frame_factor": {"bytes": 126.3e6 + 102.9e6, "source": "frame_wise_delta_b200/csrc/invert_tc.cu",
                      "sha256_16": "d4085e639e7135a8", "workload": "h3"},
-    "chunk_readout": {"bytes": 700.7e6 + 581.7e6, "source": "frame_wise_delta_b200/csrc/readout_tc.cu",
-                      "sha256_16": "c1b3db4af3bc6542", "workload": "h3"},
+    "chunk_readout": {"bytes": 700.8e6 + 581.3e6, "source": "frame_wise_delta_b200/csrc/readout_tc.cu",
+                      "sha256_16": "9a564eca14ecfc6e", "workload": "h3"},
 }
 
 

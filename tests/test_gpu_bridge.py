@@ -148,3 +148,23 @@ def test_argument_checks():
     with pytest.raises(vdn.VdnError) as e:
         vdn.vdn_stream_segment(s, dev["Q"], dev["K"], dev["V"], dev["beta"], dev["alpha"], 0, S, S, O, F, ws, info)
     assert e.value.status == vdn.VDN_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("T", [1, 2, 4, 6, 11])
+@pytest.mark.parametrize("d,dtype", [(128, "bf16"), (32, "f32")], ids=["tc", "f32"])
+def test_short_clips(T, d, dtype):
+    """Clips of one to three chunks, where every window reaches both ends
+    (and with T = 1, 2 every frame is an anchor)."""
+    w = custom(f"bridge_T{T}_{dtype}", index=94, T=T, d=d, dtype=dtype, U=70, n_text=7)
+    full = synth.generate_all(w)
+    dev = device_inputs(w, full)
+    fw = vdn.Forward(vdn.shape_for(w))
+    fw(dev["Q"], dev["K"], dev["V"], dev["beta"], dev["alpha"], dev["Kx"], dev["Vx"], dev["beta_x"])
+    torch.cuda.synchronize()
+    assert int(fw.info.item()) == 0
+    for (b, h), r in _heads(w, full).items():
+        eo = rel(fw.O[b, h], r["O"])
+        print(f"T={T} {dtype} b{b} h{h}: O {eo:.2e}")
+        assert eo <= TOL[dtype]
+        if T <= 2:
+            assert torch.count_nonzero(fw.O[b, h]) == 0
