@@ -20,6 +20,14 @@
 
 namespace vdn {
 
+// Reciprocal by the hardware approximation (PTX rcp.approx.ftz.f32, about
+// one ulp): the pivot reciprocal sits on the sweep's step-to-step critical path.
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 constexpr int kSweepGrid = 8;
 constexpr int kSweepThreads = kSweepGrid * kSweepGrid;  // 64
 
@@ -63,7 +71,7 @@ struct Sweep {
         sync();
         const float piv = c[kr * R + kb];
         bad |= !(piv > 0.f) || !isfinite(piv);
-        const float rp = __frcp_rn(piv);
+        const float rp = rcp_approx(piv);
         // c_i for this thread's rows is read from shared memory where it is used
         const float *ci = &c[rg * R];
         float2 cj2[P];  // c_j / piv for this thread's columns, as pairs
@@ -134,7 +142,7 @@ struct Sweep {
         const float p00 = c0[kr * R + kb], p01 = c0[(kr + 1) * R + kb], p11 = c1[(kr + 1) * R + kb];
         const float det = fmaf(p00, p11, -p01 * p01);
         bad |= !(p00 > 0.f) || !(det > 0.f) || !isfinite(p00) || !isfinite(det);
-        const float rd = __frcp_rn(det);
+        const float rd = rcp_approx(det);
         const float q00 = p11 * rd, q01 = -p01 * rd, q11 = p00 * rd;  // G_KK^{-1}
         const float *ci0 = &c0[rg * R], *ci1 = &c1[rg * R];
         // e_j = G_KK^{-1} (c0_j, c1_j) for this thread's columns, as pairs
