@@ -181,8 +181,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *pi_t = sm + kSlotPi, *s0 = sm + kSlotS0, *xt = sm + kSlotXT;
-  float(*cbuf)[64] = reinterpret_cast<float(*)[64]>(sm + kSlotMisc);         // single-pivot sweeps
-  float(*cbuf2)[2][64] = reinterpret_cast<float(*)[2][64]>(sm + kSlotMisc);  // pivot-pair sweeps
+  float(*cbuf)[64] = reinterpret_cast<float(*)[64]>(sm + kSlotMisc);  // sweep exchange buffer
   uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kSlotMisc + 1024);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kSlotMisc + 1032);
   volatile int *abort = reinterpret_cast<volatile int *>(sm + kSlotMisc + 1036);
@@ -249,10 +248,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           const int r = rg + kSweepGrid * a, c = cg + kSweepGrid * b;
           X.at(a, b) -= stage[r * 64 + (((c >> 2) ^ (r & 15)) << 2) + (c & 3)];
         }
-      if constexpr (PRE_P)
-        ok = X.run2(cbuf2, rg, cg, [] { bar_named(kBarSweep); }) && ok;
-      else
-        ok = X.run(cbuf, rg, cg, [] { bar_named(kBarSweep); }) && ok;
+      ok = X.run(cbuf, rg, cg, [] { bar_named(kBarSweep); }) && ok;
       store_swept_tile(X, s0, rg, cg);
       fence_proxy_async_smem();
       handoff_arrive(kBarSiReady);
