@@ -37,8 +37,8 @@ ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 NCU_TRAFFIC = {
     "frame_grams": {"bytes": 1291.9e6 + 253.8e6, "source": "frame_wise_delta_b200/csrc/gram_tc.cu",
                     "sha256_16": "00240b7db02fd61b", "workload": "h3"},
-    "frame_factor": {"bytes": 126.3e6 + 102.9e6, "source": "frame_wise_delta_b200/csrc/invert_tc.cu",
-                     "sha256_16": "d4085e639e7135a8", "workload": "h3"},
+    "frame_factor": {"bytes": 122.8e6 + 101.2e6, "source": "frame_wise_delta_b200/csrc/invert_tc.cu",
+                     "sha256_16": "d93dd215a7ca697f", "workload": "h3"},
     "chunk_readout": {"bytes": 700.8e6 + 581.3e6, "source": "frame_wise_delta_b200/csrc/readout_tc.cu",
                       "sha256_16": "9a564eca14ecfc6e", "workload": "h3"},
 }
