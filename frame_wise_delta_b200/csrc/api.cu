@@ -222,6 +222,21 @@ vdn_status run_text_state(const Geo &g, const void *Kx, const void *Vx, const fl
   return VDN_OK;
 }
 
+// One CTA waits on a barrier that nothing arrives at: the bounded wait gives
+// up after its limit and the kernel reports the timeout in *info.
+__global__ void wait_selftest_kernel(int32_t *info) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const bool ok = mbar_wait(smem_u32(&bar), 0, &abort);
+  if (!__all_sync(0xffffffffu, ok) && threadIdx.x == 0) atomicExch(info, VDN_INFO_TIMEOUT);
+}
+
 }  // namespace
 
 void vdn::set_last_error(const char *msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
@@ -242,6 +257,16 @@ const char *vdn_status_string(vdn_status st) {
 const char *vdn_last_error(void) { return g_err; }
 
 int32_t vdn_version(void) { return 100; }
+
+vdn_status vdn_selftest_wait(int32_t *info, vdn_stream_t stream) {
+  g_err[0] = 0;
+  VDN_TRY(need(info, "info", true));
+  cudaStream_t st = (cudaStream_t)stream;
+  VDN_CUDA(cudaMemsetAsync(info, 0, sizeof(int32_t), st), "memset info");
+  wait_selftest_kernel<<<1, 32, 0, st>>>(info);
+  VDN_CUDA(cudaGetLastError(), "selftest wait");
+  return VDN_OK;
+}
 
 vdn_status vdn_frame_grams(const vdn_shape *s, const void *K, const void *V, const float *beta,
                            float *A, float *Bm, int32_t *info, vdn_stream_t stream) {

@@ -89,6 +89,7 @@ _SIGS = {
     "vdn_forward_pipelined": [_P] * 13 + [ctypes.c_size_t, _P, ctypes.c_int32, _P, _P, _P, _P],
     "vdn_chunk_readout_gated": [_P] * 8,
     "vdn_chunk_readout_bridged": [_P] * 9,
+    "vdn_selftest_wait": [_P, _P],
     "vdn_stream_segment": [_P] * 6 + [ctypes.c_longlong] + [_P] * 5 + [ctypes.c_size_t, _P, _P],
 }
 
@@ -278,6 +279,11 @@ def vdn_stream_segment(s, Q, K, V, beta, alpha, frame0, S_prev, S_in, O, F, work
     _check(lib().vdn_stream_segment(_shp(s), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(alpha), int(frame0),
                                     _ptr(S_prev), _ptr(S_in), _ptr(O), _ptr(F), _ptr(workspace), nbytes,
                                     _ptr(info), _stream(stream)))
+
+
+def vdn_selftest_wait(info, stream=None):
+    """Self-test of the bounded pipeline waits (see vdn.h): *info becomes VDN_INFO_TIMEOUT."""
+    _check(lib().vdn_selftest_wait(_ptr(info), _stream(stream)))
 
 
 def vdn_status_string(status: int) -> str:

@@ -374,6 +374,16 @@ vdn_status vdn_stream_segment(const vdn_shape *s, const void *Q, const void *K,
                               size_t workspace_bytes, int32_t *info,
                               vdn_stream_t stream);
 
+/*
+ * Self-test of the bounded pipeline waits that every tensor-core kernel uses:
+ * launches one CTA whose threads wait, through the same bounded wait, on a
+ * barrier that nothing arrives at. The wait gives up after its limit (1.5 s
+ * of device time), the kernel writes VDN_INFO_TIMEOUT to *info and returns;
+ * nothing traps or hangs, and the CUDA context stays usable. info: a device
+ * int32 (overwritten). VDN_ERR_INVALID for a NULL info.
+ */
+vdn_status vdn_selftest_wait(int32_t *info, vdn_stream_t stream);
+
 /* Name of a status code (static string). */
 const char *vdn_status_string(vdn_status st);
 /* Message of the last failing call on this thread ("" if none). */
