@@ -391,41 +391,67 @@ def pipelined_stage_ms(e, G):
 
 
 def e2e_measure(args, host, d, make_forward, stream, barrier, world, frames_all, dt, og=None):
-    """Same metric through vdn_forward with the step's inputs copied from pinned
-    host memory and O copied back, inside the timed region."""
+    """Same metric through vdn_forward_pipelined with every step's inputs copied
+    from pinned host memory and its O copied back, inside the timed region.
+    Two sets of device buffers and two copy streams let step i + 1's upload
+    and step i - 1's download run while step i computes (PCIe carries both
+    directions at once); every step still moves all of its own bytes."""
     import torch
 
     from frame_wise_delta_b200 import dist as vdist
     from frame_wise_delta_b200 import vdn
 
-    fwd = make_forward(keep_states=False)
-    O_host = torch.empty(fwd.O.shape, dtype=dt).pin_memory()
+    dev = stream.device
+    fw = [make_forward(keep_states=False) for _ in range(2)]
+    din = [d, {k: torch.empty_like(v) for k, v in d.items()}]
+    # the readout epilogue's gate logits and weights travel with each buffer set
+    ogs = [og, None if og is None else vdn.out_gate(din[1]["gate"], din[1]["norm_w"], og.eps)]
+    O_host = [torch.empty(fw[0].O.shape, dtype=dt).pin_memory() for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = O_host.numel() * O_host.element_size()
+    d2h = O_host[0].numel() * O_host[0].element_size()
+    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev = {name: [torch.cuda.Event() for _ in range(2)] for name in ("uploaded", "computed", "downloaded")}
+    for evs in ev.values():  # created and recorded once, so that every wait below has an event
+        for e in evs:
+            e.record(stream)
 
-    def e2e_step():
-        for k in host:
-            d[k].copy_(host[k], non_blocking=True)
-        fwd(d["Q"], d["K"], d["V"], d["beta"], d["alpha"], d["Kx"], d["Vx"], d["beta_x"], og=og)
-        O_host.copy_(fwd.O, non_blocking=True)
+    def e2e_step(i):
+        b = i & 1
+        up.wait_event(ev["computed"][b])  # step i - 2 has read buffer b
+        with torch.cuda.stream(up):
+            for k in host:
+                din[b][k].copy_(host[k], non_blocking=True)
+        ev["uploaded"][b].record(up)
+        stream.wait_event(ev["uploaded"][b])
+        stream.wait_event(ev["downloaded"][b])  # step i - 2's O has left buffer b
+        x = din[b]
+        fw[b](x["Q"], x["K"], x["V"], x["beta"], x["alpha"], x["Kx"], x["Vx"], x["beta_x"], og=ogs[b])
+        ev["computed"][b].record(stream)
+        down.wait_event(ev["computed"][b])
+        with torch.cuda.stream(down):
+            O_host[b].copy_(fw[b].O, non_blocking=True)
+        ev["downloaded"][b].record(down)
 
-    for _ in range(2):
-        e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize()
-    e2e_steps = max(3, min(args.steps, 10))
+    e2e_steps = max(4, min(args.steps, 10))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    up.wait_stream(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    stream.wait_stream(down)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     te = vdist.max_over_ranks(e0.elapsed_time(e1))
-    assert int(fwd.info.item()) == 0
+    assert int(fw[0].info.item()) == 0 and int(fw[1].info.item()) == 0
     return {"value": frames_all / (te / e2e_steps / 1e3), "unit": "frames/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+            "overlap": "two device buffer sets; uploads and downloads on their own streams beside the compute"}
 
 
 def stream_bench(args, w, s, d, dev, stream, barrier, rank, world, local):
