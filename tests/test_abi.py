@@ -163,3 +163,59 @@ def test_gated_readout_validation(L):
     og.eps, og.gate = 1e-6, 0x1004
     assert L.vdn_chunk_readout_gated(_p(s), 16, 16, 16, ogp, 16, None, None) == vdn.VDN_ERR_INVALID
     assert "og->gate" in vdn.vdn_last_error()
+
+
+def _declared_arity():
+    """Parameter count of every function include/vdn.h declares."""
+    import re
+    with open(vdn.HEADER) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(vdn_\w+)\s*\(([^)]*)\)\s*;", text):
+        args = m.group(2).strip()
+        out[m.group(1)] = 0 if args in ("", "void") else args.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_header(L):
+    arity = _declared_arity()
+    for name, args in vdn._SIGS.items():
+        assert name in arity, name
+        assert len(args) == arity[name], (name, len(args), arity[name])
+    # every status-returning entry point of the header has a binding signature
+    ret_other = {"vdn_status_string", "vdn_last_error", "vdn_version", "vdn_text_state_workspace_bytes",
+                 "vdn_forward_workspace_bytes", "vdn_stream_workspace_bytes"}
+    assert set(arity) - ret_other == set(vdn._SIGS)
+
+
+def test_decay_bridge_flag_checks(L):
+    s = _shape()
+    s.decay_bridge = 2
+    assert L.vdn_chunk_readout(_p(s), 16, 16, 16, 16, None, None) == vdn.VDN_ERR_INVALID
+    s.decay_bridge = 1
+    # the plain readouts have no alpha to bridge with
+    assert L.vdn_chunk_readout(_p(s), 16, 16, 16, 16, None, None) == vdn.VDN_ERR_INVALID
+    assert "vdn_chunk_readout_bridged" in vdn.vdn_last_error()
+    # the bridged readout needs alpha
+    assert L.vdn_chunk_readout_bridged(_p(s), 16, 16, 16, None, None, 16, None, None) == vdn.VDN_ERR_INVALID
+    s.decay_bridge = 0
+    assert L.vdn_chunk_readout_bridged(_p(s), 16, 16, 16, 16, None, 16, None, None) == vdn.VDN_ERR_INVALID
+
+
+@pytest.mark.parametrize("frame0", [-5, 3, 7])
+def test_stream_segment_frame0_checks(L, frame0):
+    s = _shape()
+    st = L.vdn_stream_segment(_p(s), 16, 16, 16, 16, 16, frame0, 16, 16, 16, 16, 256, 1 << 30, 16, None)
+    assert st == vdn.VDN_ERR_INVALID
+    assert "frame0" in vdn.vdn_last_error()
+
+
+def test_stream_segment_rejects_the_decay_bridge(L):
+    s = _shape()
+    s.decay_bridge = 1
+    st = L.vdn_stream_segment(_p(s), 16, 16, 16, 16, 16, 0, 16, 16, 16, 16, 256, 1 << 30, 16, None)
+    assert st == vdn.VDN_ERR_UNSUPPORTED
+
+
+def test_selftest_wait_needs_info(L):
+    assert L.vdn_selftest_wait(None, None) == vdn.VDN_ERR_INVALID
