@@ -30,24 +30,24 @@ METRIC = "VDA scan+readout frames/s (tokens/s) at H3 shape on 1 B200; % of roofl
 FALLBACK_HBM_GBS = 6650.0
 # FP32 FMA peak: 148 SMs x 128 lanes x 2 flop x 1.965 GHz (max SM clock).
 ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
-# DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum)
-# at the H3 shape (profiles/launch_list_h3.md), keyed by stage, with the
-# sha256 prefix of the kernel source the counters were taken on; reported as
-# None as soon as that source changes.
+# DRAM bytes of one launch (dram__bytes_read.sum + dram__bytes_write.sum) at
+# the H3 shape, keyed by stage, with the sha256 prefix of the kernel source
+# the counters were taken on; reported as None as soon as that source changes.
+# Each was captured on one kernel of a 4-head case (408 frames) and scaled by
+# the frames a full launch processes (x6): the traffic of these kernels grows
+# in proportion to the frames they stream.
 NCU_TRAFFIC = {
-    "frame_grams": {"bytes": 1291.9e6 + 253.8e6, "source": "frame_wise_delta_b200/csrc/gram_tc.cu",
-                    "sha256_16": "00240b7db02fd61b", "workload": "h3"},
-    "frame_factor": {"bytes": 122.8e6 + 101.2e6, "source": "frame_wise_delta_b200/csrc/invert_tc.cu",
-                     "sha256_16": "d93dd215a7ca697f", "workload": "h3"},
-    "chunk_readout": {"bytes": 700.8e6 + 581.3e6, "source": "frame_wise_delta_b200/csrc/readout_tc.cu",
-                      "sha256_16": "9a564eca14ecfc6e", "workload": "h3"},
+    "frame_grams": {"bytes": 6 * (214.5e6 + 25.3e6), "source": "frame_wise_delta_b200/csrc/gram_tc.cu",
+                    "sha256_16": "00240b7db02fd61b", "workload": "h3", "capture": "h3 with 4 heads, x6"},
+    "chunk_readout": {"bytes": 6 * (118.8e6 + 58.1e6), "source": "frame_wise_delta_b200/csrc/readout_tc.cu",
+                      "sha256_16": "9a564eca14ecfc6e", "workload": "h3", "capture": "h3 with 4 heads, x6"},
 }
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["vdn", "reference"], default="vdn")
     ap.add_argument("--workload", default="h3")
@@ -100,28 +100,41 @@ def load_peaks():
 
 # --------------------------------------------------------------- clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples every 50 ms while the timed loop runs. Samples carry
+    their host timestamps; the summary keeps those taken between mark_start()
+    and mark_end() (the timed region), or the nearest one when the region is
+    shorter than the sampling period."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_MS = 50
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
-                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms",
+                 str(self.PERIOD_MS), "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
         except OSError:
             self.proc = None
         time.sleep(0.3)
         return self
 
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
     def __exit__(self, *exc):
         self.lines = []
         if self.proc is not None:
-            time.sleep(0.3)
+            time.sleep(0.1)
             self.proc.terminate()
             try:
                 out, _ = self.proc.communicate(timeout=5)
@@ -130,25 +143,40 @@ class ClockSampler:
                 out, _ = self.proc.communicate()
             self.lines = [l for l in out.splitlines() if l.strip()]
 
+    @staticmethod
+    def _stamp(s):
+        import datetime
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                return datetime.datetime.strptime(s.strip(), fmt).timestamp()
+            except ValueError:
+                continue
+        return None
+
     def summary(self):
-        sm, mx, reasons = [], [], set()
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for l in getattr(self, "lines", []):
             parts = [p.strip() for p in l.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
+                rows.append((self._stamp(parts[0]), float(parts[2]), float(parts[3]),
+                             {n for n, v in zip(names, parts[6:10]) if v.lower().startswith("active")}))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
+        if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        in_window = rows
+        if self.t0 is not None and self.t1 is not None and all(r[0] is not None for r in rows):
+            in_window = [r for r in rows if self.t0 <= r[0] <= self.t1]
+            if not in_window:  # a region shorter than the period: the sample nearest its middle
+                mid = 0.5 * (self.t0 + self.t1)
+                in_window = [min(rows, key=lambda r: abs(r[0] - mid))]
+        reasons = set().union(*(r[3] for r in in_window))
+        return {"sm_mhz": statistics.median(r[1] for r in in_window), "sm_max_mhz": max(r[2] for r in in_window),
+                "reasons": sorted(reasons), "samples": len(in_window), "period_ms": self.PERIOD_MS,
+                "window_s": None if self.t0 is None or self.t1 is None else round(self.t1 - self.t0, 4)}
 
 
 # ------------------------------------------------------------- oracle arm
@@ -183,16 +211,17 @@ def run_reference(args, w):
         return
     from frame_wise_delta_b200 import synth
 
-    full = {}
-    # one head per step: a bounded sample of the same workload
-    pairs = [(b, h) for b in range(w.B) for h in range(w.H)]
     import oracle
 
+    # One (b,h) pair per step: a bounded sample of the same workload. The
+    # pairs' inputs are drawn before the warm-up, so the timed steps run the
+    # oracle and nothing else; every pair is a whole problem of the same size,
+    # so a few distinct pairs in turn stand for all of them.
+    pairs = [(b, h) for b in range(w.B) for h in range(w.H)][:4]
+    inputs = [synth.generate_head(w, b, h) for b, h in pairs]
+
     def step(i):
-        b, h = pairs[i % len(pairs)]
-        if (b, h) not in full:
-            full[(b, h)] = synth.generate_head(w, b, h)
-        oracle.vda_head(full[(b, h)], w.chunk, w.anchors)
+        oracle.vda_head(inputs[i % len(inputs)], w.chunk, w.anchors)
 
     for i in range(args.warmup):
         step(i)
@@ -212,7 +241,8 @@ def run_reference(args, w):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(w),
         "cpu_baseline": {"value": value, "unit": "frames/s", "cores": cores, "kind": "oracle",
-                         "sample": f"one (b,h) pair of {w.name} per step, all {w.T} frames"},
+                         "sample": f"one (b,h) pair of {w.name} per step (all {w.T} frames), {len(pairs)} "
+                                   f"distinct pairs in turn, inputs drawn before the timed steps"},
         "e2e": {"value": value, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -332,9 +362,11 @@ def main():
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
                       else local) as clk:
+        clk.mark_start()
         for i in range(args.steps):
             step(evs[i])
         torch.cuda.synchronize()
+        clk.mark_end()
     barrier()
     assert int(info.item()) == 0, f"device status {int(info.item())}"
     first, last = 0, n_ev - 1
@@ -364,6 +396,7 @@ def main():
             "data": "synthetic", "config": workload_config(w, args.gated),
             "tokens_per_s": value * U,
             "hbm_frac_whole_pass": alg_bytes(w, args.gated) * world / (ms_per_step / 1e3) / (hbm_gbs * 1e9),
+            "roofline_whole_pass": whole_pass_roofline(w, ms_per_step, world, hbm_gbs, peak_src, args.gated),
             "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
             "step_ms_min_max": [min(step_ms), max(step_ms)],
             "roofline": roof,
@@ -498,11 +531,13 @@ def stream_bench(args, w, s, d, dev, stream, barrier, rank, world, local):
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local) as clk:
+        clk.mark_start()
         e0.record(stream)
         for _ in range(args.steps):
             step()
         e1.record(stream)
         torch.cuda.synchronize()
+        clk.mark_end()
     barrier()
     assert int(info.item()) == 0, f"device status {int(info.item())}"
     ms_per_step = vdist.max_over_ranks(e0.elapsed_time(e1)) / args.steps
@@ -546,12 +581,11 @@ def alg_bytes(w, gated=False):
     return qkvo + text + gates
 
 
-def roofline(w, stage_ms, hbm_gbs, peak_src, bf16_tflops=1607.7):
-    """Roofline of the dominant stage. Per-unit algorithmic figures:
-    frame_grams: per frame reads K, V (2 U d bf16) and writes A, B (2 d^2 fp32);
-      on the tensor path only rows 64.. of A (d^2/2 fp32) plus the 16 KB P^{-1}
-      tile its sweep warps produce;
-    chunk_readout: per frame reads Q, writes O (2 U d bf16) plus two states per chunk;
+def stage_work(w):
+    """Algorithmic work of one launch of each stage, with its bound:
+    frame_grams: reads K and V (2 U d input elements per frame, plus U gates
+      per frame with per-token write gates);
+    chunk_readout: reads Q and writes O (2 U d elements per frame);
     frame_factor: on the tensor path the CUDA cores sweep two 64 x 64 blocks per
       non-anchor frame (d^3 / 4 flop; the block products run on the tensor
       cores), 4 d^3 on the CUDA-core path (Gauss-Jordan on [I+A; B]);
@@ -567,15 +601,33 @@ def roofline(w, stage_ms, hbm_gbs, peak_src, bf16_tflops=1607.7):
     for c in range(C):
         fr = [t for t in range(5 * c, min(5 * c + 5, T)) if not (w.anchors and t in (0, T - 1))]
         steps += len(fr) if tensor_path else max(0, len(range(5 * c, min(5 * c + 5, T))) - 1)
-    units = {
-        "frame_grams": ("hbm", frames * (2 * U * d * e + (d * d * 4 // 2 + d * d * 4 + 16384 if tensor_path
-                                                          else 2 * d * d * 4)
-                                         + (U * 4 if w.beta_per_token else 0))),
-        "chunk_readout": ("hbm", frames * 2 * U * d * e + BH * C * 2 * d * d * 4),
+    return {
+        "frame_grams": ("hbm", frames * (2 * U * d * e + (U * 4 if w.beta_per_token else 0))),
+        "chunk_readout": ("hbm", frames * 2 * U * d * e),
         "frame_factor": ("alu", live * (d ** 3 // 4 if tensor_path else 4 * d ** 3)),
         "chunk_compose": ("tensor" if tensor_path else "alu", BH * 2 * steps * 4 * d ** 3),
         "scan_bidir": ("tensor" if tensor_path else "alu", BH * 2 * C * 2 * d ** 3),
     }
+
+
+def intermediate_bytes(w):
+    """HBM bytes a streaming stage moves beyond its algorithmic operands, per
+    launch: the Gram kernel writes B_t and (tensor path) rows 64.. of A_t plus
+    the 16 KB P^{-1} tile of its sweep warps (both A_t halves on the CUDA-core
+    path); the readout reads two fp32 states per chunk."""
+    BH, T, d, C = w.B * w.H, w.T, w.d, w.C
+    tensor_path = w.dtype == "bf16" and d == 128
+    gram = (d * d * 4 + d * d * 4 // 2 + 16384) if tensor_path else 2 * d * d * 4
+    return {"frame_grams": BH * T * gram, "chunk_readout": BH * C * 2 * d * d * 4}
+
+
+def roofline(w, stage_ms, hbm_gbs, peak_src, bf16_tflops=1607.7):
+    """Roofline of the stage with the largest event time: its algorithmic
+    work per launch (stage_work) over its mean launch time, against the
+    measured peak of its bound. Bytes the kernel moves beyond that work
+    (intermediate_bytes) and its ncu DRAM traffic are reported beside it,
+    with traffic / algorithmic bytes; neither enters `achieved`."""
+    units = stage_work(w)
     name = max((k for k in units), key=lambda k: stage_ms.get(k, 0.0))
     bound, amount = units[name]
     sec = stage_ms[name] / 1e3
@@ -598,9 +650,22 @@ def roofline(w, stage_ms, hbm_gbs, peak_src, bf16_tflops=1607.7):
         with open(os.path.join(ROOT, rec["source"]), "rb") as f:
             if hashlib.sha256(f.read()).hexdigest()[:16] == rec["sha256_16"]:
                 tr = rec["bytes"]
-    return {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-            "frac": achieved / peak, "traffic": tr, "peak_source": src,
-            "per_stage_ms": {k: round(v, 4) for k, v in stage_ms.items()}}
+    out = {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+           "frac": achieved / peak, "traffic": tr, "peak_source": src,
+           "per_stage_ms": {k: round(v, 4) for k, v in stage_ms.items()}}
+    if bound == "hbm":
+        out["algorithmic_bytes"] = amount
+        out["intermediate_bytes"] = intermediate_bytes(w).get(name, 0)
+        out["traffic_over_algorithmic"] = None if tr is None else tr / amount
+    return out
+
+
+def whole_pass_roofline(w, ms_per_step, world, hbm_gbs, peak_src, gated=False):
+    """The whole pass against HBM bandwidth: algorithmic bytes (Q, K, V read,
+    O written, gates and text) over the step time."""
+    achieved = alg_bytes(w, gated) * world / (ms_per_step / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
+            "algorithmic_bytes": alg_bytes(w, gated) * world, "peak_source": f"{peak_src} HBM copy bandwidth"}
 
 
 if __name__ == "__main__":

@@ -241,6 +241,11 @@ __global__ void wait_selftest_kernel(int32_t *info) {
 
 void vdn::set_last_error(const char *msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
 
+vdn_status vdn::validate_shape(const vdn_shape *s) {
+  Geo g;
+  return check_shape(s, &g);
+}
+
 extern "C" {
 
 const char *vdn_status_string(vdn_status st) {

@@ -90,6 +90,10 @@ cudaError_t launch_scan_tc(const uint8_t *Mimg, const float *Jf, const float *Jb
 // Message returned by vdn_last_error() on this thread.
 void set_last_error(const char *msg);
 
+// The shape checks every entry point applies (sizes, d, chunk, flags,
+// dtypes, index ranges); on failure the message is set as by the entry points.
+vdn_status validate_shape(const vdn_shape *s);
+
 // Driver entry point for tensor-map encoding (resolved once, thread-safe).
 void *tensor_map_encoder();
 int device_sm_count();

@@ -12,9 +12,12 @@
 // The scratch is a file-scope __device__ array of kScratchBytes (4 MiB). Every
 // GPU that loads the library keeps it until the process exits. Host code must
 // not pass the array's name to a kernel (on the host it only stands in for
-// the symbol), so its device address is looked up once per device with
-// cudaGetSymbolAddress, with that device current, on the first call made on
-// that device; make that first call before any stream capture.
+// the symbol), so its device address is looked up with cudaGetSymbolAddress,
+// with the device current, on the first call made on that device; make that
+// first call before any stream capture. The address is kept per device
+// together with the identity of the context it was looked up in: if that
+// context has been destroyed and another created (cudaDeviceReset), the array
+// was loaded again, possibly elsewhere, and the next call looks it up anew.
 //
 // All calls share the one array and it keeps the last call's contents.
 // Nothing in it has to start at zero: the Gram kernels overwrite every element
@@ -47,22 +50,59 @@ vdn_status fail(vdn_status st, const char *fmt, ...) {
   return st;
 }
 
-// Device address of g_text_scratch on the current device (looked up once).
+// Driver entry points for the identity of the current context (resolved once).
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+void *driver_fn(const char *name) {
+  void *p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return p;
+}
+
+// Unique id of the calling thread's current context, 0 if there is none (or
+// the driver cannot tell): then nothing is cached.
+unsigned long long current_context_id() {
+  static std::once_flag once;
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  std::call_once(once, [] {
+    get_current = reinterpret_cast<CtxGetCurrentFn>(driver_fn("cuCtxGetCurrent"));
+    get_id = reinterpret_cast<CtxGetIdFn>(driver_fn("cuCtxGetId"));
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of g_text_scratch on the current device, looked up once per
+// device and context.
 cudaError_t scratch_address(float **out) {
   static std::mutex mu;
-  static void *addr[kMaxDevices] = {};
+  struct Slot {
+    void *addr;
+    unsigned long long ctx;
+  };
+  static Slot slot[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (slot[dev].addr == nullptr || ctx == 0 || slot[dev].ctx != ctx) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_text_scratch);
     if (e != cudaSuccess) return e;
-    addr[dev] = p;
+    // the lookup makes the device's primary context current if it was not yet
+    slot[dev] = Slot{p, ctx != 0 ? ctx : current_context_id()};
   }
-  *out = static_cast<float *>(addr[dev]);
+  *out = static_cast<float *>(slot[dev].addr);
   return cudaSuccess;
 }
 
@@ -75,14 +115,9 @@ extern "C" vdn_status vdn_text_state_noalloc(const vdn_shape *s, const void *Kx,
                                              vdn_stream_t stream) {
   using namespace vdn;
   set_last_error("");
-  if (!s) return fail(VDN_ERR_INVALID, "shape is NULL");
-  if (s->B < 0 || s->H < 0 || s->n_text < 0) return fail(VDN_ERR_INVALID, "negative size");
-  if (s->dk != s->dv || (s->dk != 16 && s->dk != 32 && s->dk != 64 && s->dk != 128))
-    return fail(VDN_ERR_UNSUPPORTED, "need dk == dv in {16, 32, 64, 128}");
-  if (s->in_dtype != VDN_F32 && s->in_dtype != VDN_BF16)
-    return fail(VDN_ERR_INVALID, "in_dtype must be VDN_F32 or VDN_BF16");
-  if (s->beta_per_token != 0 && s->beta_per_token != 1)
-    return fail(VDN_ERR_INVALID, "beta_per_token must be 0 or 1");
+  // the same shape rules as vdn_text_state (and every other entry point)
+  const vdn_status vs = validate_shape(s);
+  if (vs != VDN_OK) return vs;
   const bool tokb = s->beta_per_token != 0;
   const long long BH = (long long)s->B * s->H;
   const int D = s->dk;

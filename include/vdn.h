@@ -24,8 +24,10 @@
  * Streams    : each call validates its arguments on the host, enqueues its
  *              kernels on `stream` (NULL = the legacy default stream) and
  *              returns without synchronising. There is no global mutable
- *              state; calls on different streams may run concurrently if
- *              their outputs do not overlap.
+ *              state but one: the fixed scratch array of
+ *              vdn_text_state_noalloc (see there), which calls of that entry
+ *              point share. Calls of every other entry point on different
+ *              streams may run concurrently if their outputs do not overlap.
  * Errors     : argument problems are reported synchronously (VDN_ERR_INVALID
  *              or VDN_ERR_UNSUPPORTED) before anything is enqueued; a launch
  *              failure returns VDN_ERR_CUDA. vdn_last_error() gives a one-line
@@ -268,7 +270,10 @@ vdn_status vdn_text_state(const vdn_shape *s, const void *Kx, const void *Vx,
  * 2 * B * H * dk * dk * 4 bytes must not exceed 4 MiB (B*H <= 32 at d = 128),
  * else VDN_ERR_UNSUPPORTED is returned before anything is enqueued.
  * The first call on a device looks up the array's device address (once per
- * device, with that device current); make it before any stream capture.
+ * device and context, with that device current); make it before any stream
+ * capture. A call after the device's context was destroyed and recreated
+ * (cudaDeviceReset) looks the address up again.
+ * Shapes are validated as for vdn_text_state, then against the scratch size.
  * Every call shares the array and it keeps the last call's contents (nothing
  * in it needs to start at zero); calls that overlap on the GPU race on it.
  * In/Out/info as for vdn_text_state. Allocates nothing.

@@ -326,5 +326,8 @@ def rel_frobenius(x, ref) -> float:
     den = np.linalg.norm(ref.ravel())
     num = np.linalg.norm((x - ref).ravel())
     if den == 0.0:
-        return 0.0 if num == 0.0 else math.inf
+        # a zero reference: equal arrays agree exactly, any other differs
+        # without bound (tested element by element, so a tiny difference whose
+        # square underflows still counts)
+        return 0.0 if not np.any(x != ref) else math.inf
     return float(num / den)

@@ -219,3 +219,17 @@ def test_stream_segment_rejects_the_decay_bridge(L):
 
 def test_selftest_wait_needs_info(L):
     assert L.vdn_selftest_wait(None, None) == vdn.VDN_ERR_INVALID
+
+
+@pytest.mark.parametrize("kw", [dict(chunk=0), dict(chunk=17), dict(anchors=2), dict(T=-1)])
+def test_noalloc_applies_the_same_shape_rules(L, kw):
+    """vdn_text_state_noalloc rejects every shape vdn_text_state rejects, with
+    the same status, before it touches the device."""
+    s = _shape(**kw)
+    a = L.vdn_text_state(_p(s), 16, 16, 16, 16, 16, 1 << 20, 16, None)
+    b = L.vdn_text_state_noalloc(_p(s), 16, 16, 16, 16, 16, None)
+    assert a == b == vdn.VDN_ERR_INVALID
+    for flag in ("decay_bridge", "out_dtype"):
+        s = _shape()
+        setattr(s, flag, 5)
+        assert L.vdn_text_state_noalloc(_p(s), 16, 16, 16, 16, 16, None) == vdn.VDN_ERR_INVALID

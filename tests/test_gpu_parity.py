@@ -11,7 +11,7 @@ import torch
 
 import oracle
 from frame_wise_delta_b200 import synth, vdn
-from vdn_testlib import TOL, device_fill, device_inputs, oracle_heads, rel, run_forward, tdtype, to_dev
+from vdn_testlib import OUT_GUARD, STATE_GUARD, TOL, device_fill, device_inputs, oracle_heads, rel, run_forward, tdtype, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -68,6 +68,7 @@ def test_forward_matches_oracle(w):
         eo, ef, eg = rel(fw.O[b, h], r["O"]), rel(fw.F[b, h], r["F"]), rel(fw.G[b, h], r["G"])
         print(f"{w.name} b{b} h{h}: O {eo:.2e} F {ef:.2e} G {eg:.2e}")
         assert eo <= tol and ef <= tol and eg <= tol
+        assert ef <= STATE_GUARD and eg <= STATE_GUARD and eo <= OUT_GUARD[w.dtype], (ef, eg, eo)
 
 
 # ------------------------------------------------------------- per stage
@@ -344,5 +345,6 @@ def test_full_size_sampled_heads(name, pairs):
         eo, ef, eg = rel(fw.O[b, h], r["O"]), rel(fw.F[b, h], r["F"]), rel(fw.G[b, h], r["G"])
         print(f"{name} b{b} h{h}: O {eo:.2e} F {ef:.2e} G {eg:.2e}")
         assert eo <= TOL["bf16"] and ef <= TOL["bf16"] and eg <= TOL["bf16"]
+        assert ef <= STATE_GUARD and eg <= STATE_GUARD and eo <= OUT_GUARD["bf16"], (ef, eg, eo)
     del dev, fw
     torch.cuda.empty_cache()

@@ -9,7 +9,7 @@ import torch
 
 import oracle
 from frame_wise_delta_b200 import synth, vdn
-from vdn_testlib import TOL, device_fill, device_inputs, rel, run_forward
+from vdn_testlib import OUT_GUARD, STATE_GUARD, TOL, device_fill, device_inputs, rel, run_forward
 
 pytestmark = pytest.mark.gpu
 
@@ -103,5 +103,6 @@ def test_pipelined_full_size_sampled_heads():
         eo, ef, eg = rel(fw.O[b, h], r["O"]), rel(fw.F[b, h], r["F"]), rel(fw.G[b, h], r["G"])
         print(f"h3 pipelined b{b} h{h}: O {eo:.2e} F {ef:.2e} G {eg:.2e}")
         assert eo <= TOL["bf16"] and ef <= TOL["bf16"] and eg <= TOL["bf16"]
+        assert ef <= STATE_GUARD and eg <= STATE_GUARD and eo <= OUT_GUARD["bf16"], (ef, eg, eo)
     del dev, fw
     torch.cuda.empty_cache()

@@ -17,7 +17,7 @@ import torch
 
 import oracle
 from frame_wise_delta_b200 import synth, vdn
-from vdn_testlib import TOL, device_fill, device_inputs, rel, to_dev
+from vdn_testlib import OUT_GUARD, STATE_GUARD, TOL, device_fill, device_inputs, rel, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -195,5 +195,6 @@ def test_full_size_h3_stream(pairs):
         eo, ef = rel(O[b, h], Or), rel(F[b, h], Fr)
         print(f"h3 stream b{b} h{h}: O {eo:.2e} F {ef:.2e}")
         assert eo <= TOL["bf16"] and ef <= TOL["bf16"]
+        assert ef <= STATE_GUARD and eo <= OUT_GUARD["bf16"], (ef, eo)
     del dev
     torch.cuda.empty_cache()

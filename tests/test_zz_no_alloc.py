@@ -1,15 +1,19 @@
-"""vdn_text_state_noalloc against vdn_text_state.
+"""vdn_text_state_noalloc against vdn_text_state and the fp64 oracle.
 
 The no-allocation entry point serves callers that cannot give the library a
 device workspace (a fixed memory plan, or a loop that must not call
 cudaMalloc); it keeps its scratch in a fixed device array instead. It must
 give the same text state as the workspace version, call after call, although
-every call reuses (and leaves behind) the same scratch. This file is collected
-last so that a run stopping at the first failure has run every other test.
+every call reuses (and leaves behind) the same scratch; and since it factors
+on another route than the workspace version (the CUDA-core factor kernel),
+its result is also held to the oracle's text state directly. This file is
+collected last so that a run stopping at the first failure has run every
+other test.
 """
 import pytest
 import torch
 
+import oracle
 from frame_wise_delta_b200 import synth, vdn
 from vdn_testlib import device_inputs, rel
 
@@ -53,6 +57,25 @@ def test_no_alloc_text_state_matches_workspace_version():
             assert torch.isfinite(got).all()
             e = rel(got, ref.double().cpu().numpy())
             assert e <= 1e-5, (round_, w.name, e)
+
+
+def test_no_alloc_text_state_matches_the_oracle():
+    """Each case twice in a row, against the fp64 text state of the same
+    (bf16-rounded where the case is bf16) inputs: the route's only error is
+    its float32 arithmetic."""
+    torch.cuda.set_device(0)
+    for round_ in range(2):
+        for w in CASES:
+            full = synth.generate_all(w)
+            dev = device_inputs(w, full)
+            got, info = _no_alloc(w, dev)
+            torch.cuda.synchronize()
+            assert int(info.item()) == 0
+            for b in range(w.B):
+                for h in range(w.H):
+                    ref = oracle.text_state(full["Kx"][b, h], full["Vx"][b, h], full["beta_x"][b, h])
+                    e = rel(got[b, h], ref)
+                    assert e <= 1e-5, (round_, w.name, b, h, e)
 
 
 def test_no_alloc_rejects_sizes_beyond_its_scratch():
