@@ -16,6 +16,7 @@ from .vda import (  # noqa: F401
     readout_state,
     rel_frobenius,
     scan_states,
+    stream_bridge_tail,
     stream_segment,
     text_state,
     transition,

@@ -281,7 +281,8 @@ def vda_head(inp: dict, chunk: int = 5, anchors: int = 0, bridge: bool = False) 
     return out
 
 
-def stream_segment(Q, K, V, beta, alpha, S_prev, S_in, chunk: int = 5, anchor_first: bool = False):
+def stream_segment(Q, K, V, beta, alpha, S_prev, S_in, chunk: int = 5, anchor_first: bool = False,
+                   bridge: bool = False, alpha_prev=None):
     """One segment of a live stream read through the forward memory only.
 
     Reading of the page's livestream framing ("Future directions": continuous
@@ -294,11 +295,22 @@ def stream_segment(Q, K, V, beta, alpha, S_prev, S_in, chunk: int = 5, anchor_fi
     the text state, counted once by the single scan); anchor_first makes the
     segment's first frame an anchor (the stream's frame 0).
 
+    bridge: read through the decay bridge of "Method steps" step (5), forward
+    half (the reading of bridge_factors): frame t of chunk c reads the state
+    before its window carried through the decay of the window's frames up to
+    t, R_t = F_{c-1} Diag(prod_{r=f0..t} alpha_r) with f0 the first frame of
+    chunk c - 1. For the segment's chunk 0 the window starts in the previous
+    segment's last chunk, whose decay product alpha_prev ([d_k], see
+    stream_bridge_tail; ones, or None, for the stream's first segment) joins
+    the product: R_t = S_prev Diag(alpha_prev * prod_{r=0..t} alpha_r). An
+    anchor frame's alpha counts as 1.
+
     Q, K, V: [T, U, d]; beta: [T] (or [T, U]); alpha: [T, d_k].
     Returns O [T, U, d_v] and F [C+1, d_v, d_k] with F[0] = S_in and F[j] the
     state after the segment's chunks 0..j-1 (frame by frame, no chunk maps).
     """
     Q = _f64(Q)
+    alpha = _f64(alpha)
     T = K.shape[0]
     C = num_chunks(T, chunk)
     S = _f64(S_in).copy()
@@ -309,14 +321,34 @@ def stream_segment(Q, K, V, beta, alpha, S_prev, S_in, chunk: int = 5, anchor_fi
             S = frame_update(S, alpha[t], *frame_stats(K[t], V[t], beta[t]))
         if (t + 1) % chunk == 0 or t == T - 1:
             F[num_chunks(t + 1, chunk)] = S
+    d_k = S.shape[1]
     O = np.zeros((T,) + Q.shape[1:2] + (S.shape[0],))
     for t in range(T):
         if anchor_first and t == 0:
             continue
         c = t // chunk
         R = _f64(S_prev) if c == 0 else F[c - 1]
+        if bridge:
+            p = np.ones(d_k) if (c > 0 or alpha_prev is None) else _f64(alpha_prev).copy()
+            for r in range(chunk * max(c - 1, 0), t + 1):
+                if not (anchor_first and r == 0):
+                    p = p * alpha[r]
+            R = R * p[None, :]
         O[t] = Q[t] @ R.T
     return O, F
+
+
+def stream_bridge_tail(alpha, chunk: int = 5, anchor_first: bool = False):
+    """Decay product over a segment's last chunk (the frames a next segment's
+    first chunk finds at the start of its window): prod alpha_r over
+    r = chunk * (C - 1) .. T - 1, an anchor frame counting as 1. [d_k]."""
+    alpha = _f64(alpha)
+    T, d_k = alpha.shape
+    p = np.ones(d_k)
+    for r in range(chunk * (num_chunks(T, chunk) - 1), T):
+        if not (anchor_first and r == 0):
+            p = p * alpha[r]
+    return p
 
 
 def rel_frobenius(x, ref) -> float:

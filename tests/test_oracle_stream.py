@@ -112,3 +112,80 @@ def test_segments_compose(cut):
                                    chunk=5)
     np.testing.assert_array_equal(np.concatenate([O1, O2]), O)
     np.testing.assert_array_equal(np.concatenate([F1, F2[1:]]), F)
+
+
+# ----------------------------------------------------------- decay bridge
+def _decay_only(S, alphas):
+    """Carry a state through frames whose write gates are zero: the frame
+    solve itself with beta = 0 (no bridge formula involved)."""
+    d = S.shape[1]
+    for a in alphas:
+        S = _update(S, np.zeros((1, d)), np.zeros((1, S.shape[0])), 0.0, a)
+    return S
+
+
+def test_bridged_stream_is_the_decay_only_recurrence():
+    # frame t of chunk c reads the state before its window carried through
+    # frames f0..t by the recurrence with the window's writes switched off
+    rng = np.random.default_rng(21)
+    T, U, d, chunk = 17, 3, 4, 5
+    Q, K, V, beta, alpha = _clip(rng, T, U, d)
+    S_prev = rng.standard_normal((d, d))
+    S_in = rng.standard_normal((d, d))
+    a_prev = rng.uniform(0.8, 1.0, d)
+    O, F = oracle.stream_segment(Q, K, V, beta, alpha, S_prev, S_in, chunk=chunk, bridge=True, alpha_prev=a_prev)
+    for t in range(T):
+        c = t // chunk
+        if c == 0:
+            # the previous segment's last chunk decays S_prev first (one
+            # frame whose alpha is that chunk's product), then frames 0..t
+            R = _decay_only(S_prev, [a_prev] + [alpha[r] for r in range(0, t + 1)])
+        else:
+            R = _decay_only(F[c - 1], [alpha[r] for r in range(chunk * (c - 1), t + 1)])
+        np.testing.assert_allclose(O[t], Q[t] @ R.T, rtol=1e-11, atol=1e-12)
+
+
+def test_bridged_stream_without_decay_is_the_plain_stream():
+    rng = np.random.default_rng(22)
+    T, U, d = 12, 3, 4
+    Q, K, V, beta, alpha = _clip(rng, T, U, d)
+    S = rng.standard_normal((d, d))
+    ones = np.ones_like(alpha)
+    O1, F1 = oracle.stream_segment(Q, K, V, beta, ones, S, S, chunk=5, anchor_first=True, bridge=True,
+                                   alpha_prev=np.ones(d))
+    O0, F0 = oracle.stream_segment(Q, K, V, beta, ones, S, S, chunk=5, anchor_first=True)
+    np.testing.assert_array_equal(O1, O0)
+    np.testing.assert_array_equal(F1, F0)
+
+
+def test_bridge_tail_of_a_segment():
+    rng = np.random.default_rng(23)
+    alpha = rng.uniform(0.5, 1.0, (12, 3))
+    # last chunk of 12 frames in chunks of 5: frames 10, 11
+    np.testing.assert_array_equal(oracle.stream_bridge_tail(alpha, 5), alpha[10] * alpha[11])
+    # one chunk holding the stream's anchor frame 0: frames 1..4 only
+    np.testing.assert_allclose(oracle.stream_bridge_tail(alpha[:5], 5, anchor_first=True),
+                               alpha[1] * alpha[2] * alpha[3] * alpha[4], rtol=0, atol=0)
+
+
+@pytest.mark.parametrize("cuts", [(5,), (10,), (5, 15), (5, 10, 15, 20)])
+def test_bridged_segments_compose(cuts):
+    # cutting a bridged stream at chunk boundaries and carrying
+    # (F[C-1], F[C], the last chunk's decay product) changes nothing
+    rng = np.random.default_rng(31 + len(cuts))
+    T, U, d = 23, 3, 4
+    Q, K, V, beta, alpha = _clip(rng, T, U, d, (0.7, 1.0))
+    S_T = rng.standard_normal((d, d))
+    O, F = oracle.stream_segment(Q, K, V, beta, alpha, S_T, S_T, chunk=5, anchor_first=True, bridge=True)
+    bounds = [0, *cuts, T]
+    Sp, Si, ap = S_T, S_T, np.ones(d)
+    Os, Fs = [], [F[:1]]
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        o, f = oracle.stream_segment(Q[a:b], K[a:b], V[a:b], beta[a:b], alpha[a:b], Sp, Si, chunk=5,
+                                     anchor_first=a == 0, bridge=True, alpha_prev=ap)
+        Os.append(o)
+        Fs.append(f[1:])
+        C = f.shape[0] - 1
+        Sp, Si, ap = f[C - 1], f[C], oracle.stream_bridge_tail(alpha[a:b], 5, anchor_first=a == 0)
+    np.testing.assert_allclose(np.concatenate(Os), O, rtol=1e-13, atol=1e-14)
+    np.testing.assert_array_equal(np.concatenate(Fs), F)
