@@ -2,8 +2,9 @@
 
 Every (batch, head) pair of VDA is independent (text state, frame statistics,
 factor, composition, scans and readout), so the path shards over GPUs with no
-collective on the data path: each rank owns a set of (b, h) pairs (strong
-scaling) or a whole problem of its own (weak scaling). torch.distributed is
+collective on the data path: each rank owns a contiguous share of one
+problem's (b, h) pairs (strong scaling: `bench.py --shard heads`) or a whole
+problem of its own (weak scaling). torch.distributed is
 used only to line ranks up and to take the slowest rank's time.
 """
 from __future__ import annotations
@@ -29,6 +30,23 @@ def head_ranges(B: int, H: int, rank: int, world: int) -> list[tuple[int, int, i
         else:
             runs.append((b, h, h + 1))
     return runs
+
+
+def pair_range(B: int, H: int, rank: int, world: int) -> tuple[int, int]:
+    """The rank's share of the B*H pairs as a half-open range [lo, hi) of the
+    flattened (b * H + h) index (the pairs of shard_pairs)."""
+    pairs = shard_pairs(B, H, rank, world)
+    if not pairs:
+        return (0, 0)
+    return (pairs[0][0] * H + pairs[0][1], pairs[-1][0] * H + pairs[-1][1] + 1)
+
+
+def shard_view(x, B: int, H: int, rank: int, world: int):
+    """The rank's pairs of a [B, H, ...] array or tensor as a [1, n, ...] view:
+    a contiguous range of the flattened pairs, which the library takes as one
+    batch of n heads (every pair is independent)."""
+    lo, hi = pair_range(B, H, rank, world)
+    return x.reshape((1, B * H) + tuple(x.shape[2:]))[:, lo:hi]
 
 
 def max_over_ranks(x: float) -> float:

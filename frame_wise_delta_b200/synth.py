@@ -173,26 +173,34 @@ def generate_head(w: Workload, b: int, h: int, parts=ALL_PARTS) -> dict:
     return {k: make[k]() for k in parts}
 
 
+def generate_pairs(w: Workload, pairs, threads: int = 8) -> dict:
+    """Inputs of the given (b, h) pairs stacked as [1, len(pairs), ...] float32
+    arrays: a contiguous share of the pairs laid out as one batch of that many
+    heads, each pair drawn exactly as in the full set."""
+    n = len(pairs)
+    out = {
+        "Q": np.empty((1, n, w.T, w.U, w.d), np.float32),
+        "K": np.empty((1, n, w.T, w.U, w.d), np.float32),
+        "V": np.empty((1, n, w.T, w.U, w.d), np.float32),
+        "Kx": np.empty((1, n, w.n_text, w.d), np.float32),
+        "Vx": np.empty((1, n, w.n_text, w.d), np.float32),
+        "beta": np.empty((1, n, w.T, w.U) if w.beta_per_token else (1, n, w.T), np.float32),
+        "alpha": np.empty((1, n, w.T, w.d), np.float32),
+        "beta_x": np.empty((1, n, w.n_text) if w.beta_per_token else (1, n), np.float32),
+    }
+
+    def fill(i):
+        b, h = pairs[i]
+        for k, v in generate_head(w, b, h).items():
+            out[k][0, i] = v
+
+    with ThreadPoolExecutor(max(1, threads)) as ex:
+        list(ex.map(fill, range(n)))
+    return out
+
+
 def generate_all(w: Workload, threads: int = 8) -> dict:
     """Full [B, H, ...] float32 arrays for every input of a workload."""
     pairs = [(b, h) for b in range(w.B) for h in range(w.H)]
-    full = {
-        "Q": np.empty((w.B, w.H, w.T, w.U, w.d), np.float32),
-        "K": np.empty((w.B, w.H, w.T, w.U, w.d), np.float32),
-        "V": np.empty((w.B, w.H, w.T, w.U, w.d), np.float32),
-        "Kx": np.empty((w.B, w.H, w.n_text, w.d), np.float32),
-        "Vx": np.empty((w.B, w.H, w.n_text, w.d), np.float32),
-        "beta": np.empty((w.B, w.H, w.T, w.U) if w.beta_per_token else (w.B, w.H, w.T), np.float32),
-        "alpha": np.empty((w.B, w.H, w.T, w.d), np.float32),
-        "beta_x": np.empty((w.B, w.H, w.n_text) if w.beta_per_token else (w.B, w.H), np.float32),
-    }
-
-    def fill(bh):
-        b, h = bh
-        one = generate_head(w, b, h)
-        for k, v in one.items():
-            full[k][b, h] = v
-
-    with ThreadPoolExecutor(max(1, threads)) as ex:
-        list(ex.map(fill, pairs))
-    return full
+    flat = generate_pairs(w, pairs, threads)
+    return {k: v.reshape((w.B, w.H) + v.shape[2:]) for k, v in flat.items()}

@@ -77,8 +77,9 @@ def test_whole_pass_roofline(bench):
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
     assert r["achieved"] == pytest.approx(bench.alg_bytes(w) / 0.8e-3 / 1e9)
     assert r["frac"] == pytest.approx(r["achieved"] / 6531.9)
-    # two ranks, each with its own problem: twice the bytes in the same time
-    assert bench.whole_pass_roofline(w, 0.8, 2, 6531.9, "measured")["achieved"] == pytest.approx(2 * r["achieved"])
+    # two ranks, each with its own problem: the same fraction per GPU, twice the job's bytes
+    r2 = bench.whole_pass_roofline(w, 0.8, 2, 6531.9, "measured")
+    assert r2["frac"] == pytest.approx(r["frac"]) and r2["job_bytes"] == 2 * r["algorithmic_bytes"]
 
 
 def test_reference_arm_times_only_the_oracle(bench, monkeypatch):
