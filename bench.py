@@ -63,6 +63,9 @@ def parse():
                     help="head groups of vdn_forward_pipelined (tensor path); 0 = plain vdn_forward")
     ap.add_argument("--bridge", action="store_true",
                     help="read through the decay bridge (the window's decay carried onto both states)")
+    ap.add_argument("--shard", choices=["none", "heads"], default="none",
+                    help="heads: the ranks split one problem's (b, h) pairs (strong scaling) instead of each "
+                         "running a whole problem (weak scaling)")
     ap.add_argument("--stream", type=int, default=0,
                     help="time the causal streaming call instead: the clip as a live stream in segments of "
                          "this many frames (a multiple of the chunk; >= T for one segment)")
@@ -248,7 +251,7 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(w, gated=False):
+def workload_config(w, gated=False, shard="none", world=1):
     gates = "per-token write gates" if w.beta_per_token else "per-frame write gates"
     if gated:
         gates += ", gated RMSNorm readout epilogue"
@@ -258,7 +261,8 @@ def workload_config(w, gated=False):
                         f"chunk={w.chunk} anchors={w.anchors} {w.dtype} inputs, fp32 state, {gates}",
             "global_batch": w.B, "frames": w.B * w.T, "tokens": w.B * w.T * w.U,
             "l2": "inputs larger than L2 (Q+K+V bf16 = %.2f GB > 126 MB)" % (3 * w.B * w.H * w.T * w.U * w.d * 2 / 1e9),
-            "parallelism": "heads independent; one full problem per rank"}
+            "parallelism": (f"one problem's (b,h) pairs split over {world} ranks, no data-path collective"
+                            if shard == "heads" else "heads independent; one full problem per rank")}
 
 
 # ---------------------------------------------------------- the CUDA arm
@@ -301,7 +305,17 @@ def main():
         if world > 1:
             dist.barrier()
 
-    full = synth.generate_all(w)
+    # --shard heads: this rank's contiguous share of one problem's (b, h)
+    # pairs, laid out as one batch of that many heads (strong scaling);
+    # otherwise a whole problem per rank (weak scaling)
+    whole = w
+    if args.shard == "heads":
+        import dataclasses
+        pairs = vdist.shard_pairs(w.B, w.H, rank, world)
+        w = dataclasses.replace(w, B=1, H=len(pairs), name=f"{w.name}_pairs{len(pairs)}")
+        full = synth.generate_pairs(whole, pairs)
+    else:
+        full = synth.generate_all(w)
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     host = {}
     for k in ("Q", "K", "V", "Kx", "Vx"):
@@ -310,7 +324,7 @@ def main():
         host[k] = torch.from_numpy(np.ascontiguousarray(full[k])).pin_memory()
     if args.gated:
         # gate logits ~ N(0, 4) in the input dtype, RMSNorm weights ~ U(0.5, 1.5)
-        grng = np.random.default_rng(w.seed + 1000)
+        grng = np.random.default_rng(w.seed + 1000 + rank)
         host["gate"] = torch.from_numpy(
             (2.0 * grng.standard_normal((w.B, w.H, w.T, w.U, w.d), dtype=np.float32))).to(dt).pin_memory()
         host["norm_w"] = torch.from_numpy(grng.uniform(0.5, 1.5, (w.H, w.d)).astype(np.float32)).pin_memory()
@@ -379,8 +393,9 @@ def main():
     total_ms = event_ms(evs[0][first], evs[-1][last])
     total_ms = vdist.max_over_ranks(total_ms)  # the slowest rank's device time
     ms_per_step = total_ms / args.steps
-    frames_all = world * B * T
-    value = vdist.throughput(B * T, world, ms_per_step / 1e3)
+    # whole-job frames: every rank's own problem, or the one sharded problem
+    frames_all = whole.B * whole.T if args.shard == "heads" else world * B * T
+    value = frames_all / (ms_per_step / 1e3)
 
     # ---- end to end: pinned host inputs -> device -> vdn_forward -> O to host
     e2e = (e2e_measure(args, host, d, make_forward, stream, barrier, world, frames_all, dt, og)
@@ -392,10 +407,11 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "state_dtype": "f32",
-            "data": "synthetic", "config": workload_config(w, args.gated),
+            "scaling": "strong" if args.shard == "heads" else "weak", "vs_baseline": None, "dtype": "bf16",
+            "state_dtype": "f32", "data": "synthetic",
+            "config": workload_config(whole, args.gated, shard=args.shard, world=world),
             "tokens_per_s": value * U,
-            "hbm_frac_whole_pass": alg_bytes(w, args.gated) * world / (ms_per_step / 1e3) / (hbm_gbs * 1e9),
+            "hbm_frac_whole_pass": alg_bytes(w, args.gated) / (ms_per_step / 1e3) / (hbm_gbs * 1e9),
             "roofline_whole_pass": whole_pass_roofline(w, ms_per_step, world, hbm_gbs, peak_src, args.gated),
             "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
             "step_ms_min_max": [min(step_ms), max(step_ms)],
@@ -502,8 +518,9 @@ def stream_bench(args, w, s, d, dev, stream, barrier, rank, world, local):
     if seg < w.T and seg % w.chunk:
         raise SystemExit(f"--stream {seg}: segments must hold whole chunks of {w.chunk} frames")
     cuts = [(t0, min(seg, w.T - t0)) for t0 in range(0, w.T, seg)]
+    bridged = bool(getattr(w, "decay_bridge", False))
     shapes = {T: vdn.make_shape(w.B, w.H, T, w.U, w.d, w.n_text, w.chunk, w.anchors, w.dtype,
-                                beta_per_token=w.beta_per_token) for _, T in cuts}
+                                beta_per_token=w.beta_per_token, decay_bridge=bridged) for _, T in cuts}
     ws = vdn.workspace(max(vdn.vdn_stream_workspace_bytes(x) for x in shapes.values()), dev)
     tws = vdn.workspace(vdn.vdn_text_state_workspace_bytes(s), dev)
     info = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -511,13 +528,20 @@ def stream_bench(args, w, s, d, dev, stream, barrier, rank, world, local):
     outs = [(torch.empty((w.B, w.H, T, w.U, w.d), dtype=d["Q"].dtype, device=dev),
              torch.empty((w.B, w.H, shapes[T].C + 1, w.d, w.d), dtype=torch.float32, device=dev)) for _, T in cuts]
     S_T, S_prev, S_in = (torch.empty((w.B, w.H, w.d, w.d), dtype=torch.float32, device=dev) for _ in range(3))
+    # with the decay bridge: each segment's last-chunk decay product, carried
+    tails = [torch.empty((w.B, w.H, w.d), dtype=torch.float32, device=dev) for _ in range(2)]
 
     def step():
         vdn.vdn_text_state(s, d["Kx"], d["Vx"], d["beta_x"], S_T, tws, info)
-        sp, si = S_T, S_T
-        for (t0, T), x, (O, F) in zip(cuts, parts, outs):
-            vdn.vdn_stream_segment(shapes[T], x["Q"], x["K"], x["V"], x["beta"], x["alpha"], t0, sp, si, O, F, ws,
-                                   info)
+        sp, si, ap = S_T, S_T, None
+        for i, ((t0, T), x, (O, F)) in enumerate(zip(cuts, parts, outs)):
+            if bridged:
+                vdn.vdn_stream_segment_bridged(shapes[T], x["Q"], x["K"], x["V"], x["beta"], x["alpha"], t0, sp, si,
+                                               ap, O, F, tails[i & 1], ws, info)
+                ap = tails[i & 1]
+            else:
+                vdn.vdn_stream_segment(shapes[T], x["Q"], x["K"], x["V"], x["beta"], x["alpha"], t0, sp, si, O, F,
+                                       ws, info)
             C = shapes[T].C
             S_prev.copy_(F[:, :, C - 1])
             S_in.copy_(F[:, :, C])
@@ -556,7 +580,7 @@ def stream_bench(args, w, s, d, dev, stream, barrier, rank, world, local):
             "roofline": {"kernel": "whole stream step", "bound": "hbm", "achieved": frac * hbm_gbs,
                          "peak": hbm_gbs, "unit": "GB/s", "frac": frac, "traffic": None,
                          "peak_source": f"{peak_src} HBM copy bandwidth"},
-            "gpu_launches": ((3 if tensor_path else 2) + 5 * len(cuts)) * args.steps,
+            "gpu_launches": ((3 if tensor_path else 2) + (6 if bridged else 5) * len(cuts)) * args.steps,
             "clocks": clk.summary()}), flush=True)
     if world > 1:
         dist_destroy()
@@ -661,11 +685,13 @@ def roofline(w, stage_ms, hbm_gbs, peak_src, bf16_tflops=1607.7):
 
 
 def whole_pass_roofline(w, ms_per_step, world, hbm_gbs, peak_src, gated=False):
-    """The whole pass against HBM bandwidth: algorithmic bytes (Q, K, V read,
-    O written, gates and text) over the step time."""
-    achieved = alg_bytes(w, gated) * world / (ms_per_step / 1e3) / 1e9
+    """The whole pass against HBM bandwidth, per GPU: the algorithmic bytes of
+    one rank's work (Q, K, V read, O written, gates and text) over the step
+    time, against one GPU's peak; job_bytes is all ranks' bytes."""
+    achieved = alg_bytes(w, gated) / (ms_per_step / 1e3) / 1e9
     return {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s", "frac": achieved / hbm_gbs,
-            "algorithmic_bytes": alg_bytes(w, gated) * world, "peak_source": f"{peak_src} HBM copy bandwidth"}
+            "algorithmic_bytes": alg_bytes(w, gated), "job_bytes": alg_bytes(w, gated) * world,
+            "peak_source": f"{peak_src} HBM copy bandwidth, per GPU"}
 
 
 if __name__ == "__main__":
