@@ -150,17 +150,21 @@ vdn_status run_grams(const Geo &g, const void *K, const void *V, const float *be
 // F0: the forward state chunk 0 reads instead of F[0] (streaming), or nullptr
 // alpha: the decay gates when the readout goes through the decay bridge
 // (g.bridge), otherwise ignored.
+// bridge_prev: with F0 and the bridge, the decay product that chunk 0's
+// forward factor also carries (a stream segment), or nullptr.
 vdn_status run_readout(const Geo &g, const void *Q, const float *F, const float *G, void *O,
                        int32_t *info, cudaStream_t st, const OutGate *og = nullptr,
-                       const float *F0 = nullptr, const float *alpha = nullptr) {
+                       const float *F0 = nullptr, const float *alpha = nullptr,
+                       const float *bridge_prev = nullptr) {
   if (g.BH * g.T * g.U == 0) return VDN_OK;
   const float *bridge = g.bridge ? alpha : nullptr;
+  const float *bprev = g.bridge ? bridge_prev : nullptr;
   if (readout_tc_supported(g.in_dtype, g.out_dtype, g.D, g.U)) {
-    VDN_CUDA(launch_readout_tc(Q, F, G, O, g.BH, g.T, g.U, g.chunk, g.anchors, info, st, og, F0, bridge),
+    VDN_CUDA(launch_readout_tc(Q, F, G, O, g.BH, g.T, g.U, g.chunk, g.anchors, info, st, og, F0, bridge, bprev),
              "readout_tc");
   } else {
     VDN_CUDA(launch_readout_simt(Q, g.in_dtype, F, G, O, g.out_dtype, g.BH, g.T, g.U, g.chunk,
-                                 g.anchors, g.D, st, og, F0, bridge),
+                                 g.anchors, g.D, st, og, F0, bridge, bprev),
              "readout_simt");
   }
   return VDN_OK;
@@ -211,7 +215,7 @@ vdn_status run_text_state(const Geo &g, const void *Kx, const void *Vx, const fl
     // S_T is the injection of one "frame" made of the text tokens: invert,
     // then one J-chain step (B_x W_x) on the tensor cores.
     uint8_t *Wimg = (uint8_t *)(ws + L.wimg);
-    VDN_CUDA(launch_invert_tc(Ax, nullptr, Wimg, info, g.BH, st), "text invert");
+    VDN_CUDA(launch_invert_bsweep(Ax, nullptr, Wimg, info, g.BH, st, 0), "text invert");
     VDN_CUDA(launch_compose_tc(Wimg, Bx, Ax, nullptr, S_T, nullptr, nullptr, nullptr, g.BH, 1, 1, 0,
                                /*ndirs=*/1, /*j_transposed=*/false, info, st),
              "text injection");
@@ -450,7 +454,7 @@ vdn_status vdn_frame_invert(const vdn_shape *s, const float *A, float *W, int32_
   cudaStream_t st = (cudaStream_t)stream;
   VDN_CUDA(cudaMemsetAsync(info, 0, sizeof(int32_t), st), "memset info");
   if (tensor_path(g))
-    VDN_CUDA(launch_invert_tc(A, W, nullptr, info, g.BH * g.T, st), "invert");
+    VDN_CUDA(launch_invert_bsweep(A, W, nullptr, info, g.BH * g.T, st, 0), "invert");
   else
     VDN_CUDA(launch_invert_simt(A, W, nullptr, info, g.BH * g.T, g.D, st), "invert");
   return VDN_OK;
@@ -588,17 +592,27 @@ vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K, const v
 
 size_t vdn_stream_workspace_bytes(const vdn_shape *s) { return vdn_forward_workspace_bytes(s); }
 
-vdn_status vdn_stream_segment(const vdn_shape *s, const void *Q, const void *K, const void *V,
-                              const float *beta, const float *alpha, long long frame0, const float *S_prev,
-                              const float *S_in, void *O, float *F, void *workspace, size_t workspace_bytes,
-                              int32_t *info, vdn_stream_t stream) {
+}  // extern "C"
+
+namespace {
+// One stream segment; `bridged` reads through the decay bridge (shape flag
+// decay_bridge), with alpha_prev ([BH, d] or NULL = ones) the decay product of
+// the previous segment's last chunk and alpha_tail ([BH, d] or NULL) receiving
+// this segment's.
+vdn_status stream_segment(const vdn_shape *s, const void *Q, const void *K, const void *V, const float *beta,
+                          const float *alpha, long long frame0, const float *S_prev, const float *S_in,
+                          const float *alpha_prev, void *O, float *F, float *alpha_tail, void *workspace,
+                          size_t workspace_bytes, int32_t *info, vdn_stream_t stream, bool bridged) {
   g_err[0] = 0;
   Geo g;
   VDN_TRY(check_shape(s, &g));
   if (frame0 < 0 || frame0 % g.chunk != 0)
     return fail(VDN_ERR_INVALID, "frame0 = %lld is not a non-negative multiple of chunk = %d", frame0, g.chunk);
-  if (g.bridge)
-    return fail(VDN_ERR_UNSUPPORTED, "decay_bridge: a segment's first chunk would need the previous segment's alpha");
+  if (g.bridge && !bridged)
+    return fail(VDN_ERR_UNSUPPORTED,
+                "decay_bridge: a segment's first chunk needs the previous segment's decay product: use "
+                "vdn_stream_segment_bridged");
+  if (bridged && !g.bridge) return fail(VDN_ERR_INVALID, "vdn_stream_segment_bridged needs shape.decay_bridge = 1");
   // only the stream's first frame can be an anchor; there is no last one
   g.anchors = (s->anchors && frame0 == 0) ? 1 : 0;
   const bool frames = g.BH * g.T > 0;
@@ -612,6 +626,8 @@ vdn_status vdn_stream_segment(const vdn_shape *s, const void *Q, const void *K, 
   VDN_TRY(need(O, "O", frames && g.U > 0));
   VDN_TRY(need(F, "F", g.BH > 0));
   VDN_TRY(need(info, "info", true));
+  if ((alpha_prev && !aligned16(alpha_prev)) || (alpha_tail && !aligned16(alpha_tail)))
+    return fail(VDN_ERR_INVALID, "alpha_prev / alpha_tail not 16-byte aligned");
   const FwdLayout L = fwd_layout(g);
   VDN_TRY(need(workspace, "workspace", g.BH > 0));
   if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
@@ -643,12 +659,34 @@ vdn_status vdn_stream_segment(const vdn_shape *s, const void *Q, const void *K, 
       VDN_CUDA(launch_compose_simt(A, Bm, Mf, Jf, Mb, Jb, g.BH, g.T, g.chunk, g.D, st), "compose");
       VDN_CUDA(launch_scan_simt(Mf, Jf, nullptr, nullptr, S_in, F, nullptr, g.BH, g.C, g.D, 1, st, 1.f), "scan");
     }
-    VDN_TRY(run_readout(g, Q, F, nullptr, O, info, st, nullptr, S_prev));
+    VDN_TRY(run_readout(g, Q, F, nullptr, O, info, st, nullptr, S_prev, alpha, alpha_prev));
   } else {
     VDN_CUDA(launch_scan_simt(nullptr, nullptr, nullptr, nullptr, S_in, F, nullptr, g.BH, 0, g.D, 1, st, 1.f),
              "scan");
   }
+  if (bridged && alpha_tail)
+    VDN_CUDA(launch_bridge_tail(alpha, alpha_tail, g.BH, g.T, g.chunk, g.anchors, g.D, st), "bridge tail");
   return VDN_OK;
+}
+}  // namespace
+
+extern "C" {
+
+vdn_status vdn_stream_segment(const vdn_shape *s, const void *Q, const void *K, const void *V,
+                              const float *beta, const float *alpha, long long frame0, const float *S_prev,
+                              const float *S_in, void *O, float *F, void *workspace, size_t workspace_bytes,
+                              int32_t *info, vdn_stream_t stream) {
+  return stream_segment(s, Q, K, V, beta, alpha, frame0, S_prev, S_in, nullptr, O, F, nullptr, workspace,
+                        workspace_bytes, info, stream, false);
+}
+
+vdn_status vdn_stream_segment_bridged(const vdn_shape *s, const void *Q, const void *K, const void *V,
+                                      const float *beta, const float *alpha, long long frame0,
+                                      const float *S_prev, const float *S_in, const float *alpha_prev, void *O,
+                                      float *F, float *alpha_tail, void *workspace, size_t workspace_bytes,
+                                      int32_t *info, vdn_stream_t stream) {
+  return stream_segment(s, Q, K, V, beta, alpha, frame0, S_prev, S_in, alpha_prev, O, F, alpha_tail, workspace,
+                        workspace_bytes, info, stream, true);
 }
 
 vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *K, const void *V,

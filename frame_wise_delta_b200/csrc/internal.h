@@ -37,10 +37,18 @@ struct OutGate {
 // only) and F0 ([BH, d, d], may be null) replaces F[0] for chunk 0.
 // bridge_alpha ([BH, T, d], may be null): read through the decay bridge,
 // R_t = F[max(c - 1, 0)] Diag(pf_t) + G[min(c + 2, C)] Diag(pb_t).
+// bridge_prev ([BH, d], may be null): with F0 and the bridge, chunk 0's
+// forward factor also carries this decay product (a stream segment's window
+// starting in the previous segment's last chunk).
 cudaError_t launch_readout_simt(const void *Q, int in_dtype, const float *F, const float *G, void *O,
                                 int out_dtype, long long BH, int T, int U, int chunk, int anchors,
                                 int D, cudaStream_t st, const OutGate *og = nullptr,
-                                const float *F0 = nullptr, const float *bridge_alpha = nullptr);
+                                const float *F0 = nullptr, const float *bridge_alpha = nullptr,
+                                const float *bridge_prev = nullptr);
+// Decay product over the last chunk of each b*h's frames, anchors (mask as
+// above) counting as 1: out[bh][k] = prod alpha[bh][r][k], r = chunk (C - 1) .. T - 1.
+cudaError_t launch_bridge_tail(const float *alpha, float *out, long long BH, int T, int chunk, int anchors, int D,
+                               cudaStream_t st);
 
 // Tensor-core kernels (tcgen05 + TMA), bf16 inputs, d = 128.
 bool gram_tc_supported(int in_dtype, int D, int U);
@@ -55,7 +63,7 @@ bool readout_tc_supported(int in_dtype, int out_dtype, int D, int U);
 cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, void *O, long long BH,
                               int T, int U, int chunk, int anchors, int32_t *info, cudaStream_t st,
                               const OutGate *og = nullptr, const float *F0 = nullptr,
-                              const float *bridge_alpha = nullptr);
+                              const float *bridge_alpha = nullptr, const float *bridge_prev = nullptr);
 
 // W = (I + A)^{-1} per frame (CUDA cores); W fp32 and/or Wimg (hi/lo MMA
 // images of kImgBytes per frame, d = 128 only), each optional.
@@ -65,6 +73,11 @@ cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, voi
 // Pimg: null, or the P^{-1} tiles of launch_psweep (then the kernel skips its P sweeps)
 cudaError_t launch_invert_tc(const float *A, float *W, uint8_t *Wimg, int32_t *info, long long nframes,
                              cudaStream_t st, long long frame_base = 0, const uint8_t *Pimg = nullptr);
+// (I + A)^{-1} of fp32 128 x 128 frames by the blocked symmetric sweep with
+// tensor-core updates, as fp32 row-major W and/or hi/lo MMA images (either
+// may be null). A must be symmetric: the kernel reads its columns as rows.
+cudaError_t launch_invert_bsweep(const float *A, float *W, uint8_t *Wimg, int32_t *info, long long nframes,
+                                 cudaStream_t st, long long frame_base);
 // P^{-1} (leading 64 x 64 block of I + A) of every frame as a 16 KB hi/lo tile
 constexpr long long kPTileBytes = 16384;
 cudaError_t launch_psweep(const float *A, uint8_t *Pimg, int32_t *info, long long nframes, cudaStream_t st,

@@ -20,7 +20,9 @@
 // Decay bridge (optional, step (5)): frame t reads
 //   R_t = F[max(c-1,0)] Diag(pf_t) + G[min(c+2,C)] Diag(pb_t),
 // pf_t and pb_t the products of the decay gates over the window's frames
-// f0..t and t..f1; R is then rebuilt for every frame.
+// f0..t and t..f1; R is then rebuilt for every frame. In a stream segment
+// (F0 given) chunk 0's window starts in the previous segment's last chunk,
+// whose decay product (bprev) joins pf.
 //
 // Persistent kernel, one CTA per SM, 10 warps; each CTA walks a contiguous
 // range of frames so consecutive frames usually share a chunk and R is
@@ -60,6 +62,7 @@ struct ReadoutArgs {
   const float *G;   // optional (forward reads only when null)
   const float *F0;  // optional: per-b*h forward state chunk 0 reads instead of F[0]
   const float *bal; // optional: decay gates alpha [BH, T, 128]: read through the decay bridge
+  const float *bprev; // optional [BH, 128]: extra decay of chunk 0's forward factor (with F0)
   __nv_bfloat16 *O;
   int32_t *info;
   long long nframes;
@@ -285,6 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float x = __ldg(al + (long long)r * kD);
             if (!(((p.anchors & 1) && r == 0) || ((p.anchors & 2) && r == p.T - 1))) prod *= x;
           }
+          // a stream segment's chunk 0: its window starts in the previous segment
+          if (dir == 0 && c == 0 && p.F0 && p.bprev) prod *= __ldg(p.bprev + bh * kD + k);
           bridge_fb[dir * kD + k] = prod;
           asm volatile("bar.sync 3, 256;" ::: "memory");
         }
@@ -465,7 +470,8 @@ bool readout_tc_supported(int in_dtype, int out_dtype, int D, int U) {
 
 cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, void *O, long long BH,
                               int T, int U, int chunk, int anchors, int32_t *info, cudaStream_t st,
-                              const OutGate *og, const float *F0, const float *bridge_alpha) {
+                              const OutGate *og, const float *F0, const float *bridge_alpha,
+                              const float *bridge_prev) {
   const long long nframes = BH * T;
   if (nframes <= 0) return cudaSuccess;
   CUtensorMap tmQ, tmO, tmG;
@@ -478,7 +484,7 @@ cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, voi
   if (e != cudaSuccess) return e;
   const int sms = device_sm_count();
   const long long grid = nframes < sms ? nframes : sms;
-  ReadoutArgs a{F, G, F0, bridge_alpha, (__nv_bfloat16 *)O, info, nframes, T, U, chunk, anchors,
+  ReadoutArgs a{F, G, F0, bridge_alpha, bridge_prev, (__nv_bfloat16 *)O, info, nframes, T, U, chunk, anchors,
                 (T + chunk - 1) / chunk, (U + kNT - 1) / kNT,
                 gated ? og->w : nullptr, gated ? og->eps : 0.f, gated ? og->H : 1};
   readout_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(tmQ, tmO, tmG, a);

@@ -345,7 +345,7 @@ template <int D, typename Tin, typename Tout>
 __global__ void __launch_bounds__(kThreads) readout_simt_kernel(
     const Tin *__restrict__ Q, const float *__restrict__ F, const float *__restrict__ G,
     Tout *__restrict__ O, int T, int U, int chunk, int anchors, int C, OutGate og,
-    const float *__restrict__ F0, const float *__restrict__ bal) {
+    const float *__restrict__ F0, const float *__restrict__ bal, const float *__restrict__ bprev) {
   constexpr int TU = 64;
   constexpr int RB = D / 16;
   constexpr int LD = D + 1;
@@ -380,6 +380,7 @@ __global__ void __launch_bounds__(kThreads) readout_simt_kernel(
         if (!(((anchors & 1) && r == 0) || ((anchors & 2) && r == T - 1))) pf *= al[(long long)r * D];
       for (int r = t; r <= f1; ++r)
         if (!(((anchors & 1) && r == 0) || ((anchors & 2) && r == T - 1))) pb *= al[(long long)r * D];
+      if (c == 0 && F0 && bprev) pf *= bprev[bh * D + k];  // a stream segment's window starts before it
       pfb[k] = pf;
       pfb[D + k] = pb;
     }
@@ -488,10 +489,26 @@ cudaError_t scan_d(const float *Mf, const float *Jf, const float *Mb, const floa
   return cudaGetLastError();
 }
 
+// Decay product over the last chunk of each b*h's frames (anchors count as
+// 1): what the next stream segment's first chunk finds at the start of its
+// window. One thread per (b*h, channel); T = 0 leaves the empty product 1.
+__global__ void bridge_tail_kernel(const float *__restrict__ alpha, float *__restrict__ out, long long n, int T,
+                                   int chunk, int anchors, int D) {
+  const long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (e >= n) return;
+  const long long bh = e / D;
+  const int k = (int)(e % D);
+  const int C = (T + chunk - 1) / chunk;
+  float p = 1.f;
+  for (int r = C > 0 ? chunk * (C - 1) : 0; r < T; ++r)
+    if (!(((anchors & 1) && r == 0) || ((anchors & 2) && r == T - 1))) p *= alpha[(bh * T + r) * D + k];
+  out[e] = p;
+}
+
 template <int D, typename Tin, typename Tout>
 cudaError_t readout_dt(const void *Q, const float *F, const float *G, void *O, long long BH, int T,
                        int U, int chunk, int anchors, cudaStream_t st, const OutGate &og, const float *F0,
-                       const float *bal) {
+                       const float *bal, const float *bprev) {
   const int C = (T + chunk - 1) / chunk;
   const size_t smem = (size_t)(D * (D + 1) + 64 * D + 2 * D) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(readout_simt_kernel<D, Tin, Tout>,
@@ -499,22 +516,23 @@ cudaError_t readout_dt(const void *Q, const float *F, const float *G, void *O, l
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)(BH * T), (unsigned)((U + 63) / 64));
   readout_simt_kernel<D, Tin, Tout><<<grid, kThreads, smem, st>>>(
-      (const Tin *)Q, F, G, (Tout *)O, T, U, chunk, anchors, C, og, F0, bal);
+      (const Tin *)Q, F, G, (Tout *)O, T, U, chunk, anchors, C, og, F0, bal, bprev);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t readout_d(const void *Q, int in_dtype, const float *F, const float *G, void *O,
                       int out_dtype, long long BH, int T, int U, int chunk, int anchors,
-                      cudaStream_t st, const OutGate &og, const float *F0, const float *bal) {
+                      cudaStream_t st, const OutGate &og, const float *F0, const float *bal,
+                      const float *bprev) {
   if (in_dtype == VDN_BF16) {
     if (out_dtype == VDN_BF16)
-      return readout_dt<D, __nv_bfloat16, __nv_bfloat16>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0, bal);
-    return readout_dt<D, __nv_bfloat16, float>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0, bal);
+      return readout_dt<D, __nv_bfloat16, __nv_bfloat16>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0, bal, bprev);
+    return readout_dt<D, __nv_bfloat16, float>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0, bal, bprev);
   }
   if (out_dtype == VDN_BF16)
-    return readout_dt<D, float, __nv_bfloat16>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0, bal);
-  return readout_dt<D, float, float>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0, bal);
+    return readout_dt<D, float, __nv_bfloat16>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0, bal, bprev);
+  return readout_dt<D, float, float>(Q, F, G, O, BH, T, U, chunk, anchors, st, og, F0, bal, bprev);
 }
 
 }  // namespace
@@ -564,12 +582,20 @@ cudaError_t launch_scan_simt(const float *Mf, const float *Jf, const float *Mb, 
 cudaError_t launch_readout_simt(const void *Q, int in_dtype, const float *F, const float *G, void *O,
                                 int out_dtype, long long BH, int T, int U, int chunk, int anchors,
                                 int D, cudaStream_t st, const OutGate *og, const float *F0,
-                                const float *bridge_alpha) {
+                                const float *bridge_alpha, const float *bridge_prev) {
   if (BH <= 0 || T <= 0 || U <= 0) return cudaSuccess;
   const OutGate none{nullptr, nullptr, 0.f, 1};
   const OutGate &g = og ? *og : none;
   VDN_DISPATCH_D(D, readout_d<DD_>(Q, in_dtype, F, G, O, out_dtype, BH, T, U, chunk, anchors, st, g, F0,
-                                   bridge_alpha))
+                                   bridge_alpha, bridge_prev))
+}
+
+cudaError_t launch_bridge_tail(const float *alpha, float *out, long long BH, int T, int chunk, int anchors, int D,
+                               cudaStream_t st) {
+  if (BH <= 0) return cudaSuccess;
+  const long long n = BH * D;
+  bridge_tail_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(alpha, out, n, T, chunk, anchors, D);
+  return cudaGetLastError();
 }
 
 }  // namespace vdn

@@ -91,6 +91,7 @@ _SIGS = {
     "vdn_chunk_readout_bridged": [_P] * 9,
     "vdn_selftest_wait": [_P, _P],
     "vdn_stream_segment": [_P] * 6 + [ctypes.c_longlong] + [_P] * 5 + [ctypes.c_size_t, _P, _P],
+    "vdn_stream_segment_bridged": [_P] * 6 + [ctypes.c_longlong] + [_P] * 7 + [ctypes.c_size_t, _P, _P],
 }
 
 
@@ -281,6 +282,17 @@ def vdn_stream_segment(s, Q, K, V, beta, alpha, frame0, S_prev, S_in, O, F, work
                                     _ptr(info), _stream(stream)))
 
 
+def vdn_stream_segment_bridged(s, Q, K, V, beta, alpha, frame0, S_prev, S_in, alpha_prev, O, F, alpha_tail,
+                               workspace, info, stream=None):
+    """One stream segment read through the decay bridge (see vdn.h); alpha_prev
+    None for the stream's first segment, alpha_tail None when not needed."""
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().vdn_stream_segment_bridged(_shp(s), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(alpha),
+                                            int(frame0), _ptr(S_prev), _ptr(S_in), _ptr(alpha_prev), _ptr(O),
+                                            _ptr(F), _ptr(alpha_tail), _ptr(workspace), nbytes, _ptr(info),
+                                            _stream(stream)))
+
+
 def vdn_selftest_wait(info, stream=None):
     """Self-test of the bounded pipeline waits (see vdn.h): *info becomes VDN_INFO_TIMEOUT."""
     _check(lib().vdn_selftest_wait(_ptr(info), _stream(stream)))
@@ -318,10 +330,18 @@ class Stream:
         self.S_prev = S_T.clone()
         self.S_in = S_T.clone()
         self.frame0 = 0
+        # with the decay bridge: the last chunk's decay product, carried too
+        self.alpha_tail = (torch.ones((s.B, s.H, s.dk), dtype=torch.float32, device=device)
+                           if s.decay_bridge else None)
 
     def __call__(self, Q, K, V, beta, alpha, stream=None):
-        vdn_stream_segment(self.s, Q, K, V, beta, alpha, self.frame0, self.S_prev, self.S_in, self.O, self.F,
-                           self.ws, self.info, stream)
+        if self.s.decay_bridge:
+            prev = None if self.frame0 == 0 else self.alpha_tail.clone()
+            vdn_stream_segment_bridged(self.s, Q, K, V, beta, alpha, self.frame0, self.S_prev, self.S_in, prev,
+                                       self.O, self.F, self.alpha_tail, self.ws, self.info, stream)
+        else:
+            vdn_stream_segment(self.s, Q, K, V, beta, alpha, self.frame0, self.S_prev, self.S_in, self.O,
+                               self.F, self.ws, self.info, stream)
         C = self.s.C
         if C > 0:
             self.S_prev.copy_(self.F[:, :, C - 1])

@@ -367,9 +367,10 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
  * workspace: at least vdn_stream_workspace_bytes(s) bytes, 256-byte aligned.
  * Errors: VDN_ERR_INVALID for a frame0 that is negative or not a multiple of
  * the chunk, and as for vdn_forward; VDN_ERR_UNSUPPORTED with
- * shape.decay_bridge (the bridge of a segment's first chunk would need the
- * previous segment's decay gates). Same kernels as vdn_forward (the
- * tensor-core path for bf16 d = 128), run in one direction.
+ * shape.decay_bridge (the bridge of a segment's first chunk needs the
+ * previous segment's decay product: vdn_stream_segment_bridged takes it).
+ * Same kernels as vdn_forward (the tensor-core path for bf16 d = 128), run in
+ * one direction.
  */
 size_t vdn_stream_workspace_bytes(const vdn_shape *s);
 vdn_status vdn_stream_segment(const vdn_shape *s, const void *Q, const void *K,
@@ -378,6 +379,32 @@ vdn_status vdn_stream_segment(const vdn_shape *s, const void *Q, const void *K,
                               void *O, float *F, void *workspace,
                               size_t workspace_bytes, int32_t *info,
                               vdn_stream_t stream);
+
+/*
+ * A stream segment read through the decay bridge ("Method steps" step (5):
+ * the state read at a window boundary is carried on through prod alpha_r),
+ * forward half: frame t of chunk c reads
+ *   R_t = F_{c-1} Diag(prod_{r=f0..t} alpha_r),
+ * f0 the first frame of chunk c - 1, an anchor frame's alpha counting as 1.
+ * The window of the segment's chunk 0 starts in the previous segment's last
+ * chunk, so that chunk's decay product enters its factor:
+ *   R_t = S_prev Diag(alpha_prev * prod_{r=0..t} alpha_r).
+ * Needs shape.decay_bridge = 1. Arguments as for vdn_stream_segment, plus:
+ * In : alpha_prev [B,H,dk] float32: the previous segment's alpha_tail; NULL
+ *      (all ones) for the stream's first segment.
+ * Out: alpha_tail [B,H,dk] float32 (may be NULL): prod alpha_r over this
+ *      segment's last chunk, to pass as the next segment's alpha_prev.
+ * Errors: as for vdn_stream_segment; VDN_ERR_INVALID without
+ * shape.decay_bridge.
+ */
+vdn_status vdn_stream_segment_bridged(const vdn_shape *s, const void *Q,
+                                      const void *K, const void *V,
+                                      const float *beta, const float *alpha,
+                                      long long frame0, const float *S_prev,
+                                      const float *S_in, const float *alpha_prev,
+                                      void *O, float *F, float *alpha_tail,
+                                      void *workspace, size_t workspace_bytes,
+                                      int32_t *info, vdn_stream_t stream);
 
 /*
  * Self-test of the bounded pipeline waits that every tensor-core kernel uses:

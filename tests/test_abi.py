@@ -233,3 +233,19 @@ def test_noalloc_applies_the_same_shape_rules(L, kw):
         s = _shape()
         setattr(s, flag, 5)
         assert L.vdn_text_state_noalloc(_p(s), 16, 16, 16, 16, 16, None) == vdn.VDN_ERR_INVALID
+
+
+def test_bridged_stream_segment_checks(L):
+    args = lambda s, frame0: (_p(s), 16, 16, 16, 16, 16, frame0, 16, 16, None, 16, 16, None, 16, 1 << 30, 16, None)
+    # needs the decay_bridge flag
+    assert L.vdn_stream_segment_bridged(*args(_shape(), 0)) == vdn.VDN_ERR_INVALID
+    assert "decay_bridge" in vdn.vdn_last_error()
+    s = _shape()
+    s.decay_bridge = 1
+    assert L.vdn_stream_segment_bridged(*args(s, 3)) == vdn.VDN_ERR_INVALID  # frame0 not a chunk multiple
+    assert "frame0" in vdn.vdn_last_error()
+    # misaligned carried product
+    a = list(args(s, 5))
+    a[9] = 18
+    assert L.vdn_stream_segment_bridged(*a) == vdn.VDN_ERR_INVALID
+    assert "alpha_prev" in vdn.vdn_last_error()

@@ -198,3 +198,99 @@ def test_full_size_h3_stream(pairs):
         assert ef <= STATE_GUARD and eo <= OUT_GUARD["bf16"], (ef, eo)
     del dev
     torch.cuda.empty_cache()
+
+
+# ------------------------------------------------ decay bridge in segments
+def _bridged_segment(w, dev, frame0, S_prev, S_in, alpha_prev, T=None, t0=0):
+    T = w.T if T is None else T
+    s = vdn.make_shape(w.B, w.H, T, w.U, w.d, w.n_text, w.chunk, w.anchors, w.dtype,
+                       beta_per_token=w.beta_per_token, decay_bridge=True)
+    ws = vdn.workspace(vdn.vdn_stream_workspace_bytes(s))
+    info = torch.ones(1, dtype=torch.int32, device="cuda")
+    dt = dev["Q"].dtype
+    O = torch.full((w.B, w.H, T, w.U, w.d), float("nan"), dtype=dt, device="cuda")
+    F = torch.full((w.B, w.H, s.C + 1, w.d, w.d), float("nan"), device="cuda")
+    tail = torch.full((w.B, w.H, w.d), float("nan"), device="cuda")
+    sl = slice(t0, t0 + T)
+    part = {k: dev[k][:, :, sl].contiguous() for k in ("Q", "K", "V", "beta", "alpha")}
+    vdn.vdn_stream_segment_bridged(s, part["Q"], part["K"], part["V"], part["beta"], part["alpha"], frame0,
+                                   S_prev, S_in, alpha_prev, O, F, tail, ws, info)
+    torch.cuda.synchronize()
+    assert int(info.item()) == 0
+    return O, F, tail
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+@pytest.mark.parametrize("first", [True, False], ids=["frame0", "later"])
+def test_bridged_segment_matches_oracle(w, first):
+    full = synth.generate_all(w)
+    dev = device_inputs(w, full)
+    ST, S_prev, S_in = _states(w, full, w.seed + 1)
+    rng = np.random.default_rng(w.seed + 2)
+    a_prev = rng.uniform(0.5, 1.0, (w.B, w.H, w.d))
+    if first:
+        S_prev = S_in = ST
+        a_prev = np.ones_like(a_prev)
+    frame0 = 0 if first else 3 * w.chunk
+    anchor_first = bool(w.anchors) and first
+    O, F, tail = _bridged_segment(w, dev, frame0, to_dev(S_prev), to_dev(S_in), None if first else to_dev(a_prev))
+    tol = TOL[w.dtype]
+    for b in range(w.B):
+        for h in range(w.H):
+            Or, Fr = oracle.stream_segment(full["Q"][b, h], full["K"][b, h], full["V"][b, h], full["beta"][b, h],
+                                           full["alpha"][b, h], S_prev[b, h], S_in[b, h], w.chunk, anchor_first,
+                                           bridge=True, alpha_prev=a_prev[b, h])
+            eo, ef = rel(O[b, h], Or), rel(F[b, h], Fr)
+            et = rel(tail[b, h], oracle.stream_bridge_tail(full["alpha"][b, h], w.chunk, anchor_first))
+            print(f"{w.name} bridged frame0={frame0} b{b} h{h}: O {eo:.2e} F {ef:.2e} tail {et:.2e}")
+            assert eo <= tol and ef <= tol and et <= 1e-6
+            assert ef <= STATE_GUARD and eo <= OUT_GUARD[w.dtype]
+    assert torch.isfinite(O.float()).all()
+
+
+@pytest.mark.parametrize("w", [TC, F32_D32], ids=lambda w: w.name)
+def test_bridged_segments_equal_one_call(w):
+    """A bridged stream cut at chunk boundaries, carrying (F[C-1], F[C]) and
+    the last chunk's decay product, gives the outputs of a single call."""
+    w = dataclasses.replace(w, name=w.name + "_bridged_long", T=22)
+    full = synth.generate_all(w)
+    dev = device_inputs(w, full)
+    ST, _, _ = _states(w, full, w.seed)
+    S = to_dev(ST)
+    O, F, _ = _bridged_segment(w, dev, 0, S, S, None)
+    Os = []
+    S_prev, S_in, a_prev = S, S, None
+    for t0, T in ((0, 10), (10, 5), (15, 7)):
+        Oi, Fi, tail = _bridged_segment(w, dev, t0, S_prev, S_in, a_prev, T=T, t0=t0)
+        Os.append(Oi)
+        C = Fi.shape[2] - 1
+        S_prev, S_in, a_prev = Fi[:, :, C - 1].contiguous(), Fi[:, :, C].contiguous(), tail
+    # the segments' chunks run the same kernels on the same inputs, except
+    # the bridge factor of each segment's chunk 0, formed from the carried
+    # product instead of in one loop: equal to fp32 rounding
+    e = rel(torch.cat(Os, dim=2), O.double().cpu().numpy())
+    print(f"{w.name}: bridged segments vs one call {e:.2e}")
+    assert e <= (1e-6 if w.dtype == "f32" else 4e-3)
+
+
+def test_stream_class_carries_the_bridge():
+    w = dataclasses.replace(TC, name="stream_tc_class_bridged", T=20, anchors=1)
+    full = synth.generate_all(w)
+    dev = device_inputs(w, full)
+    ST, _, _ = _states(w, full, w.seed)
+    seg = vdn.make_shape(w.B, w.H, 10, w.U, w.d, w.n_text, w.chunk, w.anchors, w.dtype, decay_bridge=True)
+    st = vdn.Stream(seg, to_dev(ST))
+    outs = []
+    for t0 in (0, 10):
+        part = {k: dev[k][:, :, t0:t0 + 10].contiguous() for k in ("Q", "K", "V", "beta", "alpha")}
+        outs.append(st(part["Q"], part["K"], part["V"], part["beta"], part["alpha"]).clone())
+    torch.cuda.synchronize()
+    assert int(st.info.item()) == 0
+    O = torch.cat(outs, dim=2)
+    for b in range(w.B):
+        for h in range(w.H):
+            Or, _ = oracle.stream_segment(full["Q"][b, h], full["K"][b, h], full["V"][b, h], full["beta"][b, h],
+                                          full["alpha"][b, h], ST[b, h], ST[b, h], w.chunk, True, bridge=True)
+            e = rel(O[b, h], Or)
+            print(f"stream class bridged b{b} h{h}: O {e:.2e}")
+            assert e <= OUT_GUARD["bf16"]
