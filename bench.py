@@ -415,6 +415,8 @@ def main():
             "roofline_whole_pass": whole_pass_roofline(w, ms_per_step, world, hbm_gbs, peak_src, args.gated),
             "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
             "step_ms_min_max": [min(step_ms), max(step_ms)],
+            "step_ms_median": statistics.median(step_ms),
+            "step_ms_p90": sorted(step_ms)[int(0.9 * (len(step_ms) - 1))],
             "roofline": roof,
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
