@@ -287,7 +287,7 @@ __global__ void __launch_bounds__((TOKB || PSW) ? 320 : 192, 1)
       const bool ok = X.run(cb, rg, cg, [nb] { asm volatile("bar.sync %0, 64;" ::"r"(nb) : "memory"); });
       if (st == 0) bulk_wait_read<0>();  // the previous P^{-1} tile has left
       asm volatile("bar.sync %0, 64;" ::"r"(nb) : "memory");
-      store_swept_tile(X, pt, rg, cg);
+      store_swept_tile<true>(X, pt, rg, cg);
       fence_proxy_async_smem();
       asm volatile("bar.sync %0, 64;" ::"r"(nb) : "memory");
       if (st == 0) {

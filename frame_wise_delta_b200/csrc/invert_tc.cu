@@ -12,8 +12,12 @@
 // P^{-1} and S^{-1} come from the symmetric sweep on the CUDA cores (a quarter
 // of the full sweep's work); the products X^T = Q^T P^{-1}, Q^T X, Y = X S^{-1},
 // Y^T = S^{-1} X^T and Y X^T run as tcgen05 MMAs (M = 128, N = 64, K = 64) on
-// hi/lo bf16 splits (hi*hi + hi*lo + lo*hi, ~fp32 accuracy), accumulating in
-// TMEM. A pivot of P or S that is not positive (G not positive definite) is
+// hi/lo splits (hi*hi + hi*lo + lo*hi), accumulating in TMEM. The two products
+// that form S take fp16 parts (~2^-22 of each operand): when I + A is
+// ill-conditioned S is much smaller than R and Q^T X, and the subtraction
+// magnifies their error. The last three take bf16 parts (~2^-17), the format
+// of the output image: their results are at most 2 in norm and meet no such
+// cancellation. A pivot of P or S that is not positive (G not positive definite) is
 // reported in *info like the sweep does.
 //
 // One CTA of 128 threads works through frames (persistent), four CTAs per SM:
@@ -41,9 +45,11 @@ constexpr int kSlotXT = 2 * kTile;      // X^T image
 constexpr int kSlotMisc = 3 * kTile;    // sweep exchange buffer, barrier, TMEM address, abort flag
 constexpr size_t kSmemBytes = 1024 + kSlotMisc + 2 * 2 * 64 * 4 + 64;
 constexpr uint32_t kTmemCols = 128;     // two 64-column accumulators
-constexpr uint32_t kIdesc = idesc_bf16_f32(128, 64, false, false);    // A, B K-major
-constexpr uint32_t kIdescAmn = idesc_bf16_f32(128, 64, true, false);  // A MN-major
-constexpr uint32_t kIdescBmn = idesc_bf16_f32(128, 64, false, true);  // B MN-major
+// X^T = Q^T P^{-1} and Q^T X multiply fp16 hi/lo tiles (A, B K-major); the
+// products after the S sweep multiply bf16 hi/lo tiles (one operand MN-major)
+constexpr uint32_t kIdescF16 = idesc_f16_f32(128, 64, false, false);
+constexpr uint32_t kIdescAmn = idesc_bf16_f32(128, 64, true, false);
+constexpr uint32_t kIdescBmn = idesc_bf16_f32(128, 64, false, true);
 
 // element (row, k) of a 64-row K-major 128-byte-swizzled tile (k < 64)
 __device__ __forceinline__ uint32_t tile_off(int row, int k) { return kmajor_sw128_offset(row, k, 64); }
@@ -52,19 +58,28 @@ __device__ __forceinline__ uint32_t tile_off(int row, int k) { return kmajor_sw1
 __device__ __forceinline__ uint32_t chunk_pos(int r, int c) { return (uint32_t)((c ^ (r & 7)) << 4); }
 
 // hi and lo 16-byte chunks of 8 values (times sign)
+template <bool F16>
 __device__ __forceinline__ void pack8(const float *v, float sign, uint4 &h, uint4 &l) {
-  split_bf16x2(sign * v[0], sign * v[1], h.x, l.x);
-  split_bf16x2(sign * v[2], sign * v[3], h.y, l.y);
-  split_bf16x2(sign * v[4], sign * v[5], h.z, l.z);
-  split_bf16x2(sign * v[6], sign * v[7], h.w, l.w);
+  if constexpr (F16) {
+    split_f16x2(sign * v[0], sign * v[1], h.x, l.x);
+    split_f16x2(sign * v[2], sign * v[3], h.y, l.y);
+    split_f16x2(sign * v[4], sign * v[5], h.z, l.z);
+    split_f16x2(sign * v[6], sign * v[7], h.w, l.w);
+  } else {
+    split_bf16x2(sign * v[0], sign * v[1], h.x, l.x);
+    split_bf16x2(sign * v[2], sign * v[3], h.y, l.y);
+    split_bf16x2(sign * v[4], sign * v[5], h.z, l.z);
+    split_bf16x2(sign * v[6], sign * v[7], h.w, l.w);
+  }
 }
 
 // Row r of a hi/lo tile (64 values) written from one thread.
+template <bool F16>
 __device__ __forceinline__ void tile_row_store(uint8_t *tile, int r, const float *v, float sign) {
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     uint4 h, l;
-    pack8(v + 8 * c, sign, h, l);
+    pack8<F16>(v + 8 * c, sign, h, l);
     const uint32_t o = (uint32_t)r * 128u + chunk_pos(r, c);
     *reinterpret_cast<uint4 *>(tile + o) = h;
     *reinterpret_cast<uint4 *>(tile + kHalf + o) = l;
@@ -104,7 +119,15 @@ __device__ __forceinline__ void handoff_wait(int id) {
 constexpr int kBarSweep = 1, kBarEpi = 2;           // within each warp pair
 constexpr int kBarPiReady = 3, kBarTReady = 4, kBarSiReady = 5, kBarPiFree = 6;
 
-// v (+)= row r of a hi/lo tile, decoded to fp32
+// the two values of a bf16x2 or fp16x2 word as fp32
+template <bool F16>
+__device__ __forceinline__ float2 unpack2(uint32_t w) {
+  if constexpr (F16) return __half22float2(*reinterpret_cast<const __half2 *>(&w));
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// v (+)= row r of a hi/lo tile (fp16 or bf16 parts), decoded to fp32
+template <bool F16>
 __device__ __forceinline__ void tile_row_add(const uint8_t *tile, int r, float (&v)[64], bool add) {
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
@@ -114,8 +137,8 @@ __device__ __forceinline__ void tile_row_add(const uint8_t *tile, int r, float (
     const uint32_t hw[4] = {h.x, h.y, h.z, h.w}, lw[4] = {l.x, l.y, l.z, l.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float x0 = __uint_as_float(hw[q] << 16) + __uint_as_float(lw[q] << 16);
-      const float x1 = __uint_as_float(hw[q] & 0xFFFF0000u) + __uint_as_float(lw[q] & 0xFFFF0000u);
+      const float2 hh = unpack2<F16>(hw[q]), ll = unpack2<F16>(lw[q]);
+      const float x0 = hh.x + ll.x, x1 = hh.y + ll.y;
       v[8 * c + 2 * q] = add ? v[8 * c + 2 * q] + x0 : x0;
       v[8 * c + 2 * q + 1] = add ? v[8 * c + 2 * q + 1] + x1 : x1;
     }
@@ -161,7 +184,7 @@ __global__ void __launch_bounds__(kSweepThreads) psweep_kernel(const float *__re
       X.at(a, b) = __ldg(Af + r * 128 + c) + (r == c ? 1.f : 0.f);
     }
   const bool ok = X.run(cbuf, rg, cg, [] { __syncthreads(); });
-  store_swept_tile(X, tile, rg, cg);
+  store_swept_tile<true>(X, tile, rg, cg);
   fence_proxy_async_smem();
   __syncthreads();
   if (tid == 0) {
@@ -226,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         ok = X.run(cbuf, rg, cg, [] { bar_named(kBarSweep); });
         if (!first) handoff_wait(kBarPiFree);  // the previous frame's last product has read P^{-1}
         first = false;
-        store_swept_tile(X, pi_t, rg, cg);
+        store_swept_tile<true>(X, pi_t, rg, cg);
         fence_proxy_async_smem();
         handoff_arrive(kBarPiReady);
       }
@@ -249,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           X.at(a, b) -= stage[r * 64 + (((c >> 2) ^ (r & 15)) << 2) + (c & 3)];
         }
       ok = X.run(cbuf, rg, cg, [] { bar_named(kBarSweep); }) && ok;
-      store_swept_tile(X, s0, rg, cg);
+      store_swept_tile<false>(X, s0, rg, cg);
       fence_proxy_async_smem();
       handoff_arrive(kBarSiReady);
       if (!ok && tid == 0) report_frame_failure(info, frame_base + f);
@@ -288,8 +311,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const int r = it * 4 + (i >> 4), c4 = i & 15;
         const float4 x = __ldg(reinterpret_cast<const float4 *>(Af + (64 + r) * 128 + 4 * c4));
         uint2 h, l;
-        split_bf16x2(x.x, x.y, h.x, l.x);
-        split_bf16x2(x.z, x.w, h.y, l.y);
+        split_f16x2(x.x, x.y, h.x, l.x);
+        split_f16x2(x.z, x.w, h.y, l.y);
         const uint32_t o = tile_off(r, 4 * c4);
         *reinterpret_cast<uint2 *>(s0 + o) = h;
         *reinterpret_cast<uint2 *>(s0 + kHalf + o) = l;
@@ -303,16 +326,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         handoff_wait(kBarPiReady);
       }
       // X^T = Q^T P^{-1}
-      issue([&] { mma_hilo(acc0, a_s0 - kHalf, a_s0, a_pi, a_pi + kHalf, false, false, 16, kIdesc); });
+      issue([&] { mma_hilo(acc0, a_s0 - kHalf, a_s0, a_pi, a_pi + kHalf, false, false, 16, kIdescF16); });
       float v[64];
       wait_mma();
       tmem_row64(acc0 + lane_off, v);
-      tile_row_store(xt, i, v, 1.f);
+      tile_row_store<true>(xt, i, v, 1.f);
       fence_proxy_async_smem();
       tc_fence_before();
       bar_named(kBarEpi);
       // Q^T X (B = Q read from the Q^T tile K-major), staged in fp32 for the S sweep
-      issue([&] { mma_hilo(acc0, a_xt - kHalf, a_xt, a_s0, a_s0 + kHalf, false, false, 16, kIdesc); });
+      issue([&] { mma_hilo(acc0, a_xt - kHalf, a_xt, a_s0, a_s0 + kHalf, false, false, 16, kIdescF16); });
       wait_mma();
       tmem_row64(acc0 + lane_off, v);
 #pragma unroll
@@ -327,6 +350,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         bulk_prefetch_l2(Af + gridDim.x * 128LL * 128 + 64 * 128, 64 * 128 * 4);
         if (PRE_P) bulk_prefetch_l2(Pimg + (f + gridDim.x) * (long long)kTile, kTile);
       }
+      // the X^T tile in bf16 parts for the products after the sweep (its
+      // fp16 form has served the two products the Schur complement needs)
+      tile_row_add<true>(xt, i, v, false);
+      tile_row_store<false>(xt, i, v, 1.f);
+      fence_proxy_async_smem();
       handoff_wait(kBarSiReady);
       issue([&] {
         // Y = X S^{-1}: A = X, the X^T tile read MN-major as the second 64-row
@@ -340,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       if (Wf) {
         w_row_store(Wf, 1, i, v, -1.f);  // top-right block: -Y
         float u[64];
-        tile_row_add(s0, i, u, false);
+        tile_row_add<false>(s0, i, u, false);
         w_row_store(Wf, 1, 64 + i, u, 1.f);  // bottom-right block: S^{-1}
       }
       // The image is written as four 64 x 64 blocks by bulk copies of the
@@ -353,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         bulk_wait_read<0>();
       }
       bar_named(kBarEpi);  // the S^{-1} tile has been read; it becomes -Y
-      tile_row_store(s0, i, v, -1.f);  // -Y: the top-right block and A of the last product
+      tile_row_store<false>(s0, i, v, -1.f);  // -Y: the top-right block and A of the last product
       fence_proxy_async_smem();
       tc_fence_before();
       bar_named(kBarEpi);
@@ -369,12 +397,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       // top-left block: P^{-1} - (-Y) X^T, written over this row of the P^{-1} tile
 #pragma unroll
       for (int e = 0; e < 64; ++e) v[e] = -v[e];
-      tile_row_add(pi_t, i, v, true);
-      tile_row_store(pi_t, i, v, 1.f);
+      tile_row_add<true>(pi_t, i, v, true);
+      tile_row_store<false>(pi_t, i, v, 1.f);
       if (Wf) w_row_store(Wf, 0, i, v, 1.f);
       // bottom-left block: -Y^T, into the X^T tile (the last product is done)
       tmem_row64(acc1 + lane_off, v);
-      tile_row_store(xt, i, v, -1.f);
+      tile_row_store<false>(xt, i, v, -1.f);
       if (Wf) w_row_store(Wf, 0, 64 + i, v, -1.f);
       fence_proxy_async_smem();
       bar_named(kBarEpi);

@@ -23,12 +23,14 @@ OUT_GUARD = {"f32": 1e-4, "bf16": 3e-3}
 
 def state_guard(w) -> float:
     """The state guard of a workload. Near-duplicate keys (cosine 0.99) make
-    cond(I + A_t) ~ 2.4e2, which amplifies rounding in the per-frame inverse:
-    even one computed exactly in fp32 is off by ~3e-5 relative there, and the
-    fused path's block inverse, whose products take bf16 hi/lo splits
-    (~2^-17), leaves the boundary states ~3e-3 off (measured). The guard
-    sits just above that; the well-conditioned workloads keep 1e-4."""
-    return 5e-3 if getattr(w, "near_dup", False) else STATE_GUARD
+    cond(I + A_t) ~ 1e2-2e2, which magnifies rounding in the per-frame
+    inverse: the Schur complement S = R - Q^T P^{-1} Q is much smaller than R
+    there, so the two products that form it take fp16 hi/lo splits (~2^-22),
+    and an inverse computed exactly in fp32 is already off by ~3e-5 relative.
+    The boundary states then sit ~1.3e-4 from the oracle (measured on the
+    batched workload; ~3e-3 when those products took bf16 splits), and the
+    guard is 5e-4; the well-conditioned workloads keep 1e-4."""
+    return 5e-4 if getattr(w, "near_dup", False) else STATE_GUARD
 
 
 def tdtype(w):
