@@ -638,12 +638,13 @@ def stage_work(w):
 
 def intermediate_bytes(w):
     """HBM bytes a streaming stage moves beyond its algorithmic operands, per
-    launch: the Gram kernel writes B_t and (tensor path) rows 64.. of A_t plus
-    the 16 KB P^{-1} tile of its sweep warps (both A_t halves on the CUDA-core
-    path); the readout reads two fp32 states per chunk."""
+    launch: the Gram kernel writes B_t and (tensor path) the 64 x 64 block R
+    of A_t plus what its sweep pairs form for the block inverse (P^{-1} and
+    X^T, 64 x 64 fp32 each, and the 36 x 64 values of S); both A_t halves on
+    the CUDA-core path; the readout reads two fp32 states per chunk."""
     BH, T, d, C = w.B * w.H, w.T, w.d, w.C
     tensor_path = w.dtype == "bf16" and d == 128
-    gram = (d * d * 4 + d * d * 4 // 2 + 16384) if tensor_path else 2 * d * d * 4
+    gram = (d * d * 4 + 3 * 64 * 64 * 4 + 36 * 64 * 4) if tensor_path else 2 * d * d * 4
     return {"frame_grams": BH * T * gram, "chunk_readout": BH * C * 2 * d * d * 4}
 
 

@@ -123,25 +123,26 @@ size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
 
 // ----------------------------------------------------------- stage calls
-// Pimg (tensor path): also write each frame's P^{-1} tile for the block inverse
+// Pinv (tensor path): also form each frame's P^{-1}, X^T and S for the block
+// inverse (schur.cuh)
 vdn_status run_grams(const Geo &g, const void *K, const void *V, const float *beta, float *A,
                      float *Bm, long long nframes, int U, int32_t *info, cudaStream_t st,
-                     uint8_t *Pimg = nullptr, long long frame_base = 0, int spare_sms = 0) {
+                     float *Pinv = nullptr, long long frame_base = 0, int spare_sms = 0) {
   if (nframes <= 0) return VDN_OK;
   const size_t bytes = (size_t)nframes * g.D * g.D * sizeof(float);
   if (U == 0) {
     VDN_CUDA(cudaMemsetAsync(A, 0, bytes, st), "memset A");
     VDN_CUDA(cudaMemsetAsync(Bm, 0, bytes, st), "memset Bm");
-    if (Pimg) VDN_CUDA(launch_psweep(A, Pimg, info, nframes, st, frame_base), "P sweep");
+    if (Pinv) VDN_CUDA(launch_schur_prep(A, Pinv, info, nframes, st, frame_base), "Schur step");
     return VDN_OK;
   }
   if (gram_tc_supported(g.in_dtype, g.D, U)) {
-    VDN_CUDA(launch_gram_tc(K, V, beta, g.tokb != 0, A, Bm, nframes, U, info, st, Pimg, frame_base, spare_sms),
+    VDN_CUDA(launch_gram_tc(K, V, beta, g.tokb != 0, A, Bm, nframes, U, info, st, Pinv, frame_base, spare_sms),
              "gram_tc");
   } else {
     VDN_CUDA(launch_gram_simt(K, V, g.in_dtype, beta, g.tokb != 0, A, Bm, nframes, U, g.D, st),
              "gram_simt");
-    if (Pimg) VDN_CUDA(launch_psweep(A, Pimg, info, nframes, st, frame_base), "P sweep");
+    if (Pinv) VDN_CUDA(launch_schur_prep(A, Pinv, info, nframes, st, frame_base), "Schur step");
   }
   return VDN_OK;
 }
@@ -462,7 +463,7 @@ vdn_status vdn_frame_invert(const vdn_shape *s, const float *A, float *W, int32_
 
 namespace {
 struct FwdLayout {
-  size_t text, st, a, b, wimg, pimg, mf, jf, mb, jb, mimg, f, g, total;
+  size_t text, st, a, b, wimg, pinv, mf, jf, mb, jb, mimg, f, g, total;
 };
 FwdLayout fwd_layout(const Geo &g) {
   FwdLayout L{};
@@ -479,7 +480,7 @@ FwdLayout fwd_layout(const Geo &g) {
   L.a = take(g.BH * g.T * dd);
   L.b = take(g.BH * g.T * dd);
   L.wimg = take(tc ? (size_t)g.BH * g.T * kImgBytes : 0);
-  L.pimg = take(tc ? (size_t)g.BH * g.T * kPTileBytes : 0);
+  L.pinv = take(tc ? (size_t)g.BH * g.T * kPinvBytes : 0);
   L.mf = take(g.BH * g.C * dd);
   L.jf = take(g.BH * g.C * dd);
   L.mb = take(g.BH * g.C * dd);
@@ -554,12 +555,12 @@ vdn_status vdn_forward(const vdn_shape *s, const void *Q, const void *K, const v
   VDN_CUDA(cudaMemsetAsync(info, 0, sizeof(int32_t), st), "memset info");
   VDN_TRY(run_text_state(g, Kx, Vx, beta_x, S_T, w + L.text, info, st));
   VDN_TRY(mark(1));
-  uint8_t *Pimg = tc ? (uint8_t *)(w + L.pimg) : nullptr;
-  if (frames) VDN_TRY(run_grams(g, K, V, beta, A, Bm, g.BH * g.T, g.U, info, st, Pimg));
+  float *Pinv = tc ? (float *)(w + L.pinv) : nullptr;
+  if (frames) VDN_TRY(run_grams(g, K, V, beta, A, Bm, g.BH * g.T, g.U, info, st, Pinv));
   VDN_TRY(mark(2));
   if (frames) {
     if (tc) {
-      VDN_CUDA(launch_invert_tc(A, nullptr, Wimg, info, g.BH * g.T, st, 0, Pimg), "invert");
+      VDN_CUDA(launch_invert_tc(A, Pinv, nullptr, Wimg, info, g.BH * g.T, st, 0), "invert");
     } else {
       // M and J overwrite A and Bm in place (each element is read and
       // written by the same thread).
@@ -644,10 +645,10 @@ vdn_status stream_segment(const vdn_shape *s, const void *Q, const void *K, cons
   const bool tc = tensor_path(g);
   VDN_CUDA(cudaMemsetAsync(info, 0, sizeof(int32_t), st), "memset info");
   if (frames) {
-    uint8_t *Pimg = tc ? (uint8_t *)(w + L.pimg) : nullptr;
-    VDN_TRY(run_grams(g, K, V, beta, A, Bm, g.BH * g.T, g.U, info, st, Pimg));
+    float *Pinv = tc ? (float *)(w + L.pinv) : nullptr;
+    VDN_TRY(run_grams(g, K, V, beta, A, Bm, g.BH * g.T, g.U, info, st, Pinv));
     if (tc) {
-      VDN_CUDA(launch_invert_tc(A, nullptr, Wimg, info, g.BH * g.T, st, 0, Pimg), "invert");
+      VDN_CUDA(launch_invert_tc(A, Pinv, nullptr, Wimg, info, g.BH * g.T, st, 0), "invert");
       VDN_CUDA(launch_compose_tc(Wimg, Bm, alpha, nullptr, Jf, nullptr, nullptr, Mimg, g.BH, g.T, g.chunk,
                                  g.anchors, 1, true, info, st),
                "compose");
@@ -733,7 +734,7 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
   float *S_T = (float *)(w + L.st);
   float *A = (float *)(w + L.a), *Bm = (float *)(w + L.b);
   uint8_t *Wimg = (uint8_t *)(w + L.wimg), *Mimg = (uint8_t *)(w + L.mimg);
-  uint8_t *Pimg = (uint8_t *)(w + L.pimg);
+  float *Pinv = (float *)(w + L.pinv);
   float *Jf = (float *)(w + L.jf), *Jb = (float *)(w + L.jb);
   float *Fo = F ? F : (float *)(w + L.f);
   float *Go = G ? G : (float *)(w + L.g);
@@ -749,8 +750,8 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
   VDN_CUDA(cudaEventRecord(ev(1), ax), "event record");
   VDN_TRY(run_text_state(g, Kx, Vx, beta_x, S_T, w + L.text, info, ax));
   VDN_CUDA(cudaEventRecord(ev(2), ax), "event record");
-  // the Grams of every group on the main stream (their kernel also writes the
-  // P^{-1} tiles of the block inverse). Their persistent grid leaves some SMs
+  // the Grams of every group on the main stream (their kernel also forms the
+  // block inverse's P^{-1}, X^T and S). Their persistent grid leaves some SMs
   // to the text state: its kernels need TMEM, which a Gram CTA takes whole.
   const int spare = g.n_text > 0 ? (int)(g.BH < device_sm_count() / 12 ? g.BH : device_sm_count() / 12) : 0;
   for (int gi = 0; gi < groups; ++gi) {
@@ -758,17 +759,17 @@ vdn_status vdn_forward_pipelined(const vdn_shape *s, const void *Q, const void *
     const long long b0 = run ? lo(gi) : 0, nbh = run ? lo(gi + 1) - b0 : 0;
     if (run)
       VDN_TRY(run_grams(g, tok(K, b0), tok(V, b0), beta + b0 * T * (g.tokb ? U : 1), A + b0 * T * DD,
-                        Bm + b0 * T * DD, nbh * T, (int)U, info, st, Pimg + b0 * T * kPTileBytes, b0 * T, spare));
+                        Bm + b0 * T * DD, nbh * T, (int)U, info, st, Pinv + b0 * T * (kPinvBytes / 4), b0 * T, spare));
     VDN_CUDA(cudaEventRecord(ev(3 + gi), st), "event record");
   }
   // the rest of the inverse, the composition, the scans and the readout over
-  // all pairs once the auxiliary stream (text state and every P sweep) is
-  // done: these are latency-bound chains whose time grows if they are split
+  // all pairs once the auxiliary stream (the text state) is done: these are
+  // latency-bound chains whose time grows if they are split
   const int tail = 3 + groups;
   VDN_CUDA(cudaStreamWaitEvent(st, ev(2), 0), "stream wait");
   VDN_CUDA(cudaEventRecord(ev(tail), st), "event record");
   if (frames)
-    VDN_CUDA(launch_invert_tc(A, nullptr, Wimg, info, g.BH * g.T, st, 0, Pimg), "invert");
+    VDN_CUDA(launch_invert_tc(A, Pinv, nullptr, Wimg, info, g.BH * g.T, st, 0), "invert");
   VDN_CUDA(cudaEventRecord(ev(tail + 1), st), "event record");
   if (frames)
     VDN_CUDA(launch_compose_tc(Wimg, Bm, alpha, nullptr, Jf, nullptr, Jb, Mimg, g.BH, g.T, g.chunk, g.anchors,

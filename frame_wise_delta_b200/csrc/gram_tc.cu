@@ -23,17 +23,20 @@
 //   warps 2..5 : epilogue: TMEM -> registers -> fp32 stores
 //   warps 6..9 : (per-token gates) the scaled K tile of each stage, or
 //                (PSW) two pairs of sweep warps: each takes every other frame's
-//                leading 64 x 64 block of I + A_t, which the epilogue stages in
-//                shared memory, and writes its inverse P^{-1} as the hi/lo tile
-//                the block inverse reads (so the CUDA-core sweeps run beside the
-//                HBM-bound stream instead of after it); A_t is then written
-//                from row 64 on only, the rows the block inverse reads
+//                leading 64 x 64 block P of I + A_t, which the epilogue stages
+//                in shared memory, sweeps it, and forms P^{-1}, X^T = Q^T P^{-1}
+//                and the Schur complement S = R - Q^T X (schur.cuh) from the
+//                rows 64..127 of A_t that the epilogue writes, so the CUDA-core
+//                half of the block inverse runs beside the HBM-bound stream
+//                instead of after it; rows 0..63 of A_t are then not written
+//                (X^T and S take their place)
 // TMEM holds two 256-column accumulators so a frame's epilogue overlaps the
 // next frame's MMAs. Every wait is bounded (see common.cuh).
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
 #include "internal.h"
+#include "schur.cuh"
 #include "sweep.cuh"
 
 namespace vdn {
@@ -44,13 +47,13 @@ constexpr int kUT = 64;                          // tokens per pipeline stage
 constexpr int kStagesMax = 4;
 constexpr int kBlockBytes = kUT * 128;           // one 64-channel block
 constexpr uint32_t kTmemCols = 512;
-constexpr int kBarBytes = 8 * (3 * kStagesMax + 2 + 2 + 1 + 4);
-// PSW: per sweep pair an fp32 staging of P (64 rows of 65 floats: no bank
-// conflicts for the sweep's loads), a hi/lo tile for the bulk store, and the
-// pair's exchange vector
-constexpr int kPStage = 64 * 65 * 4;
-constexpr int kPTile = 16384;
-constexpr int kPSmem = 2 * (kPStage + kPTile + 2 * 64 * 4);
+constexpr int kPairs = 3;  // PSW: sweep pairs, each taking every kPairs-th frame
+constexpr int kBarBytes = 8 * (3 * kStagesMax + 2 + 2 + 1 + 2 * kPairs);
+// PSW: per sweep pair an fp32 staging of P (it then holds P^{-1}, then X^T)
+// and one of Q^T, both in schur.cuh's layout, and the pair's exchange vector
+constexpr int kPStage = kSchurBytes;
+constexpr int kPTile = kSchurBytes;
+constexpr int kPSmem = kPairs * (kPStage + kPTile + 2 * 64 * 4);
 // per stage: the K and V blocks of channels 0..63 and 64..127 (+ the scaled
 // K blocks: hi part of both, then lo part of both)
 template <bool TOKB> constexpr int kStagesT = TOKB ? 3 : 4;
@@ -67,7 +70,7 @@ struct GramArgs {
   long long nframes;
   int ntiles;
   int U;
-  uint8_t *Pimg;          // PSW: [nframes] P^{-1} tiles
+  float *Pinv;            // PSW: [nframes] P^{-1} (64 x 64 fp32, schur.cuh layout)
   long long frame_base;   // PSW: frame index of frame 0 for *info
 };
 
@@ -77,7 +80,7 @@ __device__ __forceinline__ void fail(volatile int *abort, int32_t *info) {
 }
 
 template <bool TOKB, bool PSW>
-__global__ void __launch_bounds__((TOKB || PSW) ? 320 : 192, 1)
+__global__ void __launch_bounds__(TOKB ? 320 : PSW ? 192 + 64 * kPairs : 192, 1)
     gram_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    GramArgs p) {
   static_assert(!(TOKB && PSW), "one use of warps 6..9");
@@ -88,9 +91,9 @@ __global__ void __launch_bounds__((TOKB || PSW) ? 320 : 192, 1)
                                               ~uintptr_t(1023));
   uint8_t *stages = smem;
   uint8_t *pmem = smem + kStages * kStageBytes;  // PSW area
-  float *pstage = reinterpret_cast<float *>(pmem);                        // [2][64][65]
-  uint8_t *ptile = pmem + 2 * kPStage;                                    // [2][16 KB]
-  float *pcbuf = reinterpret_cast<float *>(pmem + 2 * kPStage + 2 * kPTile);  // [2][2][64]
+  float *pstage = reinterpret_cast<float *>(pmem);                               // [kPairs][16 KB] P
+  uint8_t *ptile = pmem + kPairs * kPStage;                                      // [kPairs][16 KB] Q^T
+  float *pcbuf = reinterpret_cast<float *>(pmem + kPairs * (kPStage + kPTile));  // [kPairs][2][64]
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * kStageBytes + (PSW ? kPSmem : 0));
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(bars) + kBarBytes);
   volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -103,7 +106,7 @@ __global__ void __launch_bounds__((TOKB || PSW) ? 320 : 192, 1)
   const uint32_t drain = tempty0 + 16;
   const uint32_t scaled0 = drain + 8;  // per stage: the scaled K tile is written
   const uint32_t pready0 = scaled0 + 8 * kStagesMax;  // PSW, per pair: P staged (128 arrivals)
-  const uint32_t pfree0 = pready0 + 16;               // PSW, per pair: staging read (64 arrivals)
+  const uint32_t pfree0 = pready0 + 8 * kPairs;       // PSW, per pair: stagings free (64 arrivals)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -118,7 +121,7 @@ __global__ void __launch_bounds__((TOKB || PSW) ? 320 : 192, 1)
     if (TOKB)
       for (int s = 0; s < kStages; ++s) mbar_init(scaled0 + 8 * s, 128);
     if (PSW)
-      for (int q = 0; q < 2; ++q) {
+      for (int q = 0; q < kPairs; ++q) {
         mbar_init(pready0 + 8 * q, 128);
         mbar_init(pfree0 + 8 * q, 64);
       }
@@ -262,19 +265,19 @@ __global__ void __launch_bounds__((TOKB || PSW) ? 320 : 192, 1)
       }
     }
   } else if (PSW && warp >= 6) {
-    // a sweep pair (warps 6-7 or 8-9): every other frame of this CTA
+    // sweep pair pq (warps 6 + 2 pq, 7 + 2 pq): every kPairs-th frame of this CTA
     const int pq = (warp - 6) >> 1;
     const int st = threadIdx.x - 192 - 64 * pq;  // 0..63
     const int rg = st / kSweepGrid, cg = st % kSweepGrid;
     const int nb = 3 + pq;  // the pair's named barrier
-    const float *ps = pstage + pq * (64 * 65);
-    uint8_t *pt = ptile + pq * kPTile;
+    float *ps = pstage + pq * (kPStage / 4);
+    const float *qs = reinterpret_cast<const float *>(ptile + pq * kPTile);
     float(*cb)[64] = reinterpret_cast<float(*)[64]>(pcbuf + pq * 128);
     bool okw = true;
     int it = 0;
     for (long long f = blockIdx.x; f < p.nframes; f += gridDim.x, ++it) {
-      if ((it & 1) != pq) continue;
-      if (okw && !mbar_wait(pready0 + 8 * pq, (uint32_t)(it >> 1) & 1, abort)) {
+      if (it % kPairs != pq) continue;
+      if (okw && !mbar_wait(pready0 + 8 * pq, (uint32_t)(it / kPairs) & 1, abort)) {
         fail(abort, p.info);
         okw = false;
       }
@@ -282,21 +285,17 @@ __global__ void __launch_bounds__((TOKB || PSW) ? 320 : 192, 1)
 #pragma unroll
       for (int a = 0; a < Sweep<64>::R; ++a)
 #pragma unroll
-        for (int b = 0; b <= a; ++b) X.at(a, b) = ps[(rg + kSweepGrid * a) * 65 + cg + kSweepGrid * b];
-      mbar_arrive(pfree0 + 8 * pq);  // the staging may take the pair's next frame
-      const bool ok = X.run(cb, rg, cg, [nb] { asm volatile("bar.sync %0, 64;" ::"r"(nb) : "memory"); });
-      if (st == 0) bulk_wait_read<0>();  // the previous P^{-1} tile has left
-      asm volatile("bar.sync %0, 64;" ::"r"(nb) : "memory");
-      store_swept_tile<true>(X, pt, rg, cg);
-      fence_proxy_async_smem();
-      asm volatile("bar.sync %0, 64;" ::"r"(nb) : "memory");
-      if (st == 0) {
-        bulk_store(p.Pimg + f * (long long)kPTile, smem_u32(pt), kPTile);
-        bulk_commit();
-        if (!ok) report_frame_failure(p.info, p.frame_base + f);
-      }
+        for (int b = 0; b <= a; ++b) X.at(a, b) = ps[swz64(rg + kSweepGrid * a, cg + kSweepGrid * b)];
+      auto sync = [nb] { asm volatile("bar.sync %0, 64;" ::"r"(nb) : "memory"); };
+      const bool ok = X.run(cb, rg, cg, sync);
+      if (st == 0 && !ok) report_frame_failure(p.info, p.frame_base + f);
+      // P^{-1}, then X^T, replace P in its staging; both stagings are
+      // released to the epilogue (for the pair's next frame) at the end
+      float *Af = p.A + f * (long long)(kD * kD);
+      schur_prep(X, qs, Af + 64 * kD + 64, ps, p.Pinv + f * 64LL * 64, Af + kSchurXT, Af + kSchurS, st, sync);
+      mbar_arrive(pfree0 + 8 * pq);
     }
-    if (st == 0) bulk_wait_all();
+    if (st == 0) bulk_wait_all();  // the P^{-1} and X^T copies have landed
   } else {
     // epilogue warps 2..5 -> TMEM sub-partitions 2, 3, 0, 1
     const int sub = warp & 3;
@@ -305,11 +304,13 @@ __global__ void __launch_bounds__((TOKB || PSW) ? 320 : 192, 1)
     for (long long f = blockIdx.x; f < p.nframes; f += gridDim.x, ++it) {
       const int buf = it & 1;
       const uint32_t use = (uint32_t)(it >> 1);
-      const int pq = it & 1;  // PSW: the sweep pair of this frame
-      float *ps = pstage + pq * (64 * 65);
-      if (PSW && row < 64 && use > 0) {
-        // the pair has read its staging of two frames ago
-        if (!mbar_wait(pfree0 + 8 * pq, (use - 1) & 1, abort)) fail(abort, p.info);
+      const int pq = it % kPairs;  // PSW: the sweep pair of this frame
+      const uint32_t puse = (uint32_t)(it / kPairs);
+      float *ps = pstage + pq * (kPStage / 4);
+      float *qs = reinterpret_cast<float *>(ptile + pq * kPTile);
+      if (PSW && puse > 0) {
+        // the pair is done with its stagings of kPairs frames ago
+        if (!mbar_wait(pfree0 + 8 * pq, (puse - 1) & 1, abort)) fail(abort, p.info);
       }
       // every lane waits (acquire); the warp then agrees on the outcome so
       // that it enters the aligned TMEM loads together or not at all
@@ -330,16 +331,30 @@ __global__ void __launch_bounds__((TOKB || PSW) ? 320 : 192, 1)
         // column so that a warp stores 32 consecutive floats); n >= 128 ->
         // B[n-128][row].
         float *dst = (cc < 4 ? Af + (cc * 32) * kD : Bf + ((cc - 4) * 32) * kD) + row;
-        // PSW: rows 0..63 of A (P and Q^T's transpose) are not read after
-        // this kernel (P is swept here, the block inverse reads rows 64..127)
-        if (!(PSW && cc < 2)) {
+        // PSW: P and Q^T are staged for the sweep pair instead of written;
+        // of rows 64..127 only R (columns 64..127) is written, and the pair
+        // puts X^T and S in rows 0..63
+        if (!(PSW && (cc < 2 || (cc < 4 && row < 64)))) {
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) dst[jj * kD] = bt * v[jj];
         }
         if (PSW && cc < 2 && row < 64) {
           // P = I + A[0..63][0..63] for the sweep pair (A symmetric: row `row`)
 #pragma unroll
-          for (int jj = 0; jj < 32; ++jj) ps[row * 65 + cc * 32 + jj] = bt * v[jj] + (row == cc * 32 + jj ? 1.f : 0.f);
+          for (int c4 = 0; c4 < 8; ++c4) {
+            const int c0 = cc * 32 + 4 * c4;
+            *reinterpret_cast<float4 *>(ps + swz64(row, c0)) =
+                make_float4(bt * v[4 * c4] + (row == c0 ? 1.f : 0.f), bt * v[4 * c4 + 1] + (row == c0 + 1 ? 1.f : 0.f),
+                            bt * v[4 * c4 + 2] + (row == c0 + 2 ? 1.f : 0.f),
+                            bt * v[4 * c4 + 3] + (row == c0 + 3 ? 1.f : 0.f));
+          }
+        }
+        if (PSW && cc < 2 && row >= 64) {
+          // Q^T: row row - 64, columns 32 cc .. + 31
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4)
+            *reinterpret_cast<float4 *>(qs + swz64(row - 64, cc * 32 + 4 * c4)) =
+                make_float4(bt * v[4 * c4], bt * v[4 * c4 + 1], bt * v[4 * c4 + 2], bt * v[4 * c4 + 3]);
         }
       }
       tc_fence_before();
@@ -385,26 +400,26 @@ cudaError_t launch_gram_t(const CUtensorMap &tmK, const CUtensorMap &tmV, const 
   int sms = device_sm_count() - spare_sms;
   if (sms < 1) sms = 1;
   const long long grid = a.nframes < sms ? a.nframes : sms;
-  gram_tc_kernel<TOKB, PSW><<<(unsigned)grid, (TOKB || PSW) ? 320 : 192, smem, st>>>(tmK, tmV, a);
+  gram_tc_kernel<TOKB, PSW><<<(unsigned)grid, TOKB ? 320 : PSW ? 192 + 64 * kPairs : 192, smem, st>>>(tmK, tmV, a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gram_tc(const void *K, const void *V, const float *beta, bool per_token, float *A,
-                           float *Bm, long long nframes, int U, int32_t *info, cudaStream_t st, uint8_t *Pimg,
+                           float *Bm, long long nframes, int U, int32_t *info, cudaStream_t st, float *Pinv,
                            long long frame_base, int spare_sms) {
   if (nframes <= 0) return cudaSuccess;
   CUtensorMap tmK, tmV;
   if (!make_rows_map(&tmK, K, nframes, U, kUT) || !make_rows_map(&tmV, V, nframes, U, kUT))
     return cudaErrorInvalidValue;
-  GramArgs a{A, Bm, beta, info, nframes, (U + kUT - 1) / kUT, U, Pimg, frame_base};
+  GramArgs a{A, Bm, beta, info, nframes, (U + kUT - 1) / kUT, U, Pinv, frame_base};
   if (per_token) {
-    // the per-token stages use warps 6..9 and most of shared memory: the
-    // P^{-1} tiles then come from their own kernel
+    // the per-token stages use warps 6..9 and most of shared memory: P^{-1},
+    // X^T and S then come from their own kernel
     cudaError_t e = launch_gram_t<true, false>(tmK, tmV, a, st, spare_sms);
-    if (e != cudaSuccess || !Pimg) return e;
-    return launch_psweep(A, Pimg, info, nframes, st, frame_base);
+    if (e != cudaSuccess || !Pinv) return e;
+    return launch_schur_prep(A, Pinv, info, nframes, st, frame_base);
   }
-  return Pimg ? launch_gram_t<false, true>(tmK, tmV, a, st, spare_sms)
+  return Pinv ? launch_gram_t<false, true>(tmK, tmV, a, st, spare_sms)
               : launch_gram_t<false, false>(tmK, tmV, a, st, spare_sms);
 }
 

@@ -52,13 +52,14 @@ cudaError_t launch_bridge_tail(const float *alpha, float *out, long long BH, int
 
 // Tensor-core kernels (tcgen05 + TMA), bf16 inputs, d = 128.
 bool gram_tc_supported(int in_dtype, int D, int U);
-// Pimg: null, or where to write each frame's P^{-1} tile (the leading 64 x 64
-// block of I + A inverted, as launch_psweep does), swept beside the stream;
-// then only rows 64..127 of A are written (all the block inverse reads).
+// Pinv: null, or where to write each frame's P^{-1} (the leading 64 x 64
+// block of I + A inverted): the sweep pairs then also form X^T and the Schur
+// complement S (schur.cuh, as launch_schur_prep does) beside the stream, in
+// rows 0..63 of each frame of A.
 // spare_sms: SMs the persistent grid leaves free for a concurrent stream.
 cudaError_t launch_gram_tc(const void *K, const void *V, const float *beta, bool per_token, float *A,
                            float *Bm, long long nframes, int U, int32_t *info, cudaStream_t st,
-                           uint8_t *Pimg = nullptr, long long frame_base = 0, int spare_sms = 0);
+                           float *Pinv = nullptr, long long frame_base = 0, int spare_sms = 0);
 bool readout_tc_supported(int in_dtype, int out_dtype, int D, int U);
 cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, void *O, long long BH,
                               int T, int U, int chunk, int anchors, int32_t *info, cudaStream_t st,
@@ -68,20 +69,23 @@ cudaError_t launch_readout_tc(const void *Q, const float *F, const float *G, voi
 // W = (I + A)^{-1} per frame (CUDA cores); W fp32 and/or Wimg (hi/lo MMA
 // images of kImgBytes per frame, d = 128 only), each optional.
 // frame_base: index of the first frame, for the failure index in *info.
-// (I + A)^{-1} of fp32 128 x 128 frames by the tensor-core block inverse, as
-// fp32 row-major W and/or hi/lo MMA images (either may be null)
-// Pimg: null, or the P^{-1} tiles of launch_psweep (then the kernel skips its P sweeps)
-cudaError_t launch_invert_tc(const float *A, float *W, uint8_t *Wimg, int32_t *info, long long nframes,
-                             cudaStream_t st, long long frame_base = 0, const uint8_t *Pimg = nullptr);
+// (I + A)^{-1} of 128 x 128 frames by the tensor-core block inverse, from the
+// P^{-1}, X^T and S that launch_schur_prep (or the Gram kernel's sweep pairs)
+// left in Pinv and A, as fp32 row-major W and/or hi/lo MMA images (either
+// may be null)
+cudaError_t launch_invert_tc(const float *A, const float *Pinv, float *W, uint8_t *Wimg, int32_t *info,
+                             long long nframes, cudaStream_t st, long long frame_base = 0);
 // (I + A)^{-1} of fp32 128 x 128 frames by the blocked symmetric sweep with
 // tensor-core updates, as fp32 row-major W and/or hi/lo MMA images (either
 // may be null). A must be symmetric: the kernel reads its columns as rows.
 cudaError_t launch_invert_bsweep(const float *A, float *W, uint8_t *Wimg, int32_t *info, long long nframes,
                                  cudaStream_t st, long long frame_base);
-// P^{-1} (leading 64 x 64 block of I + A) of every frame as a 16 KB hi/lo tile
-constexpr long long kPTileBytes = 16384;
-cudaError_t launch_psweep(const float *A, uint8_t *Pimg, int32_t *info, long long nframes, cudaStream_t st,
-                          long long frame_base = 0);
+// P^{-1} (leading 64 x 64 block of I + A, 16 KB fp32) of every frame into
+// Pinv, and X^T = Q^T P^{-1} and the Schur complement S into rows 0..63 of
+// each frame of A (schur.cuh), from a full fp32 A
+constexpr long long kPinvBytes = 16384;
+cudaError_t launch_schur_prep(float *A, float *Pinv, int32_t *info, long long nframes, cudaStream_t st,
+                              long long frame_base = 0);
 cudaError_t launch_invert_simt(const float *A, float *W, uint8_t *Wimg, int32_t *info,
                                long long nframes, int D, cudaStream_t st, long long frame_base = 0);
 // Chunk maps from W images (tensor cores, d = 128): per (direction, b*h,

@@ -1,5 +1,5 @@
 // W_t = (I + A_t)^{-1} for every frame (d = 128), as a 2 x 2 block inverse
-// whose four 64 x 64 x 64 products run on the tensor cores.
+// whose last three 64 x 64 x 64 products run on the tensor cores.
 // Paper: "Video DeltaNet: A Video-Native Hybrid Attention for Livestream
 // Video Generation" (summary page), "Core method" (the closed form
 // S_t = (Sbar_t + B_t)(I + A_t)^{-1}) and "Method steps" step (3) (factor
@@ -9,26 +9,28 @@
 // definite) the Schur complement S = R - Q^T P^{-1} Q is positive definite too
 // and, with X = P^{-1} Q and Y = X S^{-1},
 //   G^{-1} = [[P^{-1} + Y X^T, -Y], [-Y^T, S^{-1}]].
-// P^{-1} and S^{-1} come from the symmetric sweep on the CUDA cores (a quarter
-// of the full sweep's work); the products X^T = Q^T P^{-1}, Q^T X, Y = X S^{-1},
-// Y^T = S^{-1} X^T and Y X^T run as tcgen05 MMAs (M = 128, N = 64, K = 64) on
-// hi/lo splits (hi*hi + hi*lo + lo*hi), accumulating in TMEM. The two products
-// that form S take fp16 parts (~2^-22 of each operand): when I + A is
-// ill-conditioned S is much smaller than R and Q^T X, and the subtraction
-// magnifies their error. The last three take bf16 parts (~2^-17), the format
-// of the output image: their results are at most 2 in norm and meet no such
-// cancellation. A pivot of P or S that is not positive (G not positive definite) is
-// reported in *info like the sweep does.
+// P^{-1}, X^T and S arrive in fp32 from the step in schur.cuh (run beside the
+// Gram stream, or by schur_prep_kernel below). This kernel sweeps S on the
+// CUDA cores (symmetric sweep) and runs Y = X S^{-1}, Y^T = S^{-1} X^T and
+// Y X^T as tcgen05 MMAs (M = 128, N = 64, K = 64) on bf16 hi/lo splits
+// (hi*hi + hi*lo + lo*hi, ~2^-17 of each operand: these results are at most 2
+// in norm and involve no cancellation), accumulating in TMEM. A pivot of S
+// that is not positive (G not positive definite) is reported in *info like
+// the sweep does.
 //
 // One CTA of 128 threads works through frames (persistent), four CTAs per SM:
-// warps 0-1 run the sweeps, warps 2-3 own TMEM lanes 64-127 and do the loads,
-// the epilogues and the output; thread 64 issues the MMAs. The two pairs are
-// one frame apart where they can be (named-barrier hand-offs).
+//   warps 0-1 (sweep): load S, sweep it, write the S^{-1} tile -> (SiReady)
+//   warps 2-3 (epilogue, TMEM lanes 64-127; thread 64 issues the MMAs):
+//            X^T tile from the fp32 rows -> [SiReady] -> Y, Y^T -> Y X^T ->
+//            the image's four blocks -> (SiFree)
+// The sweep of frame f + 1 runs while the epilogue finishes frame f; only
+// the S^{-1} tile's slot is handed back and forth (named barriers).
 // Every product keeps its 64 useful rows in lanes 64-127: the A operand's
 // descriptor starts 64 rows (8 KB) before the useful rows, so lanes 0-63
 // compute throw-away rows from whatever shared memory lies there.
 #include "common.cuh"
 #include "internal.h"
+#include "schur.cuh"
 #include "sweep.cuh"
 
 namespace vdn {
@@ -39,47 +41,32 @@ constexpr int kCtasPerSm = 4;          // x 128 TMEM columns <= 512
 constexpr int kHalf = 64 * 128;         // one 64 x 64 bf16 tile, 128-byte rows: 8 KB
 constexpr int kTile = 2 * kHalf;        // hi + lo: 16 KB
 // shared memory slots (offsets from the 1024-aligned base)
-constexpr int kSlotPi = 0;              // P^{-1} image
-constexpr int kSlotS0 = kTile;          // Q^T image -> fp32 Q^T X staging -> S^{-1} image -> Y image
-constexpr int kSlotXT = 2 * kTile;      // X^T image
+constexpr int kSlotTL = 0;              // top-left block of the image
+constexpr int kSlotS0 = kTile;          // S^{-1} tile -> -Y tile
+constexpr int kSlotXT = 2 * kTile;      // X^T tile -> bottom-left block of the image
 constexpr int kSlotMisc = 3 * kTile;    // sweep exchange buffer, barrier, TMEM address, abort flag
 constexpr size_t kSmemBytes = 1024 + kSlotMisc + 2 * 2 * 64 * 4 + 64;
 constexpr uint32_t kTmemCols = 128;     // two 64-column accumulators
-// X^T = Q^T P^{-1} and Q^T X multiply fp16 hi/lo tiles (A, B K-major); the
-// products after the S sweep multiply bf16 hi/lo tiles (one operand MN-major)
-constexpr uint32_t kIdescF16 = idesc_f16_f32(128, 64, false, false);
-constexpr uint32_t kIdescAmn = idesc_bf16_f32(128, 64, true, false);
-constexpr uint32_t kIdescBmn = idesc_bf16_f32(128, 64, false, true);
-
-// element (row, k) of a 64-row K-major 128-byte-swizzled tile (k < 64)
-__device__ __forceinline__ uint32_t tile_off(int row, int k) { return kmajor_sw128_offset(row, k, 64); }
+constexpr uint32_t kIdescAmn = idesc_bf16_f32(128, 64, true, false);  // A MN-major
+constexpr uint32_t kIdescBmn = idesc_bf16_f32(128, 64, false, true);  // B MN-major
 
 // physical 16-byte chunk of logical chunk c in row r (both tile and image layouts)
 __device__ __forceinline__ uint32_t chunk_pos(int r, int c) { return (uint32_t)((c ^ (r & 7)) << 4); }
 
 // hi and lo 16-byte chunks of 8 values (times sign)
-template <bool F16>
 __device__ __forceinline__ void pack8(const float *v, float sign, uint4 &h, uint4 &l) {
-  if constexpr (F16) {
-    split_f16x2(sign * v[0], sign * v[1], h.x, l.x);
-    split_f16x2(sign * v[2], sign * v[3], h.y, l.y);
-    split_f16x2(sign * v[4], sign * v[5], h.z, l.z);
-    split_f16x2(sign * v[6], sign * v[7], h.w, l.w);
-  } else {
-    split_bf16x2(sign * v[0], sign * v[1], h.x, l.x);
-    split_bf16x2(sign * v[2], sign * v[3], h.y, l.y);
-    split_bf16x2(sign * v[4], sign * v[5], h.z, l.z);
-    split_bf16x2(sign * v[6], sign * v[7], h.w, l.w);
-  }
+  split_bf16x2(sign * v[0], sign * v[1], h.x, l.x);
+  split_bf16x2(sign * v[2], sign * v[3], h.y, l.y);
+  split_bf16x2(sign * v[4], sign * v[5], h.z, l.z);
+  split_bf16x2(sign * v[6], sign * v[7], h.w, l.w);
 }
 
 // Row r of a hi/lo tile (64 values) written from one thread.
-template <bool F16>
 __device__ __forceinline__ void tile_row_store(uint8_t *tile, int r, const float *v, float sign) {
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     uint4 h, l;
-    pack8<F16>(v + 8 * c, sign, h, l);
+    pack8(v + 8 * c, sign, h, l);
     const uint32_t o = (uint32_t)r * 128u + chunk_pos(r, c);
     *reinterpret_cast<uint4 *>(tile + o) = h;
     *reinterpret_cast<uint4 *>(tile + kHalf + o) = l;
@@ -116,19 +103,11 @@ __device__ __forceinline__ void handoff_arrive(int id) {
 __device__ __forceinline__ void handoff_wait(int id) {
   asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
 }
-constexpr int kBarSweep = 1, kBarEpi = 2;           // within each warp pair
-constexpr int kBarPiReady = 3, kBarTReady = 4, kBarSiReady = 5, kBarPiFree = 6;
+constexpr int kBarSweep = 1, kBarEpi = 2;  // within each warp pair
+constexpr int kBarSiReady = 3, kBarSiFree = 4;
 
-// the two values of a bf16x2 or fp16x2 word as fp32
-template <bool F16>
-__device__ __forceinline__ float2 unpack2(uint32_t w) {
-  if constexpr (F16) return __half22float2(*reinterpret_cast<const __half2 *>(&w));
-  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-}
-
-// v (+)= row r of a hi/lo tile (fp16 or bf16 parts), decoded to fp32
-template <bool F16>
-__device__ __forceinline__ void tile_row_add(const uint8_t *tile, int r, float (&v)[64], bool add) {
+// v = row r of a bf16 hi/lo tile, decoded to fp32
+__device__ __forceinline__ void tile_row_load(const uint8_t *tile, int r, float (&v)[64]) {
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     const uint32_t o = (uint32_t)r * 128u + chunk_pos(r, c);
@@ -137,11 +116,21 @@ __device__ __forceinline__ void tile_row_add(const uint8_t *tile, int r, float (
     const uint32_t hw[4] = {h.x, h.y, h.z, h.w}, lw[4] = {l.x, l.y, l.z, l.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float2 hh = unpack2<F16>(hw[q]), ll = unpack2<F16>(lw[q]);
-      const float x0 = hh.x + ll.x, x1 = hh.y + ll.y;
-      v[8 * c + 2 * q] = add ? v[8 * c + 2 * q] + x0 : x0;
-      v[8 * c + 2 * q + 1] = add ? v[8 * c + 2 * q + 1] + x1 : x1;
+      v[8 * c + 2 * q] = __uint_as_float(hw[q] << 16) + __uint_as_float(lw[q] << 16);
+      v[8 * c + 2 * q + 1] = __uint_as_float(hw[q] & 0xFFFF0000u) + __uint_as_float(lw[q] & 0xFFFF0000u);
     }
+  }
+}
+
+// v (+)= row r of a 64 x 64 fp32 block in schur.cuh's permuted-chunk layout
+__device__ __forceinline__ void block_row_load(const float *blk, int r, float (&v)[64], bool add) {
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const float4 x = __ldg(reinterpret_cast<const float4 *>(blk + r * 64 + ((c ^ (r & 15)) << 2)));
+    v[4 * c] = add ? v[4 * c] + x.x : x.x;
+    v[4 * c + 1] = add ? v[4 * c + 1] + x.y : x.y;
+    v[4 * c + 2] = add ? v[4 * c + 2] + x.z : x.z;
+    v[4 * c + 3] = add ? v[4 * c + 3] + x.w : x.w;
   }
 }
 
@@ -165,55 +154,55 @@ __device__ __forceinline__ void fail(volatile int *abort, int32_t *info) {
   if (info) atomicExch(info, VDN_INFO_TIMEOUT);
 }
 
-// P^{-1} of every frame as a hi/lo tile in global memory (16 KB per frame,
-// the layout of the kernel below's P^{-1} slot), by the same sweep: lets the
-// block inverse skip its own P sweeps.
-__global__ void __launch_bounds__(kSweepThreads) psweep_kernel(const float *__restrict__ A, uint8_t *__restrict__ Pimg,
-                                                               int32_t *__restrict__ info, long long frame_base) {
-  __shared__ __align__(1024) uint8_t tile[kTile];
+// P^{-1}, X^T and S of every frame (schur.cuh) from a full A, one CTA of 64
+// threads per frame: for Grams computed without the sweep pairs (per-token
+// gates, no tokens, CUDA-core Grams).
+__global__ void __launch_bounds__(kSweepThreads) schur_prep_kernel(float *__restrict__ A, float *__restrict__ Pinv,
+                                                                   int32_t *__restrict__ info, long long frame_base) {
+  __shared__ __align__(16) float bp[64 * 64];
+  __shared__ __align__(16) float qs[64 * 64];
   __shared__ __align__(16) float cbuf[2][64];
   const long long f = blockIdx.x;
   const int tid = threadIdx.x, rg = tid / kSweepGrid, cg = tid % kSweepGrid;
-  const float *Af = A + f * 128LL * 128;
+  float *Af = A + f * 128LL * 128;
   Sweep<64> X;
+  // P = I + A[0..63][0..63]; rows 0..63 of A then receive X^T and S
 #pragma unroll
   for (int a = 0; a < Sweep<64>::R; ++a)
 #pragma unroll
     for (int b = 0; b <= a; ++b) {
       const int r = rg + kSweepGrid * a, c = cg + kSweepGrid * b;
-      X.at(a, b) = __ldg(Af + r * 128 + c) + (r == c ? 1.f : 0.f);
+      X.at(a, b) = Af[r * 128 + c] + (r == c ? 1.f : 0.f);
     }
-  const bool ok = X.run(cbuf, rg, cg, [] { __syncthreads(); });
-  store_swept_tile<true>(X, tile, rg, cg);
-  fence_proxy_async_smem();
-  __syncthreads();
-  if (tid == 0) {
-    bulk_store(Pimg + f * (long long)kTile, smem_u32(tile), kTile);
-    bulk_commit();
-    bulk_wait_all();
-    if (!ok) report_frame_failure(info, frame_base + f);
+  // Q^T (rows 64..127, columns 0..63) into shared memory
+#pragma unroll
+  for (int it = 0; it < 16; ++it) {
+    const int r = it * 4 + (tid >> 4), c4 = tid & 15;
+    *reinterpret_cast<float4 *>(qs + swz64(r, 4 * c4)) =
+        *reinterpret_cast<const float4 *>(Af + (64 + r) * 128 + 4 * c4);
   }
+  auto sync = [] { __syncthreads(); };
+  const bool ok = X.run(cbuf, rg, cg, sync);  // its barriers also publish qs
+  if (!ok && tid == 0) report_frame_failure(info, frame_base + f);
+  schur_prep(X, qs, Af + 64 * 128 + 64, bp, Pinv + f * 64LL * 64, Af + kSchurXT, Af + kSchurS, tid, sync);
+  if (tid == 0) bulk_wait_all();
 }
 
-// PRE_P: the P^{-1} tiles come from psweep_kernel (Pimg) instead of the sweep warps.
-template <bool PRE_P>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    invert_tc_kernel(const float *__restrict__ A, float *__restrict__ W, uint8_t *__restrict__ Wimg,
-                     int32_t *__restrict__ info, long long nframes, long long frame_base,
-                     const uint8_t *__restrict__ Pimg) {
+    invert_tc_kernel(const float *__restrict__ A, const float *__restrict__ Pinv, float *__restrict__ W,
+                     uint8_t *__restrict__ Wimg, int32_t *__restrict__ info, long long nframes,
+                     long long frame_base) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *pi_t = sm + kSlotPi, *s0 = sm + kSlotS0, *xt = sm + kSlotXT;
+  uint8_t *tl_t = sm + kSlotTL, *s0 = sm + kSlotS0, *xt = sm + kSlotXT;
   float(*cbuf)[64] = reinterpret_cast<float(*)[64]>(sm + kSlotMisc);  // sweep exchange buffer
   uint64_t *bar = reinterpret_cast<uint64_t *>(sm + kSlotMisc + 1024);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kSlotMisc + 1032);
   volatile int *abort = reinterpret_cast<volatile int *>(sm + kSlotMisc + 1036);
-  const uint32_t pbar = smem_u32(sm + kSlotMisc + 1040);  // (PRE_P) the P^{-1} tile has landed
   const int tid = threadIdx.x, warp = tid >> 5;
   const uint32_t mbar = smem_u32(bar);
   if (tid == 0) {
     mbar_init(mbar, 1);
-    mbar_init(pbar, 1);
     *abort = 0;
     fence_barrier_init();
   }
@@ -222,57 +211,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   __syncthreads();
   tc_fence_after();
   const uint32_t acc0 = *tmem_slot, acc1 = acc0 + 64;
-  float *stage = reinterpret_cast<float *>(s0);  // fp32 Q^T X, rows with swizzled 16-byte chunks
 
-  // The two warp pairs run their own loops over the same frames and meet at
-  // the hand-off barriers, so that the sweep of frame f + 1's P overlaps the
-  // last products and the output of frame f:
-  //   sweep warps:    P sweep -> [P^{-1} free] -> P^{-1} tile -> (PiReady)
-  //                   [TReady] -> S sweep -> S^{-1} tile -> (SiReady)
-  //   epilogue warps: Q^T tile -> [PiReady] -> X^T -> Q^T X staged -> (TReady)
-  //                   [SiReady] -> Y, Y^T -> Y X^T -> (P^{-1} free) -> output
   if (tid < 64) {
     const int rg = tid / kSweepGrid, cg = tid % kSweepGrid;
     bool first = true;
     for (long long f = blockIdx.x; f < nframes; f += gridDim.x) {
-      const float *Af = A + f * 128LL * 128;
+      const float *Sf = A + f * 128LL * 128 + kSchurS;
       Sweep<64> X;
-      bool ok = true;
-      if constexpr (!PRE_P) {
-#pragma unroll
-        for (int a = 0; a < Sweep<64>::R; ++a)
-#pragma unroll
-          for (int b = 0; b <= a; ++b) {
-            const int r = rg + kSweepGrid * a, c = cg + kSweepGrid * b;
-            X.at(a, b) = __ldg(Af + r * 128 + c) + (r == c ? 1.f : 0.f);
-          }
-        ok = X.run(cbuf, rg, cg, [] { bar_named(kBarSweep); });
-        if (!first) handoff_wait(kBarPiFree);  // the previous frame's last product has read P^{-1}
-        first = false;
-        store_swept_tile<true>(X, pi_t, rg, cg);
-        fence_proxy_async_smem();
-        handoff_arrive(kBarPiReady);
-      }
-      // S = R - Q^T X and S^{-1} by the sweep; S^{-1} replaces the staging
-      // (every thread has read its part before the sweep's first barrier).
-      // R + I is read while the epilogue warps still compute Q^T X.
 #pragma unroll
       for (int a = 0; a < Sweep<64>::R; ++a)
 #pragma unroll
-        for (int b = 0; b <= a; ++b) {
-          const int r = rg + kSweepGrid * a, c = cg + kSweepGrid * b;
-          X.at(a, b) = __ldg(Af + (64 + r) * 128 + 64 + c) + (r == c ? 1.f : 0.f);
-        }
-      handoff_wait(kBarTReady);
-#pragma unroll
-      for (int a = 0; a < Sweep<64>::R; ++a)
-#pragma unroll
-        for (int b = 0; b <= a; ++b) {
-          const int r = rg + kSweepGrid * a, c = cg + kSweepGrid * b;
-          X.at(a, b) -= stage[r * 64 + (((c >> 2) ^ (r & 15)) << 2) + (c & 3)];
-        }
-      ok = X.run(cbuf, rg, cg, [] { bar_named(kBarSweep); }) && ok;
-      store_swept_tile<false>(X, s0, rg, cg);
+        for (int b = 0; b <= a; ++b) X.at(a, b) = __ldg(Sf + (a * (a + 1) / 2 + b) * 64 + tid);
+      const bool ok = X.run(cbuf, rg, cg, [] { bar_named(kBarSweep); });
+      // the epilogue is done with the previous frame's S^{-1} and -Y tiles
+      if (!first) handoff_wait(kBarSiFree);
+      first = false;
+      store_swept_tile(X, s0, rg, cg);
       fence_proxy_async_smem();
       handoff_arrive(kBarSiReady);
       if (!ok && tid == 0) report_frame_failure(info, frame_base + f);
@@ -280,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   } else {
     const int i = tid - 64;  // TMEM lane 64 + i, row i of every product
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t a_pi = smem_u32(pi_t), a_s0 = smem_u32(s0), a_xt = smem_u32(xt);
+    const uint32_t a_tl = smem_u32(tl_t), a_s0 = smem_u32(s0), a_xt = smem_u32(xt);
     uint32_t nwait = 0;
     auto wait_mma = [&]() {
       if (!mbar_wait(mbar, nwait & 1, abort)) fail(abort, info);
@@ -294,68 +248,25 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         tc_commit(mbar);
       }
     };
-    uint32_t puse = 0;
     for (long long f = blockIdx.x; f < nframes; f += gridDim.x) {
       const float *Af = A + f * 128LL * 128;
+      const float *Pf = Pinv + f * 64LL * 64;
       uint8_t *img = Wimg ? Wimg + f * (long long)kImgBytes : nullptr;
       float *Wf = W ? W + f * 128LL * 128 : nullptr;
-      if (PRE_P && i == 0) {
-        // the P^{-1} slot is free (the last frame's output copies have read it)
-        mbar_arrive_expect_tx(pbar, kTile);
-        bulk_load(a_pi, Pimg + f * (long long)kTile, kTile, pbar);
-      }
-      // Q^T = G[64 + r][0 .. 63] as a hi/lo tile, read row-contiguously (all
-      // loads in flight at once)
-#pragma unroll
-      for (int it = 0; it < 16; ++it) {
-        const int r = it * 4 + (i >> 4), c4 = i & 15;
-        const float4 x = __ldg(reinterpret_cast<const float4 *>(Af + (64 + r) * 128 + 4 * c4));
-        uint2 h, l;
-        split_f16x2(x.x, x.y, h.x, l.x);
-        split_f16x2(x.z, x.w, h.y, l.y);
-        const uint32_t o = tile_off(r, 4 * c4);
-        *reinterpret_cast<uint2 *>(s0 + o) = h;
-        *reinterpret_cast<uint2 *>(s0 + kHalf + o) = l;
-      }
-      fence_proxy_async_smem();
-      if constexpr (PRE_P) {
-        if (!mbar_wait(pbar, puse & 1, abort)) fail(abort, info);
-        ++puse;
-        bar_named(kBarEpi);  // every epilogue thread's Q^T rows are written
-      } else {
-        handoff_wait(kBarPiReady);
-      }
-      // X^T = Q^T P^{-1}
-      issue([&] { mma_hilo(acc0, a_s0 - kHalf, a_s0, a_pi, a_pi + kHalf, false, false, 16, kIdescF16); });
+      // the X^T tile from its fp32 rows (the previous frame's output copies
+      // have read the slot)
       float v[64];
-      wait_mma();
-      tmem_row64(acc0 + lane_off, v);
-      tile_row_store<true>(xt, i, v, 1.f);
+      block_row_load(Af + kSchurXT, i, v, false);
+      tile_row_store(xt, i, v, 1.f);
       fence_proxy_async_smem();
-      tc_fence_before();
-      bar_named(kBarEpi);
-      // Q^T X (B = Q read from the Q^T tile K-major), staged in fp32 for the S sweep
-      issue([&] { mma_hilo(acc0, a_xt - kHalf, a_xt, a_s0, a_s0 + kHalf, false, false, 16, kIdescF16); });
-      wait_mma();
-      tmem_row64(acc0 + lane_off, v);
-#pragma unroll
-      for (int c = 0; c < 16; ++c)
-        *reinterpret_cast<float4 *>(stage + i * 64 + ((c ^ (i & 15)) << 2)) =
-            make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-      tc_fence_before();
-      handoff_arrive(kBarTReady);
-      // while the S sweep runs: the next frame's rows 64..127 of A (Q^T and
-      // R) into L2, so its Q^T tile and S assembly read them from there
       if (i == 0 && f + gridDim.x < nframes) {
-        bulk_prefetch_l2(Af + gridDim.x * 128LL * 128 + 64 * 128, 64 * 128 * 4);
-        if (PRE_P) bulk_prefetch_l2(Pimg + (f + gridDim.x) * (long long)kTile, kTile);
+        // the next frame's inputs into L2 while this one is finished
+        const float *An = Af + gridDim.x * 128LL * 128;
+        bulk_prefetch_l2(An + kSchurXT, kSchurBytes);
+        bulk_prefetch_l2(An + kSchurS, kSchurSPerThread * 64 * 4);
+        bulk_prefetch_l2(Pf + gridDim.x * 64LL * 64, kSchurBytes);
       }
-      // the X^T tile in bf16 parts for the products after the sweep (its
-      // fp16 form has served the two products the Schur complement needs)
-      tile_row_add<true>(xt, i, v, false);
-      tile_row_store<false>(xt, i, v, 1.f);
-      fence_proxy_async_smem();
-      handoff_wait(kBarSiReady);
+      handoff_wait(kBarSiReady);  // the S^{-1} tile is written; so is every row of X^T
       issue([&] {
         // Y = X S^{-1}: A = X, the X^T tile read MN-major as the second 64-row
         // block (lanes 64-127) of a descriptor that starts one tile earlier
@@ -368,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       if (Wf) {
         w_row_store(Wf, 1, i, v, -1.f);  // top-right block: -Y
         float u[64];
-        tile_row_add<false>(s0, i, u, false);
+        tile_row_load(s0, i, u);
         w_row_store(Wf, 1, 64 + i, u, 1.f);  // bottom-right block: S^{-1}
       }
       // The image is written as four 64 x 64 blocks by bulk copies of the
@@ -381,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         bulk_wait_read<0>();
       }
       bar_named(kBarEpi);  // the S^{-1} tile has been read; it becomes -Y
-      tile_row_store<false>(s0, i, v, -1.f);  // -Y: the top-right block and A of the last product
+      tile_row_store(s0, i, v, -1.f);  // -Y: the top-right block and A of the last product
       fence_proxy_async_smem();
       tc_fence_before();
       bar_named(kBarEpi);
@@ -394,29 +305,29 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       }
       wait_mma();
       tmem_row64(acc0 + lane_off, v);
-      // top-left block: P^{-1} - (-Y) X^T, written over this row of the P^{-1} tile
+      // top-left block: P^{-1} - (-Y) X^T
 #pragma unroll
       for (int e = 0; e < 64; ++e) v[e] = -v[e];
-      tile_row_add<true>(pi_t, i, v, true);
-      tile_row_store<false>(pi_t, i, v, 1.f);
+      block_row_load(Pf, i, v, true);
+      tile_row_store(tl_t, i, v, 1.f);
       if (Wf) w_row_store(Wf, 0, i, v, 1.f);
       // bottom-left block: -Y^T, into the X^T tile (the last product is done)
       tmem_row64(acc1 + lane_off, v);
-      tile_row_store<false>(xt, i, v, -1.f);
+      tile_row_store(xt, i, v, -1.f);
       if (Wf) w_row_store(Wf, 0, 64 + i, v, -1.f);
       fence_proxy_async_smem();
       bar_named(kBarEpi);
       if (img && i == 0) {
-        bulk_store(img, a_pi, kHalf);
-        bulk_store(img + kImgHalf, a_pi + kHalf, kHalf);
+        bulk_store(img, a_tl, kHalf);
+        bulk_store(img + kImgHalf, a_tl + kHalf, kHalf);
         bulk_store(img + 64 * 128, a_xt, kHalf);
         bulk_store(img + kImgHalf + 64 * 128, a_xt + kHalf, kHalf);
         bulk_commit();
-        bulk_wait_read<0>();  // the P^{-1}, X^T and -Y tiles may be reused
+        bulk_wait_read<0>();  // the top-left, X^T and -Y tiles may be reused
       }
       bar_named(kBarEpi);
-      // the sweep warps may now write the next frame's P^{-1} tile
-      if (!PRE_P && f + gridDim.x < nframes) handoff_arrive(kBarPiFree);
+      // the sweep warps may now write the next frame's S^{-1} tile
+      if (f + gridDim.x < nframes) handoff_arrive(kBarSiFree);
       tc_fence_before();
     }
   }
@@ -430,22 +341,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
 }  // namespace
 
-cudaError_t launch_invert_tc(const float *A, float *W, uint8_t *Wimg, int32_t *info, long long nframes,
-                             cudaStream_t st, long long frame_base, const uint8_t *Pimg) {
+cudaError_t launch_invert_tc(const float *A, const float *Pinv, float *W, uint8_t *Wimg, int32_t *info,
+                             long long nframes, cudaStream_t st, long long frame_base) {
   if (nframes <= 0) return cudaSuccess;
-  auto kern = Pimg ? invert_tc_kernel<true> : invert_tc_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  if (!A || !Pinv) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(invert_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   const long long cap = (long long)kCtasPerSm * device_sm_count();
   const long long grid = nframes < cap ? nframes : cap;
-  kern<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(A, W, Wimg, info, nframes, frame_base, Pimg);
+  invert_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(A, Pinv, W, Wimg, info, nframes, frame_base);
   return cudaGetLastError();
 }
 
-cudaError_t launch_psweep(const float *A, uint8_t *Pimg, int32_t *info, long long nframes, cudaStream_t st,
-                          long long frame_base) {
+cudaError_t launch_schur_prep(float *A, float *Pinv, int32_t *info, long long nframes, cudaStream_t st,
+                              long long frame_base) {
   if (nframes <= 0) return cudaSuccess;
-  psweep_kernel<<<(unsigned)nframes, kSweepThreads, 0, st>>>(A, Pimg, info, frame_base);
+  schur_prep_kernel<<<(unsigned)nframes, kSweepThreads, 0, st>>>(A, Pinv, info, frame_base);
   return cudaGetLastError();
 }
 

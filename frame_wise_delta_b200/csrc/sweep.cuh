@@ -198,12 +198,9 @@ struct Sweep {
   }
 };
 
-// -G^{-1} of a 64 x 64 block from the sweep, stored as the hi/lo tile of
+// -G^{-1} of a 64 x 64 block from the sweep, stored as the bf16 hi/lo tile of
 // G^{-1} (both triangles; 64 rows of 128 bytes per part, K-major with the
-// 128-byte swizzle, hi part then lo part 8 KB later) that the tensor cores read
-// as an operand: fp16 parts (F16, ~2^-22 of each value; the inverses of the
-// blocks of I + A are at most 1 in norm) or bf16 parts (~2^-17).
-template <bool F16>
+// 128-byte swizzle, hi part then lo part 8 KB later) that the tensor cores read.
 __device__ __forceinline__ void store_swept_tile(Sweep<64> &X, uint8_t *tile, int rg, int cg) {
   constexpr int kPart = 64 * 128;
 #pragma unroll
@@ -211,24 +208,14 @@ __device__ __forceinline__ void store_swept_tile(Sweep<64> &X, uint8_t *tile, in
 #pragma unroll
     for (int b = 0; b <= a; ++b) {
       const int i = rg + kSweepGrid * a, j = cg + kSweepGrid * b;
-      const float x = -X.at(a, b);
-      uint16_t h, l;
-      if constexpr (F16) {
-        const __half hh = __float2half_rn(x);
-        h = __half_as_ushort(hh);
-        l = __half_as_ushort(__float2half_rn(x - __half2float(hh)));
-      } else {
-        __nv_bfloat16 hh, ll;
-        split_bf16(x, hh, ll);
-        h = __bfloat16_as_ushort(hh);
-        l = __bfloat16_as_ushort(ll);
-      }
+      __nv_bfloat16 h, l;
+      split_bf16(-X.at(a, b), h, l);
       const uint32_t oij = kmajor_sw128_offset(i, j, 64), oji = kmajor_sw128_offset(j, i, 64);
-      *reinterpret_cast<uint16_t *>(tile + oij) = h;
-      *reinterpret_cast<uint16_t *>(tile + kPart + oij) = l;
+      *reinterpret_cast<__nv_bfloat16 *>(tile + oij) = h;
+      *reinterpret_cast<__nv_bfloat16 *>(tile + kPart + oij) = l;
       if (a != b) {
-        *reinterpret_cast<uint16_t *>(tile + oji) = h;
-        *reinterpret_cast<uint16_t *>(tile + kPart + oji) = l;
+        *reinterpret_cast<__nv_bfloat16 *>(tile + oji) = h;
+        *reinterpret_cast<__nv_bfloat16 *>(tile + kPart + oji) = l;
       }
     }
 }

@@ -45,7 +45,7 @@ def test_roofline_of_the_dominant_stage(bench):
     assert r["achieved"] == pytest.approx(kv / 0.25e-3 / 1e9)
     assert r["frac"] == pytest.approx(r["achieved"] / 6531.9)
     # what the kernel writes beyond that is reported beside it, not counted in it
-    assert r["intermediate_bytes"] == frames * (128 * 128 * 4 + 128 * 128 * 4 // 2 + 16384)
+    assert r["intermediate_bytes"] == frames * (128 * 128 * 4 + 3 * 64 * 64 * 4 + 36 * 64 * 4)
     # the traffic record is reported while its kernel source is the one it was taken on
     rec = bench.NCU_TRAFFIC["frame_grams"]
     with open(os.path.join(ROOT, rec["source"]), "rb") as f:
