@@ -37,10 +37,10 @@ ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # the frames a full launch processes (x6): the traffic of these kernels grows
 # in proportion to the frames they stream.
 NCU_TRAFFIC = {
-    "frame_grams": {"bytes": 6 * (214.5e6 + 25.3e6), "source": "frame_wise_delta_b200/csrc/gram_tc.cu",
-                    "sha256_16": "00240b7db02fd61b", "workload": "h3", "capture": "h3 with 4 heads, x6"},
-    "chunk_readout": {"bytes": 6 * (118.8e6 + 58.1e6), "source": "frame_wise_delta_b200/csrc/readout_tc.cu",
-                      "sha256_16": "9a564eca14ecfc6e", "workload": "h3", "capture": "h3 with 4 heads, x6"},
+    "frame_grams": {"bytes": 6 * (212.71e6 + 21.12e6), "source": "frame_wise_delta_b200/csrc/gram_tc.cu",
+                    "sha256_16": "73b57c89dc3adf04", "workload": "h3", "capture": "h3 with 4 heads, x6"},
+    "chunk_readout": {"bytes": 6 * (118.99e6 + 56.81e6), "source": "frame_wise_delta_b200/csrc/readout_tc.cu",
+                      "sha256_16": "a4185e26db062a56", "workload": "h3", "capture": "h3 with 4 heads, x6"},
 }
 
 
