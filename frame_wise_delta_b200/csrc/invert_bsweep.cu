@@ -11,9 +11,10 @@
 //
 // This kernel serves the text state and the stage call vdn_frame_invert:
 // every frame's whole inverse in one CTA, lower latency per frame than the
-// block inverse (which needs its leading block swept elsewhere) and fp16
+// block inverse (which needs its first half formed elsewhere) and fp16
 // splits in every product. The fused frame path keeps the block inverse,
-// whose leading-block sweeps run inside the Gram kernel beside the HBM stream.
+// whose first half (P^{-1}, X^T and the Schur complement) the Gram kernel's
+// sweep pairs form beside the HBM stream.
 //
 // Sweeping the pivot block K (indices k0 .. k0 + 31) of a symmetric G maps
 //   G_KK -> -G_KK^{-1},   G_iK -> G_iK G_KK^{-1} = c_i,   G_Kj -> c_j^T,

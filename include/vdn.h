@@ -138,10 +138,12 @@ vdn_status vdn_frame_factor(const vdn_shape *s, const float *A, const float *Bm,
  * is produced directly, without a separate solve pipeline).
  * In : A [B,H,T,dk,dk] float32.  Out: W [B,H,T,dk,dk] float32.
  * *info is reset to 0 and then set as for vdn_frame_factor.
- * Shapes of the fused tensor-core pass (bf16 in/out, d = 128) use its kernel:
- * a 2 x 2 block inverse whose products run on the tensor cores in split bf16
- * (about fp32 accuracy, relative error ~1e-5); other shapes use the fp32
- * symmetric sweep on the CUDA cores.
+ * Shapes of the fused tensor-core pass (bf16 in/out, d = 128) use the blocked
+ * symmetric sweep with the matrix in tensor memory, its rank-32 updates on
+ * the tensor cores in split fp16 (about fp32 accuracy, relative error ~1e-6);
+ * other shapes use the fp32 symmetric sweep on the CUDA cores. (The fused
+ * passes themselves form the frames' inverses as a 2 x 2 block inverse whose
+ * first half runs inside the Gram kernel.)
  */
 vdn_status vdn_frame_invert(const vdn_shape *s, const float *A, float *W,
                             int32_t *info, vdn_stream_t stream);

@@ -25,11 +25,11 @@ def state_guard(w) -> float:
     """The state guard of a workload. Near-duplicate keys (cosine 0.99) make
     cond(I + A_t) ~ 1e2-2e2, which magnifies rounding in the per-frame
     inverse: the Schur complement S = R - Q^T P^{-1} Q is much smaller than R
-    there, so the two products that form it take fp16 hi/lo splits (~2^-22),
-    and an inverse computed exactly in fp32 is already off by ~3e-5 relative.
-    The boundary states then sit ~1.3e-4 from the oracle (measured on the
-    batched workload; ~3e-3 when those products took bf16 splits), and the
-    guard is 5e-4; the well-conditioned workloads keep 1e-4."""
+    there, so it is formed in fp32 on the CUDA cores, and an inverse computed
+    exactly in fp32 is already off by ~3e-5 relative. The boundary states
+    then sit ~1.1e-4 from the oracle (measured on the batched workload; ~3e-3
+    when the products forming S took bf16 hi/lo splits on the tensor cores),
+    and the guard is 5e-4; the well-conditioned workloads keep 1e-4."""
     return 5e-4 if getattr(w, "near_dup", False) else STATE_GUARD
 
 
