@@ -318,6 +318,25 @@ def test_nonpositive_pivot_is_reported_by_block_invert():
     assert rel(W[0, 0], ref) <= 1e-4
 
 
+@pytest.mark.parametrize("w", [TC_SMALL, TC_TB], ids=lambda w: w.name)
+def test_fused_pass_reports_an_indefinite_frame(w):
+    # a negative write gate makes I + A_t indefinite for one frame: the fused
+    # tensor-core pass sweeps its leading block (in the Gram kernel's sweep
+    # pairs, or the separate Schur step with per-token gates) and then its
+    # Schur complement, and reports that frame in *info (frame index + 1)
+    full = _full(w)
+    b, h, t = w.B - 1, w.H - 1, 4
+    full["beta"] = np.array(full["beta"], copy=True)
+    full["beta"][b, h, t] = -2.0
+    dev = device_inputs(w, full)
+    fw = run_forward(w, dev)
+    assert int(fw.info.item()) == 1 + (b * w.H + h) * w.T + t
+    # the same inputs with the gate restored pass
+    full["beta"][b, h, t] = 0.5
+    fw = run_forward(w, device_inputs(w, full))
+    assert int(fw.info.item()) == 0
+
+
 def test_nonpositive_pivot_is_reported():
     w = custom("poison", index=46, dtype="f32", d=16, T=9, anchors=0)
     full = _full(w)
